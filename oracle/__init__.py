@@ -1,0 +1,184 @@
+"""CPU oracle for the BitLinear forward -- TEST INFRASTRUCTURE ONLY.
+
+Loads the plain single-threaded C++ oracle (bitnet_oracle.cpp, built into
+liboracle.so beside this file) and wraps it for numpy arrays.  Only the
+tests, the smoke check and the CPU-baseline leg of the benchmark use it; the
+CUDA library never imports or links it.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bitnet_oracle.cpp")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_CXXFLAGS = ["-std=c++17", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so with g++ (IEEE fp32, no contraction) if stale."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["g++", *_CXXFLAGS, _SRC, "-o", tmp])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        F = ctypes.c_float
+        L.oracle_absmean_gamma.argtypes = [P, I64, I64]
+        L.oracle_absmean_gamma.restype = F
+        L.oracle_ternarize.argtypes = [P, I64, I64, F, P, P]
+        L.oracle_ternarize.restype = ctypes.c_int
+        L.oracle_pack_codes.argtypes = [P, I64, I64, P]
+        L.oracle_pack_codes.restype = None
+        L.oracle_unpack_codes.argtypes = [P, I64, I64, P]
+        L.oracle_unpack_codes.restype = I64
+        L.oracle_pack_weights.argtypes = [P, I64, I64, F, P, P]
+        L.oracle_pack_weights.restype = ctypes.c_int
+        L.oracle_rmsnorm_row.argtypes = [P, P, I64, F, P]
+        L.oracle_rmsnorm_row.restype = None
+        L.oracle_quant_act.argtypes = [P, I64, I64, P, F, P, P, P]
+        L.oracle_quant_act.restype = None
+        L.oracle_dot.argtypes = [P, P, I64, F, F, P, P]
+        L.oracle_dot.restype = ctypes.c_int
+        L.oracle_bitlinear.argtypes = [P, F, I64, I64, P, P, I64, P, P]
+        L.oracle_bitlinear.restype = ctypes.c_int
+        L.oracle_bitlinear_sampled.argtypes = [P, F, I64, I64, P, P, I64, P, P, I64, P, P]
+        L.oracle_bitlinear_sampled.restype = ctypes.c_int
+        L.oracle_f32_to_bf16.argtypes = [P, I64, P]
+        L.oracle_f32_to_bf16.restype = None
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags.c_contiguous
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f32(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def absmean_gamma(W: np.ndarray) -> np.float32:
+    W = _f32(W)
+    N, K = W.shape
+    return np.float32(lib().oracle_absmean_gamma(_p(W), N, K))
+
+
+def ternarize(W: np.ndarray, eps: float):
+    """Returns (q int8 N x K, gamma float32).  Raises on non-finite W."""
+    W = _f32(W)
+    N, K = W.shape
+    q = np.empty((N, K), dtype=np.int8)
+    g = np.zeros(1, dtype=np.float32)
+    st = lib().oracle_ternarize(_p(W), N, K, eps, _p(q), _p(g))
+    if st != 0:
+        raise ValueError(f"oracle_ternarize status {st}")
+    return q, g[0]
+
+
+def pack_codes(q: np.ndarray) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    N, K = q.shape
+    out = np.empty((N, K // 4), dtype=np.uint8)
+    lib().oracle_pack_codes(_p(q), N, K, _p(out))
+    return out
+
+
+def unpack_codes(packed: np.ndarray, K: int):
+    """Returns (q int8 N x K, number of illegal code-3 fields)."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    N = packed.shape[0]
+    q = np.empty((N, K), dtype=np.int8)
+    bad = lib().oracle_unpack_codes(_p(packed), N, K, _p(q))
+    return q, int(bad)
+
+
+def pack_weights(W: np.ndarray, eps: float):
+    """Returns (packed uint8 N x K/4, gamma float32), or raises on non-finite W."""
+    W = _f32(W)
+    N, K = W.shape
+    out = np.empty((N, K // 4), dtype=np.uint8)
+    g = np.zeros(1, dtype=np.float32)
+    st = lib().oracle_pack_weights(_p(W), N, K, eps, _p(out), _p(g))
+    if st != 0:
+        raise ValueError(f"oracle_pack_weights status {st}")
+    return out, g[0]
+
+
+def rmsnorm_row(v: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
+    v = _f32(v)
+    g = _f32(g)
+    h = np.empty_like(v)
+    lib().oracle_rmsnorm_row(_p(v), _p(g), v.shape[0], eps, _p(h))
+    return h
+
+
+def quant_act(x: np.ndarray, gain=None, rms_eps: float = 1e-5):
+    """x: M x K fp32 values.  Returns (x_q int8 M x K, a float32 M, rowsum int32 M)."""
+    x = _f32(x)
+    M, K = x.shape
+    xq = np.empty((M, K), dtype=np.int8)
+    a = np.empty(M, dtype=np.float32)
+    rs = np.empty(M, dtype=np.int32)
+    gp = None
+    if gain is not None:
+        gain = _f32(gain)
+        gp = _p(gain)
+    lib().oracle_quant_act(_p(x), M, K, gp, rms_eps, _p(xq), _p(a), _p(rs))
+    return xq, a, rs
+
+
+def bitlinear(packed: np.ndarray, gamma, K: int, xq: np.ndarray, a: np.ndarray):
+    """Returns (acc int32 M x N, y float32 M x N)."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    xq = np.ascontiguousarray(xq, dtype=np.int8)
+    a = _f32(a)
+    N = packed.shape[0]
+    M = xq.shape[0]
+    acc = np.empty((M, N), dtype=np.int32)
+    y = np.empty((M, N), dtype=np.float32)
+    st = lib().oracle_bitlinear(_p(packed), np.float32(gamma), N, K, _p(xq), _p(a), M, _p(acc), _p(y))
+    if st != 0:
+        raise ValueError(f"oracle_bitlinear status {st}")
+    return acc, y
+
+
+def bitlinear_sampled(packed: np.ndarray, gamma, K: int, xq: np.ndarray, a: np.ndarray,
+                      ms: np.ndarray, ns: np.ndarray):
+    """The product at positions (ms[i], ns[i]) only.  Returns (acc int32, y float32)."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    xq = np.ascontiguousarray(xq, dtype=np.int8)
+    a = _f32(a)
+    ms = np.ascontiguousarray(ms, dtype=np.int64)
+    ns = np.ascontiguousarray(ns, dtype=np.int64)
+    N = packed.shape[0]
+    M = xq.shape[0]
+    acc = np.empty(ms.shape[0], dtype=np.int32)
+    y = np.empty(ms.shape[0], dtype=np.float32)
+    st = lib().oracle_bitlinear_sampled(_p(packed), np.float32(gamma), N, K, _p(xq), _p(a), M,
+                                        _p(ms), _p(ns), ms.shape[0], _p(acc), _p(y))
+    if st != 0:
+        raise ValueError(f"oracle_bitlinear_sampled status {st}")
+    return acc, y
+
+
+def f32_to_bf16(y: np.ndarray) -> np.ndarray:
+    y = _f32(y)
+    out = np.empty(y.shape, dtype=np.uint16)
+    lib().oracle_f32_to_bf16(_p(y), y.size, _p(out))
+    return out
