@@ -1,1 +1,211 @@
-"""BitNet b1.58 BitLinear forward (W1.58A8) for NVIDIA B200 (sm_100a)."""
+"""BitNet b1.58 BitLinear forward (W1.58A8) on NVIDIA B200 (sm_100a).
+
+Python binding of the C ABI in include/bitnet.h.  Every function has the
+name of the C entry point it calls and does argument marshalling only
+(PyTorch tensors -> device pointers, sizes, the current CUDA stream); all of
+the computation runs in the library's CUDA kernels.  There is no CPU path:
+if libbitnet_b200.so is missing or cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbitnet_b200.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "bitnet.h")
+
+BITNET_OK = 0
+BITNET_ERR_INVALID_ARG = 1
+BITNET_ERR_UNSUPPORTED_SHAPE = 2
+BITNET_ERR_NONFINITE = 3
+BITNET_ERR_CUDA = 4
+BITNET_ERR_TIMEOUT = 5
+
+BITNET_F32 = 0
+BITNET_BF16 = 1
+BITNET_I32 = 2
+
+_lib = None
+
+
+class BitnetError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: status {status} ({status_string(status)})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library.  Raises if it is not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing "
+                               "(run python -m bitlinear_absmean_ternary_b200.build)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, F, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int
+        L.bitnet_pack_workspace_bytes.argtypes = [I64, I64]
+        L.bitnet_pack_workspace_bytes.restype = ctypes.c_size_t
+        L.bitnet_pack_weights.argtypes = [P, I64, I64, F, P, P, P, ctypes.c_size_t, P]
+        L.bitnet_pack_weights.restype = I
+        L.bitnet_quant_act.argtypes = [P, I, I64, I64, P, F, P, P, P, P]
+        L.bitnet_quant_act.restype = I
+        for name in ("bitnet_linear_gemv", "bitnet_linear_gemm"):
+            fn = getattr(L, name)
+            fn.argtypes = [P, P, I64, I64, P, P, P, I64, P, I, P]
+            fn.restype = I
+        L.bitnet_get_device_status.argtypes = [P]
+        L.bitnet_get_device_status.restype = I
+        L.bitnet_status_string.argtypes = [I]
+        L.bitnet_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def declared_functions() -> list:
+    """Names of the entry points include/bitnet.h declares."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bitnet_[a-z_]+)\s*\(", text)))
+
+
+def status_string(status: int) -> str:
+    try:
+        return lib().bitnet_status_string(int(status)).decode()
+    except Exception:  # the library itself is unavailable
+        return "unknown"
+
+
+def _check(fn: str, status: int) -> None:
+    if status != BITNET_OK:
+        raise BitnetError(fn, status)
+
+
+# ----------------------------------------------------------------- marshalling
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device) -> int:
+    torch = _torch()
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _dtype_code(dtype) -> int:
+    torch = _torch()
+    if dtype == torch.float32:
+        return BITNET_F32
+    if dtype == torch.bfloat16:
+        return BITNET_BF16
+    if dtype == torch.int32:
+        return BITNET_I32
+    raise ValueError(f"unsupported dtype {dtype}")
+
+
+def _need_cuda(*ts) -> None:
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("tensor must live on a CUDA device")
+            if not t.is_contiguous():
+                raise ValueError("tensor must be contiguous")
+
+
+def bitnet_pack_workspace_bytes(N: int, K: int) -> int:
+    return int(lib().bitnet_pack_workspace_bytes(N, K))
+
+
+def bitnet_pack_weights(W, eps: float = 1e-5, W_packed=None, gamma=None, workspace=None):
+    """Absmean ternarisation + 2-bit packing of fp32 W (N x K) on the GPU.
+
+    Returns (W_packed uint8 N x K/4, gamma float32 [1]).  Synchronises.
+    """
+    torch = _torch()
+    _need_cuda(W)
+    N, K = W.shape
+    if W_packed is None:
+        W_packed = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    if gamma is None:
+        gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    nbytes = bitnet_pack_workspace_bytes(N, K)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    _need_cuda(W_packed, gamma, workspace)
+    st = lib().bitnet_pack_weights(_ptr(W), N, K, eps, _ptr(W_packed), _ptr(gamma), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(W.device))
+    _check("bitnet_pack_weights", st)
+    return W_packed, gamma
+
+
+def bitnet_quant_act(x, rms_gain=None, rms_eps: float = 1e-5, x_q=None, a_scale=None, x_rowsum=None,
+                     want_rowsum: bool = False):
+    """Fused RMSNorm (when rms_gain is given) + per-token absmax int8 quant.
+
+    x: M x K float32 or bfloat16 on the GPU.  Returns (x_q int8, a_scale
+    float32 [M], x_rowsum int32 [M] or None).  Asynchronous.
+    """
+    torch = _torch()
+    _need_cuda(x, rms_gain)
+    M, K = x.shape
+    if x_q is None:
+        x_q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if a_scale is None:
+        a_scale = torch.empty(M, dtype=torch.float32, device=x.device)
+    if x_rowsum is None and want_rowsum:
+        x_rowsum = torch.empty(M, dtype=torch.int32, device=x.device)
+    _need_cuda(x_q, a_scale, x_rowsum)
+    st = lib().bitnet_quant_act(_ptr(x), _dtype_code(x.dtype), M, K, _ptr(rms_gain), rms_eps, _ptr(x_q),
+                                _ptr(a_scale), _ptr(x_rowsum), _stream(x.device))
+    _check("bitnet_quant_act", st)
+    return x_q, a_scale, x_rowsum
+
+
+def _linear(name: str, W_packed, gamma, x_q, a_scale, x_rowsum=None, y=None, out_dtype=None):
+    torch = _torch()
+    _need_cuda(W_packed, gamma, x_q, a_scale, x_rowsum, y)
+    N = W_packed.shape[0]
+    K = W_packed.shape[1] * 4
+    M = x_q.shape[0]
+    if x_q.shape[1] != K:
+        raise ValueError("x_q and W_packed disagree on K")
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype or torch.bfloat16, device=x_q.device)
+    st = getattr(lib(), name)(_ptr(W_packed), _ptr(gamma), N, K, _ptr(x_q), _ptr(a_scale), _ptr(x_rowsum), M,
+                              _ptr(y), _dtype_code(y.dtype), _stream(x_q.device))
+    _check(name, st)
+    return y
+
+
+def bitnet_linear_gemv(W_packed, gamma, x_q, a_scale, x_rowsum=None, y=None, out_dtype=None):
+    """W1.58A8 product for M <= 8 tokens (CUDA cores).  Returns y (M x N)."""
+    return _linear("bitnet_linear_gemv", W_packed, gamma, x_q, a_scale, x_rowsum, y, out_dtype)
+
+
+def bitnet_linear_gemm(W_packed, gamma, x_q, a_scale, x_rowsum=None, y=None, out_dtype=None):
+    """W1.58A8 product for any M (tcgen05 tensor cores).  Returns y (M x N)."""
+    return _linear("bitnet_linear_gemm", W_packed, gamma, x_q, a_scale, x_rowsum, y, out_dtype)
+
+
+def bitnet_get_device_status(device=None) -> int:
+    """Synchronises the current stream and returns (and clears) the device error status."""
+    torch = _torch()
+    dev = device if device is not None else torch.cuda.current_device()
+    return int(lib().bitnet_get_device_status(_stream(dev)))
+
+
+def bitlinear(x, W_packed, gamma, rms_gain=None, rms_eps: float = 1e-5, out_dtype=None):
+    """One BitLinear forward: quantise x (fused RMSNorm when rms_gain is given),
+    then the ternary product with dequant.  Picks the decode kernel for M <= 8."""
+    x_q, a, rs = bitnet_quant_act(x, rms_gain, rms_eps, want_rowsum=True)
+    if x.shape[0] <= 8:
+        return bitnet_linear_gemv(W_packed, gamma, x_q, a, rs, out_dtype=out_dtype)
+    return bitnet_linear_gemm(W_packed, gamma, x_q, a, rs, out_dtype=out_dtype)

@@ -1,0 +1,308 @@
+// Host side of the BitLinear C ABI declared in include/bitnet.h: argument
+// checks, launch configuration and stream-ordered launches.  One translation
+// unit holds every kernel so that the device error word has a single home.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "bitnet.h"
+#include "gemm.cuh"
+#include "gemv.cuh"
+#include "pack.cuh"
+#include "ptx.cuh"
+#include "quant.cuh"
+
+namespace {
+
+using namespace bitnet;
+
+constexpr int kMaxDevices = 64;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool valid_k(int64_t K) { return K >= 64 && K % 64 == 0 && K <= (int64_t{1} << 30); }
+
+int current_device() {
+  int d = 0;
+  cudaGetDevice(&d);
+  return d;
+}
+
+int sm_count() {
+  static int cache[kMaxDevices] = {};
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return 148;
+  if (cache[d] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n <= 0) n = 148;
+    cache[d] = n;
+  }
+  return cache[d];
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory (once per device).
+template <typename F>
+cudaError_t set_smem(F* fn, int bytes, bool (&done)[kMaxDevices]) {
+  const int d = current_device();
+  if (d >= 0 && d < kMaxDevices && done[d]) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && d >= 0 && d < kMaxDevices) done[d] = true;
+  return e;
+}
+
+// Launch with programmatic stream serialisation, so the kernel may start its
+// independent prologue while the previous kernel on the stream finishes; the
+// kernels call griddepcontrol.wait before touching that kernel's outputs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+bitnet_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA; }
+
+// ------------------------------------------------------------ tensor maps
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D byte tensor [rows][cols] with row pitch `pitch` bytes, box {box_cols, box_rows}.
+bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t pitch, uint32_t box_cols,
+                 uint32_t box_rows, CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------ launchers
+
+template <typename T, int MAXC>
+cudaError_t launch_quant_t(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
+                           int32_t* rs, cudaStream_t s) {
+  return launch_pdl(quant_act_kernel<T, MAXC>, dim3(static_cast<unsigned>(M)), dim3(kQuantThreads), 0, s,
+                    static_cast<const T*>(x), K, static_cast<const T*>(gain), eps, xq, a, rs);
+}
+
+template <typename T>
+cudaError_t launch_quant(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
+                         int32_t* rs, cudaStream_t s) {
+  const int per_thread = (K / 8 + kQuantThreads - 1) / kQuantThreads;
+  if (per_thread <= 1) return launch_quant_t<T, 1>(x, M, K, gain, eps, xq, a, rs, s);
+  if (per_thread <= 2) return launch_quant_t<T, 2>(x, M, K, gain, eps, xq, a, rs, s);
+  if (per_thread <= 4) return launch_quant_t<T, 4>(x, M, K, gain, eps, xq, a, rs, s);
+  if (per_thread <= 8) return launch_quant_t<T, 8>(x, M, K, gain, eps, xq, a, rs, s);
+  if constexpr (sizeof(T) == 2) return launch_quant_t<T, 16>(x, M, K, gain, eps, xq, a, rs, s);
+  return cudaErrorInvalidValue;
+}
+
+template <int MT, bool U8>
+cudaError_t launch_gemv_t(const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
+                          const int32_t* rs, void* y, int yd, cudaStream_t s) {
+  static bool done[kMaxDevices] = {};
+  const cudaError_t e = set_smem(gemv_kernel<MT, U8>, kGemvSmemBytes, done);
+  if (e != cudaSuccess) return e;
+  const int64_t groups = (N + kGemvRows - 1) / kGemvRows;
+  const int grid = static_cast<int>(groups < sm_count() ? groups : sm_count());
+  return launch_pdl(gemv_kernel<MT, U8>, dim3(grid), dim3(kGemvWarps * 32), kGemvSmemBytes, s, Wp, gamma, N, K, xq,
+                    a, rs, y, yd);
+}
+
+template <bool U8>
+cudaError_t launch_gemv_u(int M, const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
+                          const int32_t* rs, void* y, int yd, cudaStream_t s) {
+  switch (M) {
+    case 1: return launch_gemv_t<1, U8>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+    case 2: return launch_gemv_t<2, U8>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+    case 3: return launch_gemv_t<3, U8>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+    case 4: return launch_gemv_t<4, U8>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+    case 5: return launch_gemv_t<5, U8>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+    case 6: return launch_gemv_t<6, U8>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+    case 7: return launch_gemv_t<7, U8>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+    case 8: return launch_gemv_t<8, U8>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int BN, int STAGES, bool U8>
+cudaError_t launch_gemm_t(const CUtensorMap& mx, const CUtensorMap& mw, const float* gamma, const float* a,
+                          const int32_t* rs, int M, int N, int K, void* y, int yd, cudaStream_t s) {
+  using C = GemmCfg<BN, STAGES>;
+  static bool done[kMaxDevices] = {};
+  const cudaError_t e = set_smem(gemm_kernel<BN, STAGES, U8>, C::kSmemBytes, done);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((N + kGemmBM - 1) / kGemmBM, (M + BN - 1) / BN);
+  return launch_pdl(gemm_kernel<BN, STAGES, U8>, grid, dim3(kGemmThreads), C::kSmemBytes, s, mx, mw, gamma, a, rs, M,
+                    N, K, y, yd);
+}
+
+template <int BN, int STAGES>
+cudaError_t launch_gemm_bn(const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
+                           const int32_t* rs, int M, void* y, int yd, cudaStream_t s) {
+  CUtensorMap mx, mw;
+  if (!make_map_u8(&mx, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(K), kGemmBK, BN,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!make_map_u8(&mw, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4),
+                   kGemmBK / 4, kGemmBM, CU_TENSOR_MAP_SWIZZLE_32B))
+    return cudaErrorInvalidValue;
+  if (rs != nullptr) return launch_gemm_t<BN, STAGES, true>(mx, mw, gamma, a, rs, M, N, K, y, yd, s);
+  return launch_gemm_t<BN, STAGES, false>(mx, mw, gamma, a, rs, M, N, K, y, yd, s);
+}
+
+bitnet_status check_linear(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K, const int8_t* xq,
+                           const float* a, const int32_t* rs, int64_t M, void* y, int yd) {
+  if (Wp == nullptr || gamma == nullptr || xq == nullptr || a == nullptr || y == nullptr) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(Wp, 16) || !aligned(xq, 16) || !aligned(y, 16) || !aligned(gamma, 4) || !aligned(a, 4) ||
+      !aligned(rs, 4))
+    return BITNET_ERR_INVALID_ARG;
+  if (yd != BITNET_F32 && yd != BITNET_BF16 && yd != BITNET_I32) return BITNET_ERR_INVALID_ARG;
+  if (!valid_k(K) || N < 1 || M < 1 || N > INT32_MAX || M > INT32_MAX) return BITNET_ERR_UNSUPPORTED_SHAPE;
+  return BITNET_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t bitnet_pack_workspace_bytes(int64_t N, int64_t K) {
+  (void)K;
+  if (N < 1) return 0;
+  const size_t bytes = static_cast<size_t>(N) * sizeof(double) + 16;
+  return (bytes + 255) & ~size_t(255);
+}
+
+bitnet_status bitnet_pack_weights(const float* W, int64_t N, int64_t K, float eps, uint8_t* W_packed, float* gamma,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (W == nullptr || W_packed == nullptr || gamma == nullptr || workspace == nullptr) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(W_packed, 16) || !aligned(gamma, 4) || !aligned(workspace, 16))
+    return BITNET_ERR_INVALID_ARG;
+  if (!std::isfinite(eps) || !(eps > 0.0f)) return BITNET_ERR_INVALID_ARG;
+  if (!valid_k(K) || N < 1 || N > (int64_t{1} << 31) || N * K > (int64_t{1} << 40)) return BITNET_ERR_UNSUPPORTED_SHAPE;
+  if (workspace_bytes < bitnet_pack_workspace_bytes(N, K)) return BITNET_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  double* rowsum = static_cast<double*>(workspace);
+  float* d = reinterpret_cast<float*>(rowsum + N);
+  unsigned int* flag = reinterpret_cast<unsigned int*>(d + 1);
+
+  if (cudaMemsetAsync(flag, 0, sizeof(unsigned int), s) != cudaSuccess) return BITNET_ERR_CUDA;
+  const int64_t warps_wanted = N;
+  const int blocks1 = static_cast<int>(std::min<int64_t>((warps_wanted + 7) / 8, int64_t{sm_count()} * 8));
+  pack_rowsum_kernel<<<blocks1, 256, 0, s>>>(W, N, K, rowsum, flag);
+  pack_gamma_kernel<<<1, 32, 0, s>>>(rowsum, N, K, eps, gamma, d);
+  const int64_t nwords = N * K / 16;
+  const int blocks3 = static_cast<int>(std::min<int64_t>((nwords + 255) / 256, int64_t{sm_count()} * 16));
+  pack_codes_kernel<<<blocks3, 256, 0, s>>>(W, nwords, d, reinterpret_cast<uint32_t*>(W_packed));
+  if (cudaGetLastError() != cudaSuccess) return BITNET_ERR_CUDA;
+  unsigned int host_flag = 0;
+  if (cudaMemcpyAsync(&host_flag, flag, sizeof(host_flag), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BITNET_ERR_CUDA;
+  return host_flag != 0 ? BITNET_ERR_NONFINITE : BITNET_OK;
+}
+
+bitnet_status bitnet_quant_act(const void* x, int x_dtype, int64_t M, int64_t K, const void* rms_gain, float rms_eps,
+                               int8_t* x_q, float* a_scale, int32_t* x_rowsum, void* stream) {
+  if (x == nullptr || x_q == nullptr || a_scale == nullptr) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(x_q, 16) || !aligned(rms_gain, 16) || !aligned(a_scale, 4) || !aligned(x_rowsum, 4))
+    return BITNET_ERR_INVALID_ARG;
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
+  if (rms_gain != nullptr && (!std::isfinite(rms_eps) || !(rms_eps > 0.0f))) return BITNET_ERR_INVALID_ARG;
+  const int64_t kmax = x_dtype == BITNET_BF16 ? 32768 : 16384;
+  if (!valid_k(K) || K > kmax || M < 1 || M > INT32_MAX) return BITNET_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t e =
+      x_dtype == BITNET_BF16
+          ? launch_quant<__nv_bfloat16>(x, M, static_cast<int>(K), rms_gain, rms_eps, x_q, a_scale, x_rowsum, s)
+          : launch_quant<float>(x, M, static_cast<int>(K), rms_gain, rms_eps, x_q, a_scale, x_rowsum, s);
+  return from_cuda(e);
+}
+
+bitnet_status bitnet_linear_gemv(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, const int8_t* x_q,
+                                 const float* a_scale, const int32_t* x_rowsum, int64_t M, void* y, int y_dtype,
+                                 void* stream) {
+  const bitnet_status st = check_linear(W_packed, gamma, N, K, x_q, a_scale, x_rowsum, M, y, y_dtype);
+  if (st != BITNET_OK) return st;
+  if (M > 8) return BITNET_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int n = static_cast<int>(N), k = static_cast<int>(K), m = static_cast<int>(M);
+  const cudaError_t e = x_rowsum != nullptr
+                            ? launch_gemv_u<true>(m, W_packed, gamma, n, k, x_q, a_scale, x_rowsum, y, y_dtype, s)
+                            : launch_gemv_u<false>(m, W_packed, gamma, n, k, x_q, a_scale, x_rowsum, y, y_dtype, s);
+  return from_cuda(e);
+}
+
+bitnet_status bitnet_linear_gemm(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, const int8_t* x_q,
+                                 const float* a_scale, const int32_t* x_rowsum, int64_t M, void* y, int y_dtype,
+                                 void* stream) {
+  const bitnet_status st = check_linear(W_packed, gamma, N, K, x_q, a_scale, x_rowsum, M, y, y_dtype);
+  if (st != BITNET_OK) return st;
+  if ((M + 15) / 16 > 65535) return BITNET_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int n = static_cast<int>(N), k = static_cast<int>(K), m = static_cast<int>(M);
+  cudaError_t e;
+  if (m <= 16) e = launch_gemm_bn<16, 4>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
+  else if (m <= 32) e = launch_gemm_bn<32, 4>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
+  else if (m <= 64) e = launch_gemm_bn<64, 4>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
+  else if ((m + 127) / 128 <= 65535)
+    e = launch_gemm_bn<128, 4>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
+  else return BITNET_ERR_UNSUPPORTED_SHAPE;
+  return from_cuda(e);
+}
+
+bitnet_status bitnet_get_device_status(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BITNET_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, bitnet::g_device_error, sizeof(v)) != cudaSuccess) return BITNET_ERR_CUDA;
+  if (v != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(bitnet::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return BITNET_ERR_CUDA;
+    return BITNET_ERR_TIMEOUT;
+  }
+  return BITNET_OK;
+}
+
+const char* bitnet_status_string(bitnet_status s) {
+  switch (s) {
+    case BITNET_OK: return "ok";
+    case BITNET_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, bad dtype or eps)";
+    case BITNET_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (K must be a positive multiple of 64; M, N >= 1)";
+    case BITNET_ERR_NONFINITE: return "weight matrix holds a non-finite value";
+    case BITNET_ERR_CUDA: return "CUDA error";
+    case BITNET_ERR_TIMEOUT: return "a kernel timed out waiting on a barrier";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

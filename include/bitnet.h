@@ -1,0 +1,175 @@
+/*
+ * bitnet.h -- C ABI of the BitNet b1.58 BitLinear forward (W1.58A8) for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The four steps of BitLinear, as the BitNet b1.58 pages describe them
+ * (comrad404.com, "BitNet b1.58: что показала работа Microsoft об «эре
+ * 1-битных LLM»", section "Метод: как устроен BitNet b1.58"): normalise the
+ * input, quantise the activations to 8 bits, replace the weights by ternary
+ * {-1, 0, 1} ones obtained by absmean, then a low-bit matrix product followed
+ * by rescaling of the result.
+ *
+ * Conventions for every call below:
+ *   - All array pointers are DEVICE pointers, allocated and owned by the
+ *     caller.  The library allocates no memory and keeps no per-call state.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call is enqueued on that stream and returns without
+ *     waiting, except bitnet_pack_weights and bitnet_get_device_status,
+ *     which synchronise the stream.
+ *   - Matrices are dense, row-major and contiguous.  W is N x K (row n is
+ *     output feature n), activations are M x K (row m is token m), outputs
+ *     are M x N.
+ *   - K must be a positive multiple of 64 (so a packed row is a whole number
+ *     of 16-byte units); M >= 1 and N >= 1 are arbitrary.
+ *   - Every pointer must be 16-byte aligned.
+ *   - Errors are returned as bitnet_status; nothing is launched when an
+ *     argument is rejected.  No C++ exception crosses this boundary.
+ *
+ * Packed weight layout (2 bits per weight; the pages say only that the three
+ * states are stored on two bits plus some structure -- inferownia.pl,
+ * "BitNet b1.58: era 1-bitowych LLM-ów", section "Skąd te 1,58 bita"):
+ *   code c = q + 1 in {0, 1, 2} (3 never occurs); a row takes K/4 bytes; one
+ *   little-endian 32-bit word holds 16 consecutive weights k0..k0+15, weight
+ *   k0 + 4j + b in byte b, bits 2j..2j+1.  So (word >> 2j) & 0x03030303 gives
+ *   the codes of weights k0+4j .. k0+4j+3 in its four bytes.
+ */
+#ifndef BITNET_H_
+#define BITNET_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum bitnet_status {
+  BITNET_OK = 0,
+  BITNET_ERR_INVALID_ARG = 1,       /* null/misaligned pointer, bad dtype, bad eps */
+  BITNET_ERR_UNSUPPORTED_SHAPE = 2, /* K not a positive multiple of 64, M/N < 1, sizes too large */
+  BITNET_ERR_NONFINITE = 3,         /* bitnet_pack_weights: W holds Inf or NaN */
+  BITNET_ERR_CUDA = 4,              /* a CUDA runtime or driver call failed */
+  BITNET_ERR_TIMEOUT = 5            /* a kernel gave up waiting on a barrier (see get_device_status) */
+} bitnet_status;
+
+typedef enum bitnet_dtype {
+  BITNET_F32 = 0,
+  BITNET_BF16 = 1,
+  BITNET_I32 = 2 /* outputs only: the raw int32 accumulator, no dequantisation */
+} bitnet_dtype;
+
+/* Bytes of scratch memory bitnet_pack_weights needs for an N x K matrix. */
+size_t bitnet_pack_workspace_bytes(int64_t N, int64_t K);
+
+/*
+ * Absmean ternarisation and 2-bit packing of a latent fp32 weight matrix
+ * (inferownia.pl, "BitNet b1.58: era 1-bitowych LLM-ów", section "Trenowany
+ * od zera": the whole matrix is scaled by its mean absolute value and every
+ * entry goes to the nearest integer of {-1, 0, +1}).
+ *
+ *   gamma = mean |W| over all N*K entries.  Summation order is fixed, so the
+ *           result is reproducible bit for bit: per row, 32 fp64 partials
+ *           (partial l takes k = l, l+32, ... in increasing k) combined by the
+ *           halving tree p[l] += p[l+s], s = 16, 8, 4, 2, 1; rows added in
+ *           increasing n in fp64; gamma = RN32(S / (N*K)).
+ *   q     = clamp(RNE(RN32(w / RN32(gamma + eps))), -1, 1), ties to even.
+ *
+ * W         [in]  N x K fp32, device.
+ * eps       [in]  finite, > 0 (keeps the divisor positive for an all-zero W).
+ * W_packed  [out] N x K/4 bytes, device, layout above.
+ * gamma     [out] 1 fp32, device: the per-tensor scale used by the product.
+ * workspace [in]  device scratch of at least bitnet_pack_workspace_bytes(N, K)
+ *                 bytes; its contents on entry do not matter.
+ * Synchronises `stream`.  Returns BITNET_ERR_NONFINITE (outputs unspecified)
+ * if W holds a non-finite value.
+ */
+bitnet_status bitnet_pack_weights(const float* W, int64_t N, int64_t K, float eps,
+                                  uint8_t* W_packed, float* gamma,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Per-token absmax int8 quantisation of activations, optionally fused with
+ * the RMSNorm that precedes it (comrad404.com review, section "Метод":
+ * 8-bit activations, RMSNorm in the LLaMA-like stack, "normalise, then
+ * quantise").  One pass over x.  For each token row v (values widened to
+ * fp32 exactly):
+ *   with rms_gain:  ss = sum of RN32(v_k^2) in a fixed order (256 lanes, lane
+ *                   l owning the 8-element chunks c = l, l+256, ... summed in
+ *                   increasing k; then the halving tree l += l+128, ..., l+1);
+ *                   r = RN32(1 / RN32(sqrt(RN32(RN32(ss / K) + rms_eps))));
+ *                   h_k = RN32(RN32(v_k * r) * g_k)
+ *   without:        h = v
+ *   amax = max |h|;  s = RN32(127 / amax);
+ *   x_q  = clamp(RNE(RN32(h * s)), -127, 127);  a_scale = RN32(amax / 127);
+ *   a token with amax == 0 gets x_q = 0 and a_scale = 0.
+ *
+ * x        [in]  M x K, dtype x_dtype (BITNET_F32 or BITNET_BF16), device.
+ * rms_gain [in]  K values of the same dtype as x, or NULL for no RMSNorm.
+ * rms_eps  [in]  finite, > 0 when rms_gain is given; ignored otherwise.
+ * x_q      [out] M x K int8.
+ * a_scale  [out] M fp32 per-token dequant scales.
+ * x_rowsum [out] M int32 sums of x_q per token, or NULL to skip.
+ * K <= 32768 for BF16 input, K <= 16384 for F32.  Non-finite inputs give
+ * unspecified codes.  Asynchronous.
+ */
+bitnet_status bitnet_quant_act(const void* x, int x_dtype, int64_t M, int64_t K,
+                               const void* rms_gain, float rms_eps,
+                               int8_t* x_q, float* a_scale, int32_t* x_rowsum, void* stream);
+
+/*
+ * W1.58A8 product with exact int32 accumulation and fused dequant epilogue,
+ * for small batches (decode), on CUDA cores: packed weights are streamed
+ * once through shared memory with bulk asynchronous copies, each warp forms
+ * byte dot products (dp4a) and reduces them with warp shuffles.
+ * The ternary product is the sum of the inputs with weight +1 minus the sum
+ * of those with weight -1 (Habr repost on juhe.plus, section "Когда - три
+ * лучше двух"); the integer result is exact.
+ *
+ *   acc[m][n] = sum_k q[n][k] * x_q[m][k]              (exact, int32)
+ *   y[m][n]   = RN32(RN32(float(acc) * gamma) * a_scale[m])   (F32), or its
+ *               round-half-even bf16 (BF16), or acc itself (I32).
+ *
+ * W_packed [in]  N x K/4 bytes from bitnet_pack_weights.
+ * gamma    [in]  1 fp32, device, from bitnet_pack_weights.
+ * x_q, a_scale [in] from bitnet_quant_act (M x K int8, M fp32).
+ * x_rowsum [in]  M int32 = sum_k x_q[m][k], or NULL.  When given, the kernel
+ *                multiplies by the unsigned codes c = q + 1 and subtracts
+ *                the row sum, which saves work; the result is identical.
+ * M        [in]  1 <= M <= 8.
+ * y        [out] M x N of dtype y_dtype (BITNET_F32, BITNET_BF16 or BITNET_I32).
+ * Asynchronous.
+ */
+bitnet_status bitnet_linear_gemv(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K,
+                                 const int8_t* x_q, const float* a_scale, const int32_t* x_rowsum,
+                                 int64_t M, void* y, int y_dtype, void* stream);
+
+/*
+ * The same product for any M >= 1 on the 5th-generation tensor cores
+ * (tcgen05 kind::i8, int32 accumulators in tensor memory): packed weight
+ * tiles and activation tiles arrive in shared memory by TMA, the ternary
+ * codes are expanded to 8-bit in registers and written to tensor memory as
+ * the A operand, the activations are the B operand in shared memory.
+ * Same arguments, formulas and results as bitnet_linear_gemv.
+ * M <= 2^31 - 1, N <= 2^31 - 1, K <= 2^31 - 1 with M*N fitting the output.
+ * Asynchronous.
+ */
+bitnet_status bitnet_linear_gemm(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K,
+                                 const int8_t* x_q, const float* a_scale, const int32_t* x_rowsum,
+                                 int64_t M, void* y, int y_dtype, void* stream);
+
+/*
+ * Synchronises `stream`, then reports and clears the device-side error word
+ * that kernels set when a bounded wait on a barrier runs out (they then skip
+ * their remaining work and exit instead of hanging).  Returns BITNET_OK,
+ * BITNET_ERR_TIMEOUT, or BITNET_ERR_CUDA if the stream itself failed.
+ */
+bitnet_status bitnet_get_device_status(void* stream);
+
+/* Static English description of a status code. */
+const char* bitnet_status_string(bitnet_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITNET_H_ */

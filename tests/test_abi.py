@@ -1,0 +1,107 @@
+"""The C ABI library: it loads on a machine without a GPU, exports every
+entry point include/bitnet.h declares, and rejects bad arguments on the
+host before touching CUDA (every call below fails validation, so nothing is
+launched and no CUDA call is made)."""
+import ctypes
+
+import pytest
+
+import bitlinear_absmean_ternary_b200 as bl
+from bitlinear_absmean_ternary_b200 import build as blbuild
+
+
+@pytest.fixture(scope="module")
+def L():
+    blbuild.build()
+    return bl.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = bl.declared_functions()
+    assert set(names) >= {"bitnet_pack_weights", "bitnet_quant_act", "bitnet_linear_gemv", "bitnet_linear_gemm",
+                          "bitnet_pack_workspace_bytes", "bitnet_get_device_status", "bitnet_status_string"}
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code in range(6):
+        s = bl.status_string(code)
+        assert s and s != "unknown status"
+    assert bl.status_string(99) == "unknown status"
+
+
+def test_workspace_bytes(L):
+    assert bl.bitnet_pack_workspace_bytes(0, 64) == 0
+    for N in (1, 7, 2560, 21504):
+        b = bl.bitnet_pack_workspace_bytes(N, 2560)
+        assert b >= 8 * N + 8 and b % 256 == 0
+
+
+FAKE = 0x10000  # a 16-byte aligned address that is never dereferenced: validation fails first
+MIS = FAKE + 4   # misaligned for 16-byte rules
+
+
+def pack(L, W=FAKE, N=4, K=64, eps=1e-5, out=FAKE, g=FAKE, ws=FAKE, wsb=1 << 20):
+    return L.bitnet_pack_weights(W, N, K, eps, out, g, ws, wsb, None)
+
+
+def test_pack_rejects_bad_arguments(L):
+    assert pack(L, W=None) == bl.BITNET_ERR_INVALID_ARG
+    assert pack(L, out=None) == bl.BITNET_ERR_INVALID_ARG
+    assert pack(L, W=MIS) == bl.BITNET_ERR_INVALID_ARG
+    assert pack(L, eps=0.0) == bl.BITNET_ERR_INVALID_ARG
+    assert pack(L, eps=-1.0) == bl.BITNET_ERR_INVALID_ARG
+    assert pack(L, eps=float("nan")) == bl.BITNET_ERR_INVALID_ARG
+    assert pack(L, K=100) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert pack(L, K=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert pack(L, N=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert pack(L, wsb=16) == bl.BITNET_ERR_INVALID_ARG
+
+
+def quant(L, x=FAKE, dt=bl.BITNET_BF16, M=2, K=64, g=None, eps=1e-5, xq=FAKE, a=FAKE, rs=None):
+    return L.bitnet_quant_act(x, dt, M, K, g, eps, xq, a, rs, None)
+
+
+def test_quant_rejects_bad_arguments(L):
+    assert quant(L, x=None) == bl.BITNET_ERR_INVALID_ARG
+    assert quant(L, a=None) == bl.BITNET_ERR_INVALID_ARG
+    assert quant(L, x=MIS) == bl.BITNET_ERR_INVALID_ARG
+    assert quant(L, dt=bl.BITNET_I32) == bl.BITNET_ERR_INVALID_ARG
+    assert quant(L, dt=7) == bl.BITNET_ERR_INVALID_ARG
+    assert quant(L, g=FAKE, eps=0.0) == bl.BITNET_ERR_INVALID_ARG
+    assert quant(L, rs=FAKE + 2) == bl.BITNET_ERR_INVALID_ARG
+    assert quant(L, K=96) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert quant(L, M=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert quant(L, K=32768 + 64) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert quant(L, dt=bl.BITNET_F32, K=16384 + 64) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+
+
+@pytest.mark.parametrize("name", ["bitnet_linear_gemv", "bitnet_linear_gemm"])
+def test_linear_rejects_bad_arguments(L, name):
+    fn = getattr(L, name)
+
+    def call(W=FAKE, g=FAKE, N=8, K=64, xq=FAKE, a=FAKE, rs=None, M=1, y=FAKE, yd=bl.BITNET_BF16):
+        return fn(W, g, N, K, xq, a, rs, M, y, yd, None)
+
+    assert call(W=None) == bl.BITNET_ERR_INVALID_ARG
+    assert call(g=None) == bl.BITNET_ERR_INVALID_ARG
+    assert call(y=None) == bl.BITNET_ERR_INVALID_ARG
+    assert call(W=MIS) == bl.BITNET_ERR_INVALID_ARG
+    assert call(y=MIS) == bl.BITNET_ERR_INVALID_ARG
+    assert call(g=FAKE + 1) == bl.BITNET_ERR_INVALID_ARG
+    assert call(yd=5) == bl.BITNET_ERR_INVALID_ARG
+    assert call(K=32) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(K=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(N=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(M=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(N=1 << 31) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    if name == "bitnet_linear_gemv":
+        assert call(M=9) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(bl, "_lib", None)
+    monkeypatch.setattr(bl, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        bl.lib()

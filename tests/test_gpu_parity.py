@@ -1,0 +1,311 @@
+"""GPU parity: every step of the CUDA path against the CPU oracle, element by
+element, on the same seeded inputs.
+
+Integer results (packed weight bytes, int8 activations, int32 accumulators)
+and the fp32 scales must match bit for bit.  Dequantised outputs must lie
+within 1 ulp (fp32) or 1 bf16 ulp of the oracle; both sides run the same
+sequence of correctly rounded fp32 operations, so in practice they match
+exactly, and the tests also report that.
+"""
+import numpy as np
+import pytest
+
+import bitlinear_absmean_ternary_b200 as bl
+from bitlinear_absmean_ternary_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+EPS_W = 1e-5
+EPS_RMS = 1e-5
+
+
+@pytest.fixture(scope="module")
+def dev():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    bl.lib()
+    return torch.device("cuda:0")
+
+
+def _t(a, dev, dtype=None):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    return t if dtype is None else t.to(dtype)
+
+
+def _x_dev(x32, dtype, dev):
+    """fp32 values already rounded to dtype -> device tensor of that dtype (exact)."""
+    import torch
+    if dtype == "bf16":
+        bits = synth.f32_to_bf16_bits(x32).view(np.int16)
+        return torch.from_numpy(bits.copy()).to(dev).view(torch.bfloat16)
+    return _t(x32.astype(np.float32), dev)
+
+
+def ulp_diff_f32(a, b):
+    ai = np.asarray(a, np.float32).view(np.int32).astype(np.int64)
+    bi = np.asarray(b, np.float32).view(np.int32).astype(np.int64)
+    ai = np.where(ai < 0, -(ai & 0x7FFFFFFF), ai)
+    bi = np.where(bi < 0, -(bi & 0x7FFFFFFF), bi)
+    return np.abs(ai - bi)
+
+
+def ulp_diff_bf16(a_bits, b_bits):
+    ai = np.asarray(a_bits, np.uint16).astype(np.int64)
+    bi = np.asarray(b_bits, np.uint16).astype(np.int64)
+    ai = np.where(ai >= 0x8000, -(ai & 0x7FFF), ai)
+    bi = np.where(bi >= 0x8000, -(bi & 0x7FFF), bi)
+    return np.abs(ai - bi)
+
+
+# --------------------------------------------------------------------------- pack
+
+PACK_SHAPES = [(256, 256, 0.02), (6912, 2560, 0.02), (2560, 6912, 0.02), (1, 64, 0.02), (7, 192, 1.0),
+               (300, 640, 0.01), (13824, 2560, 0.02), (129, 2048, 3.0)]
+
+
+@pytest.mark.parametrize("N,K,sigma", PACK_SHAPES)
+def test_pack_parity(dev, orc, N, K, sigma):
+    W = synth.weights(N, K, sigma, 7, 1)
+    p_gpu, g_gpu = bl.bitnet_pack_weights(_t(W, dev), EPS_W)
+    p_ref, g_ref = orc.pack_weights(W, EPS_W)
+    assert g_gpu.cpu().numpy()[0] == g_ref
+    np.testing.assert_array_equal(p_gpu.cpu().numpy(), p_ref)
+
+
+def test_pack_parity_27b_shape(dev, orc):
+    W = synth.weights(21504, 5376, 0.01, 0, 91)
+    p_gpu, g_gpu = bl.bitnet_pack_weights(_t(W, dev), EPS_W)
+    p_ref, g_ref = orc.pack_weights(W, EPS_W)
+    assert g_gpu.cpu().numpy()[0] == g_ref
+    assert np.array_equal(p_gpu.cpu().numpy(), p_ref)
+
+
+def test_pack_edge_cases(dev, orc):
+    # all-zero matrix: gamma 0, every code 0 (byte 0x55)
+    p, g = bl.bitnet_pack_weights(_t(np.zeros((5, 128), np.float32), dev), EPS_W)
+    assert g.item() == 0.0 and np.all(p.cpu().numpy() == 0x55)
+    # +-2^j: gamma exact, codes = sign
+    rng = np.random.default_rng(1)
+    W = (rng.choice([-1.0, 1.0], size=(64, 256)) * 0.25).astype(np.float32)
+    p, g = bl.bitnet_pack_weights(_t(W, dev), EPS_W)
+    assert g.item() == 0.25
+    q, bad = orc.unpack_codes(p.cpu().numpy(), 256)
+    assert bad == 0 and np.array_equal(q, np.sign(W).astype(np.int8))
+    # exact ties, with the divisor made exactly 1 (eps = 1 - gamma)
+    row = np.full(64, 0.125, np.float32)
+    row[:6] = [0.5, -0.5, 1.5, -1.5, 2.5, 0.75]
+    g_ref = orc.absmean_gamma(row[None])
+    eps = float(np.float32(1.0) - g_ref)
+    p, g = bl.bitnet_pack_weights(_t(row[None], dev), eps)
+    p_ref, _ = orc.pack_weights(row[None], eps)
+    np.testing.assert_array_equal(p.cpu().numpy(), p_ref)
+    # non-finite input is reported
+    W = synth.weights(8, 64, 0.02, 0, 1)
+    W[3, 9] = np.nan
+    with pytest.raises(bl.BitnetError) as e:
+        bl.bitnet_pack_weights(_t(W, dev), EPS_W)
+    assert e.value.status == bl.BITNET_ERR_NONFINITE
+
+
+# --------------------------------------------------------------------------- quant
+
+QUANT_CASES = [
+    # M, K, dist, outlier frac, outlier scale, dtype, norm
+    (4, 256, "normal", 0.0, 1.0, "f32", False),
+    (1, 2560, "normal", 0.01, 20.0, "bf16", False),
+    (1, 6912, "normal", 0.01, 20.0, "bf16", False),
+    (64, 2560, "normal", 0.0, 1.0, "bf16", True),
+    (64, 6912, "normal", 0.0, 1.0, "bf16", True),
+    (4096, 2560, "student_t4", 0.0, 1.0, "bf16", False),
+    (16, 21504, "normal", 0.005, 30.0, "bf16", False),
+    (2048, 5376, "normal", 0.005, 30.0, "bf16", False),
+    (3, 64, "normal", 0.0, 1.0, "bf16", True),
+    (5, 1344, "student_t4", 0.0, 1.0, "f32", True),
+    (2, 32768, "normal", 0.0, 1.0, "bf16", True),
+    (2, 16384, "normal", 0.0, 1.0, "f32", False),
+]
+
+
+@pytest.mark.parametrize("M,K,dist,of,osc,dt,norm", QUANT_CASES)
+def test_quant_parity(dev, orc, M, K, dist, of, osc, dt, norm):
+    x = synth.activations(M, K, 3, 2, dist, of, osc, dt)
+    g = synth.gain(K, 3, 3, dt) if norm else None
+    xq, a, rs = bl.bitnet_quant_act(_x_dev(x, dt, dev), None if g is None else _x_dev(g, dt, dev), EPS_RMS,
+                                    want_rowsum=True)
+    xq_r, a_r, rs_r = orc.quant_act(x, g, EPS_RMS)
+    np.testing.assert_array_equal(xq.cpu().numpy(), xq_r)
+    np.testing.assert_array_equal(a.cpu().numpy(), a_r)
+    np.testing.assert_array_equal(rs.cpu().numpy(), rs_r)
+
+
+def test_quant_edge_tokens(dev, orc):
+    K = 128
+    x = synth.activations(6, K, 1, 2, "normal", 0.0, 1.0, "f32")
+    x[0] = 0.0                                   # zero token
+    x[1] = 0.0
+    x[1, 77] = -3.0                              # one-hot
+    x[2, :10] = [127, 0.5, 1.5, 2.5, -2.5, -0.5, 126.5, 3.5, -3.5, 0.25]
+    x[2, 10:] = 0.0                              # exact ties
+    x[3] *= np.float32(2.0 ** 40)                # huge
+    x[4] *= np.float32(2.0 ** -60)               # tiny
+    for norm in (False, True):
+        g = synth.gain(K, 1, 3, "f32") if norm else None
+        xq, a, rs = bl.bitnet_quant_act(_t(x, dev), None if g is None else _t(g, dev), EPS_RMS, want_rowsum=True)
+        xq_r, a_r, rs_r = orc.quant_act(x, g, EPS_RMS)
+        np.testing.assert_array_equal(xq.cpu().numpy(), xq_r)
+        np.testing.assert_array_equal(a.cpu().numpy(), a_r)
+        np.testing.assert_array_equal(rs.cpu().numpy(), rs_r)
+    # the quantisation without rowsum output gives the same codes
+    xq2, a2, rs2 = bl.bitnet_quant_act(_t(x, dev))
+    assert rs2 is None
+    np.testing.assert_array_equal(xq2.cpu().numpy(), orc.quant_act(x)[0])
+
+
+# --------------------------------------------------------------------------- linear
+
+def _ref_linear(orc, packed, gamma, K, xq, a):
+    acc, y = orc.bitlinear(packed, gamma, K, xq, a)
+    return acc, y
+
+
+def _check_linear(dev, orc, fn, M, N, K, seed=0, zero_row=None, zero_tok=None, sample=None):
+    import torch
+    rng = np.random.default_rng(seed)
+    q = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    if zero_row is not None:
+        q[zero_row] = 0
+    packed = orc.pack_codes(q)
+    x = synth.activations(M, K, seed, 5, "student_t4", 0.0, 1.0, "f32")
+    if zero_tok is not None:
+        x[zero_tok] = 0.0
+    xq, a, rs = orc.quant_act(x)
+    gamma = np.float32(0.0173)
+    P, G = _t(packed, dev), _t(np.array([gamma], np.float32), dev)
+    XQ, A, RS = _t(xq, dev), _t(a, dev), _t(rs, dev)
+    if sample is None:
+        acc_r, y_r = orc.bitlinear(packed, gamma, K, xq, a)
+    else:
+        ms = np.concatenate([rng.integers(0, M, sample), np.arange(M), np.full(N if N < 64 else 64, M - 1)])
+        ns = np.concatenate([rng.integers(0, N, sample), np.full(M, N - 1), np.arange(N if N < 64 else 64)])
+        acc_r, y_r = orc.bitlinear_sampled(packed, gamma, K, xq, a, ms, ns)
+    for rowsum in (None, RS):
+        acc_g = fn(P, G, XQ, A, rowsum, out_dtype=torch.int32).cpu().numpy()
+        y32 = fn(P, G, XQ, A, rowsum, out_dtype=torch.float32).cpu().numpy()
+        yb = fn(P, G, XQ, A, rowsum, out_dtype=torch.bfloat16).view(torch.int16).cpu().numpy().view(np.uint16)
+        if sample is not None:
+            acc_g, y32, yb = acc_g[ms, ns], y32[ms, ns], yb[ms, ns]
+        np.testing.assert_array_equal(acc_g, acc_r)
+        d32 = ulp_diff_f32(y32, y_r)
+        assert d32.max() <= 1, f"fp32 output off by {d32.max()} ulp"
+        db = ulp_diff_bf16(yb, orc.f32_to_bf16(y_r))
+        assert db.max() <= 1, f"bf16 output off by {db.max()} ulp"
+        assert d32.max() == 0 and db.max() == 0, "expected bit-exact outputs"
+
+
+GEMV_CASES = [(1, 256, 256), (4, 256, 256), (8, 6912, 2560), (1, 2560, 6912), (3, 129, 192), (5, 1, 64),
+              (2, 37, 4160), (7, 300, 640), (1, 1000, 21504), (6, 77, 8192)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMV_CASES)
+def test_gemv_parity(dev, orc, M, N, K):
+    _check_linear(dev, orc, bl.bitnet_linear_gemv, M, N, K, seed=M + N + K, zero_row=min(3, N - 1), zero_tok=0)
+
+
+GEMM_CASES = [(4, 256, 256), (16, 256, 256), (1, 128, 128), (17, 129, 192), (64, 3840, 2560), (33, 200, 64),
+              (100, 300, 640), (129, 257, 1088), (256, 512, 1024), (300, 1000, 2048), (64, 2560, 6912)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_CASES)
+def test_gemm_parity(dev, orc, M, N, K):
+    _check_linear(dev, orc, bl.bitnet_linear_gemm, M, N, K, seed=M * 7 + N + K, zero_row=min(5, N - 1),
+                  zero_tok=min(2, M - 1))
+
+
+@pytest.mark.parametrize("M,N,K", [(4096, 6912, 2560), (2048, 5376, 21504), (16, 21504, 5376)])
+def test_gemm_parity_large_sampled(dev, orc, M, N, K):
+    _check_linear(dev, orc, bl.bitnet_linear_gemm, M, N, K, seed=1, sample=3000)
+
+
+def test_gemv_and_gemm_agree(dev, orc):
+    import torch
+    rng = np.random.default_rng(9)
+    N, K = 640, 2560
+    P = _t(orc.pack_codes(rng.integers(-1, 2, size=(N, K)).astype(np.int8)), dev)
+    G = _t(np.array([0.02], np.float32), dev)
+    for M in range(1, 9):
+        x = synth.activations(M, K, M, 5, "normal", 0.0, 1.0, "bf16")
+        xq, a, rs = bl.bitnet_quant_act(_x_dev(x, "bf16", dev), want_rowsum=True)
+        y1 = bl.bitnet_linear_gemv(P, G, xq, a, rs, out_dtype=torch.float32)
+        y2 = bl.bitnet_linear_gemm(P, G, xq, a, None, out_dtype=torch.float32)
+        assert torch.equal(y1, y2)
+
+
+# --------------------------------------------------------------------------- whole workloads
+
+_PACKED = {}
+
+
+def _packed_weights(lin, dev, orc):
+    """(device pack, oracle pack) of a workload's weights, checked once per weight spec."""
+    key = (lin.N, lin.K, lin.w_sigma, lin.w_id)
+    if key not in _PACKED:
+        if len(_PACKED) >= 2:
+            _PACKED.clear()
+        W = lin.make_w(0)
+        P, G = bl.bitnet_pack_weights(_t(W, dev), EPS_W)
+        p_ref, g_ref = orc.pack_weights(W, EPS_W)
+        assert G.item() == g_ref
+        assert np.array_equal(P.cpu().numpy(), p_ref)
+        _PACKED[key] = (P, G, p_ref, g_ref)
+    return _PACKED[key]
+
+
+@pytest.mark.parametrize("workload", list(synth.WORKLOADS))
+def test_workload_end_to_end(dev, orc, workload):
+    """pack -> quant -> product on each named workload at full size, in the
+    launch configuration the benchmark uses; outputs checked on samples."""
+    import torch
+    for lin in synth.WORKLOADS[workload]:
+        x = lin.make_x(0)
+        g = lin.make_gain(0)
+        P, G, p_ref, g_ref = _packed_weights(lin, dev, orc)
+        xq, a, rs = bl.bitnet_quant_act(_x_dev(x, lin.x_dtype, dev),
+                                        None if g is None else _x_dev(g, lin.x_dtype, dev), EPS_RMS,
+                                        want_rowsum=True)
+        xq_r, a_r, rs_r = orc.quant_act(x, g, EPS_RMS)
+        assert np.array_equal(xq.cpu().numpy(), xq_r)
+        assert np.array_equal(a.cpu().numpy(), a_r)
+        out = torch.float32 if lin.y_dtype == "f32" else torch.bfloat16
+        fns = [bl.bitnet_linear_gemv, bl.bitnet_linear_gemm] if lin.M <= 8 else [bl.bitnet_linear_gemm]
+        rng = np.random.default_rng(0)
+        ms = rng.integers(0, lin.M, 2000)
+        ns = rng.integers(0, lin.N, 2000)
+        acc_r, y_r = orc.bitlinear_sampled(p_ref, g_ref, lin.K, xq_r, a_r, ms, ns)
+        for fn in fns:
+            acc = fn(P, G, xq, a, rs, out_dtype=torch.int32).cpu().numpy()[ms, ns]
+            np.testing.assert_array_equal(acc, acc_r)
+            y = fn(P, G, xq, a, rs, out_dtype=out)
+            if out == torch.float32:
+                assert ulp_diff_f32(y.cpu().numpy()[ms, ns], y_r).max() == 0
+            else:
+                yb = y.view(torch.int16).cpu().numpy().view(np.uint16)[ms, ns]
+                assert ulp_diff_bf16(yb, orc.f32_to_bf16(y_r)).max() == 0
+
+
+def test_repeatable_and_status_clean(dev, orc):
+    import torch
+    lin = synth.WORKLOADS["decode_m64_2p5b_block"][3]
+    P, G = bl.bitnet_pack_weights(_t(lin.make_w(0), dev), EPS_W)
+    x = _x_dev(lin.make_x(0), "bf16", dev)
+    g = _x_dev(lin.make_gain(0), "bf16", dev)
+    outs = []
+    for _ in range(3):
+        xq, a, rs = bl.bitnet_quant_act(x, g, EPS_RMS, want_rowsum=True)
+        y = bl.bitnet_linear_gemm(P, G, xq, a, rs, out_dtype=torch.float32)
+        outs.append((xq.clone(), a.clone(), rs.clone(), y))
+    for o in outs[1:]:
+        for u, v in zip(outs[0], o):
+            assert torch.equal(u, v)
+    assert bl.bitnet_get_device_status() == bl.BITNET_OK
