@@ -88,6 +88,32 @@ bitnet_status bitnet_pack_weights(const float* W, int64_t N, int64_t K, float ep
                                   void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * bitnet_pack_weights without a caller workspace.  The BitNet b1.58 pages
+ * have no counterpart to this: it exists for callers that cannot allocate
+ * device memory -- code that runs inside a host application whose memory
+ * pool owns every device allocation, or services that must not allocate
+ * once they have started -- and so cannot provide the workspace buffer.
+ *
+ * Same arguments (minus the workspace), results and error behaviour as
+ * bitnet_pack_weights; it calls no cudaMalloc, cudaFree or allocating
+ * library routine.  Its scratch is a fixed array inside the library,
+ * 8 * BITNET_PACK_NOALLOC_MAX_ROWS + 256 bytes (about 512 KB), which every
+ * GPU that loads the library holds until the process exits.
+ *   - N above BITNET_PACK_NOALLOC_MAX_ROWS is rejected with
+ *     BITNET_ERR_UNSUPPORTED_SHAPE before anything is launched.
+ *   - The first call on each device looks up the device address of that
+ *     array (cudaGetSymbolAddress) with that device current; make that first
+ *     call before any stream capture.
+ *   - All calls share the array and it keeps the previous call's contents;
+ *     the call clears what must start at zero.  Calls that overlap on the GPU
+ *     (for example from two host threads on two streams) race on it.
+ * Synchronises `stream`.
+ */
+#define BITNET_PACK_NOALLOC_MAX_ROWS 65536
+bitnet_status bitnet_pack_weights_noalloc(const float* W, int64_t N, int64_t K, float eps,
+                                          uint8_t* W_packed, float* gamma, void* stream);
+
+/*
  * Per-token absmax int8 quantisation of activations, optionally fused with
  * the RMSNorm that precedes it (comrad404.com review, section "Метод":
  * 8-bit activations, RMSNorm in the LLaMA-like stack, "normalise, then
