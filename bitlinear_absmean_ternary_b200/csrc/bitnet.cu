@@ -45,12 +45,18 @@ int sm_count() {
   return cache[d];
 }
 
-// Opt a kernel into more than 48 KB of dynamic shared memory (once per device).
+// Opt a kernel into more than 48 KB of dynamic shared memory and ask for the
+// largest shared-memory carveout (once per device).  With every kernel of the
+// library on the same carveout, a kernel launched with programmatic
+// dependent launch can place its CTAs next to the previous kernel's CTAs
+// without the SM first draining to change its L1/shared split.
 template <typename F>
 cudaError_t set_smem(F* fn, int bytes, bool (&done)[kMaxDevices]) {
   const int d = current_device();
   if (d >= 0 && d < kMaxDevices && done[d]) return cudaSuccess;
-  const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess && d >= 0 && d < kMaxDevices) done[d] = true;
   return e;
 }
@@ -110,6 +116,9 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t row
 template <typename T, int MAXC>
 cudaError_t launch_quant_t(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
                            int32_t* rs, cudaStream_t s) {
+  static bool done[kMaxDevices] = {};
+  const cudaError_t e = set_smem(quant_act_kernel<T, MAXC>, 0, done);
+  if (e != cudaSuccess) return e;
   return launch_pdl(quant_act_kernel<T, MAXC>, dim3(static_cast<unsigned>(M)), dim3(kQuantThreads), 0, s,
                     static_cast<const T*>(x), K, static_cast<const T*>(gain), eps, xq, a, rs);
 }
@@ -126,16 +135,25 @@ cudaError_t launch_quant(const void* x, int64_t M, int K, const void* gain, floa
   return cudaErrorInvalidValue;
 }
 
-template <int MT, bool U8>
-cudaError_t launch_gemv_t(const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
+template <int MT, bool U8, bool XS>
+cudaError_t launch_gemv_x(const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
                           const int32_t* rs, void* y, int yd, cudaStream_t s) {
   static bool done[kMaxDevices] = {};
-  const cudaError_t e = set_smem(gemv_kernel<MT, U8>, kGemvSmemBytes, done);
+  constexpr int smem = gemv_smem_bytes(XS);
+  const cudaError_t e = set_smem(gemv_kernel<MT, U8, XS>, smem, done);
   if (e != cudaSuccess) return e;
   const int64_t groups = (N + kGemvRows - 1) / kGemvRows;
   const int grid = static_cast<int>(groups < sm_count() ? groups : sm_count());
-  return launch_pdl(gemv_kernel<MT, U8>, dim3(grid), dim3(kGemvWarps * 32), kGemvSmemBytes, s, Wp, gamma, N, K, xq,
-                    a, rs, y, yd);
+  return launch_pdl(gemv_kernel<MT, U8, XS>, dim3(grid), dim3(kGemvWarps * 32), smem, s, Wp, gamma, N, K, xq, a, rs,
+                    y, yd);
+}
+
+template <int MT, bool U8>
+cudaError_t launch_gemv_t(const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
+                          const int32_t* rs, void* y, int yd, cudaStream_t s) {
+  if (static_cast<int64_t>(MT) * K <= kGemvXMaxBytes)
+    return launch_gemv_x<MT, U8, true>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+  return launch_gemv_x<MT, U8, false>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
 }
 
 template <bool U8>
@@ -154,19 +172,20 @@ cudaError_t launch_gemv_u(int M, const uint8_t* Wp, const float* gamma, int N, i
   }
 }
 
-template <int BN, int STAGES, bool U8>
+template <int BN, bool U8>
 cudaError_t launch_gemm_t(const CUtensorMap& mx, const CUtensorMap& mw, const float* gamma, const float* a,
                           const int32_t* rs, int M, int N, int K, void* y, int yd, cudaStream_t s) {
-  using C = GemmCfg<BN, STAGES>;
+  using C = GemmCfg<BN>;
   static bool done[kMaxDevices] = {};
-  const cudaError_t e = set_smem(gemm_kernel<BN, STAGES, U8>, C::kSmemBytes, done);
+  const cudaError_t e = set_smem(gemm_kernel<BN, U8>, C::kSmemBytes, done);
   if (e != cudaSuccess) return e;
-  const dim3 grid((N + kGemmBM - 1) / kGemmBM, (M + BN - 1) / BN);
-  return launch_pdl(gemm_kernel<BN, STAGES, U8>, grid, dim3(kGemmThreads), C::kSmemBytes, s, mx, mw, gamma, a, rs, M,
+  const int64_t tiles = static_cast<int64_t>((N + kGemmBM - 1) / kGemmBM) * ((M + BN - 1) / BN);
+  const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
+  return launch_pdl(gemm_kernel<BN, U8>, dim3(grid), dim3(kGemmThreads), C::kSmemBytes, s, mx, mw, gamma, a, rs, M,
                     N, K, y, yd);
 }
 
-template <int BN, int STAGES>
+template <int BN>
 cudaError_t launch_gemm_bn(const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
                            const int32_t* rs, int M, void* y, int yd, cudaStream_t s) {
   CUtensorMap mx, mw;
@@ -176,8 +195,8 @@ cudaError_t launch_gemm_bn(const uint8_t* Wp, const float* gamma, int N, int K, 
   if (!make_map_u8(&mw, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4),
                    kGemmBK / 4, kGemmBM, CU_TENSOR_MAP_SWIZZLE_32B))
     return cudaErrorInvalidValue;
-  if (rs != nullptr) return launch_gemm_t<BN, STAGES, true>(mx, mw, gamma, a, rs, M, N, K, y, yd, s);
-  return launch_gemm_t<BN, STAGES, false>(mx, mw, gamma, a, rs, M, N, K, y, yd, s);
+  if (rs != nullptr) return launch_gemm_t<BN, true>(mx, mw, gamma, a, rs, M, N, K, y, yd, s);
+  return launch_gemm_t<BN, false>(mx, mw, gamma, a, rs, M, N, K, y, yd, s);
 }
 
 bitnet_status check_linear(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K, const int8_t* xq,
@@ -324,16 +343,13 @@ bitnet_status bitnet_linear_gemm(const uint8_t* W_packed, const float* gamma, in
                                  void* stream) {
   const bitnet_status st = check_linear(W_packed, gamma, N, K, x_q, a_scale, x_rowsum, M, y, y_dtype);
   if (st != BITNET_OK) return st;
-  if ((M + 15) / 16 > 65535) return BITNET_ERR_UNSUPPORTED_SHAPE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int n = static_cast<int>(N), k = static_cast<int>(K), m = static_cast<int>(M);
   cudaError_t e;
-  if (m <= 16) e = launch_gemm_bn<16, 4>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
-  else if (m <= 32) e = launch_gemm_bn<32, 4>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
-  else if (m <= 64) e = launch_gemm_bn<64, 4>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
-  else if ((m + 127) / 128 <= 65535)
-    e = launch_gemm_bn<128, 4>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
-  else return BITNET_ERR_UNSUPPORTED_SHAPE;
+  if (m <= 16) e = launch_gemm_bn<16>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
+  else if (m <= 32) e = launch_gemm_bn<32>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
+  else if (m <= 64) e = launch_gemm_bn<64>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
+  else e = launch_gemm_bn<128>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
   return from_cuda(e);
 }
 

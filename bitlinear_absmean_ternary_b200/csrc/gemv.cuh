@@ -2,19 +2,28 @@
 //
 // The ternary product is "the sum of the inputs with weight +1 minus the sum
 // of those with weight -1" (Habr repost on juhe.plus, section "Когда - три
-// лучше двух"); here each group of four weights is expanded to four signed
-// bytes and combined with four int8 activations by one dp4a, which is that
-// add/subtract exactly, in integers.
+// лучше двух"); here each group of four weights is expanded to four bytes
+// and combined with four int8 activations by one dp4a, which is that
+// add/subtract exactly, in integers.  With the per-token sum of x_q at hand
+// the bytes hold the unsigned codes c = q + 1 in {0, 1, 2} and the row sum
+// is subtracted once per output (sum c*x - sum x = sum q*x), which saves two
+// instructions per four weights.
 //
-// Work split: CTA c owns the contiguous rows [N*c/G, N*(c+1)/G) (G = grid);
-// inside a CTA, warps take groups of 4 consecutive rows round-robin.  A row
-// group is streamed in K-chunks of up to 4096 weights (4 x 1 KB): lane 0 of
-// the warp issues one bulk asynchronous copy per row into a 4-slot ring of
-// shared memory owned by that warp; all 32 lanes then read 16-byte pieces
-// (64 weights) of the 4 rows, so every activation load is reused 4 times.
-// Lane partial sums are reduced with warp shuffles.  The first ring slots are
-// requested before waiting on the previous kernel (programmatic dependent
-// launch), because the weights never depend on it.
+// Work split: CTA c owns the contiguous rows [N*c/G, N*(c+1)/G) (G = grid,
+// one CTA per SM); its warps take groups of 4 consecutive rows round-robin.
+// A group is streamed in items of up to 4096 weights per row (4 KB): lane 0
+// of the warp issues the bulk asynchronous copies of an item into a 2-slot
+// ring of shared memory owned by that warp.  The activations x_q (M*K bytes)
+// are copied into shared memory once per CTA when they fit.  Lane l handles
+// 16 consecutive weights of each of the 4 rows per 512-weight step, so the
+// warp's loads of codes (4 bytes per lane) and of activations (16 bytes per
+// lane) are contiguous and free of bank conflicts, and each activation load
+// serves 4 rows.  Lane partial sums are reduced with warp shuffles.
+//
+// The first weight items are requested before waiting on the previous
+// kernel (programmatic dependent launch), because the weights never depend
+// on it; under 100 KB of shared memory per CTA lets the next kernel's CTA sit
+// on the same SM and do the same.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -24,13 +33,19 @@
 namespace bitnet {
 
 constexpr int kGemvWarps = 8;
-constexpr int kGemvRows = 4;       // rows per group
-constexpr int kGemvSlots = 4;      // ring depth per warp
-constexpr int kGemvKChunk = 4096;  // weights per row per slot
-constexpr int kGemvSlotBytes = kGemvRows * kGemvKChunk / 4;
-constexpr int kGemvSmemBytes = kGemvWarps * kGemvSlots * kGemvSlotBytes + kGemvWarps * kGemvSlots * 8;
+constexpr int kGemvRows = 4;                                 // rows per group
+constexpr int kGemvSlots = 2;                                // ring depth per warp
+constexpr int kGemvSlotBytes = 4096;                         // one item: 4 rows x 1 KB
+constexpr int kGemvKChunk = kGemvSlotBytes * 4 / kGemvRows;  // 4096 weights per row per item
+constexpr int kGemvRingBytes = kGemvWarps * kGemvSlots * kGemvSlotBytes;
+constexpr int kGemvXMaxBytes = 21504;  // x_q is staged in shared memory when M*K fits
+constexpr int kGemvBarBytes = 256;
 
-template <int MT, bool U8>
+__host__ __device__ constexpr int gemv_smem_bytes(bool xs) {
+  return kGemvRingBytes + kGemvBarBytes + (xs ? kGemvXMaxBytes : 0);
+}
+
+template <int MT, bool U8, bool XS>
 __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __restrict__ Wp,
                                                                const float* __restrict__ gamma_ptr, int N, int K,
                                                                const int8_t* __restrict__ xq,
@@ -40,7 +55,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __
   extern __shared__ __align__(1024) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint8_t* ring = smem + warp * kGemvSlots * kGemvSlotBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGemvWarps * kGemvSlots * kGemvSlotBytes) + warp * kGemvSlots;
+  uint64_t* all_bars = reinterpret_cast<uint64_t*>(smem + kGemvRingBytes);
+  uint64_t* bars = all_bars + warp * kGemvSlots;
+  uint64_t* xbar = all_bars + kGemvWarps * kGemvSlots;
+  uint8_t* xs = smem + kGemvRingBytes + kGemvBarBytes;
 
   const int64_t row_lo = static_cast<int64_t>(N) * blockIdx.x / gridDim.x;
   const int64_t row_hi = static_cast<int64_t>(N) * (blockIdx.x + 1) / gridDim.x;
@@ -49,13 +67,15 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __
   const int kchunk = K < kGemvKChunk ? K : kGemvKChunk;
   const int nkc = (K + kchunk - 1) / kchunk;
   const int items = my_groups * nkc;
-  const int row_bytes = K >> 2;
+  const int64_t row_bytes = K >> 2;
+  const int slot_row = kchunk >> 2;  // bytes per row inside a slot
 
   if (lane == 0) {
     for (int s = 0; s < kGemvSlots; ++s) mbar_init(&bars[s], 1);
+    if (warp == 0) mbar_init(xbar, 1);
     fence_barrier_init();
   }
-  __syncwarp();
+  __syncthreads();
 
   const uint64_t policy = policy_evict_first();
   // Issue item j into ring slot j % kGemvSlots (lane 0 only).
@@ -69,17 +89,37 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __
     uint64_t* bar = &bars[j % kGemvSlots];
     uint8_t* dst = ring + (j % kGemvSlots) * kGemvSlotBytes;
     mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nr * len));
-    for (int r = 0; r < nr; ++r)
-      bulk_copy_g2s(dst + r * (kchunk >> 2), Wp + (r0 + r) * row_bytes + (k0 >> 2), static_cast<uint32_t>(len), bar,
-                    policy);
+    if (len == row_bytes) {
+      // whole rows: the group's rows are contiguous in memory, one copy
+      bulk_copy_g2s(dst, Wp + r0 * row_bytes, static_cast<uint32_t>(nr * len), bar, policy);
+    } else {
+      for (int r = 0; r < nr; ++r)
+        bulk_copy_g2s(dst + r * slot_row, Wp + (r0 + r) * row_bytes + (k0 >> 2), static_cast<uint32_t>(len), bar,
+                      policy);
+    }
   };
   if (lane == 0)
     for (int j = 0; j < kGemvSlots && j < items; ++j) issue(j);
 
   // Everything below reads the outputs of the previous kernel.
-  pdl_wait();
   pdl_launch_dependents();
-  const float gamma = *gamma_ptr;
+  pdl_wait();
+  if constexpr (XS) {
+    if (warp == 0 && lane == 0) {
+      mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(MT * K));
+      bulk_copy_g2s(xs, xq, static_cast<uint32_t>(MT * K), xbar, policy_evict_last());
+    }
+  }
+  const float gamma = __ldg(gamma_ptr);
+  float asc[MT];
+  int rsum[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    asc[m] = __ldg(a_scale + m);
+    rsum[m] = U8 ? __ldg(rowsum + m) : 0;
+  }
+  bool xok = true;
+  if constexpr (XS) xok = __all_sync(0xffffffffu, mbar_wait(xbar, 0));
 
   int acc[kGemvRows][MT];
 #pragma unroll
@@ -87,8 +127,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __
 #pragma unroll
     for (int m = 0; m < MT; ++m) acc[r][m] = 0;
 
-  int failed_at = -1;
-  for (int j = 0; j < items; ++j) {
+  int failed_at = xok ? -1 : 0;
+  for (int j = 0; xok && j < items; ++j) {
     const int slot = j % kGemvSlots;
     // Every lane acquires the barrier itself; the warp leaves together if any gave up.
     const bool got = mbar_wait(&bars[slot], (j / kGemvSlots) & 1);
@@ -99,39 +139,35 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __
     const int gi = j / nkc, kc = j - gi * nkc;
     const int k0 = kc * kchunk;
     const int len = min(kchunk, K - k0);  // weights per row in this item
-    const uint32_t sbase = smem_addr(ring + slot * kGemvSlotBytes);
-    for (int ci = lane; ci < (len >> 6); ci += 32) {
-      // 64 weights per row: 16 bytes of codes per row, 64 bytes of x per token.
-      uint32_t wq[kGemvRows][16];
-#pragma unroll
-      for (int r = 0; r < kGemvRows; ++r) {
-        const uint4 p = lds128(sbase + r * (kchunk >> 2) + ci * 16);
-        const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
-#pragma unroll
-        for (int wi = 0; wi < 4; ++wi)
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            const uint32_t c4 = (pw[wi] >> (2 * jj)) & 0x03030303u;
-            wq[r][4 * wi + jj] = U8 ? c4 : codes_to_signed(c4);
-          }
-      }
+    const uint32_t sw = smem_addr(ring + slot * kGemvSlotBytes);
+#pragma unroll 1
+    for (int kk = lane * 16; kk < len; kk += 512) {
+      // This lane: weights k0+kk .. k0+kk+15 of the 4 rows.
+      uint32_t xv[MT][4];
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
-        const uint4* xp = reinterpret_cast<const uint4*>(xq + static_cast<int64_t>(m) * K + k0 + ci * 64);
-        uint32_t xv[16];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 u = __ldg(xp + q);
-          xv[4 * q + 0] = u.x;
-          xv[4 * q + 1] = u.y;
-          xv[4 * q + 2] = u.z;
-          xv[4 * q + 3] = u.w;
+        uint4 u;
+        if constexpr (XS) {
+          u = lds128(smem_addr(xs) + m * K + k0 + kk);
+        } else {
+          u = __ldg(reinterpret_cast<const uint4*>(xq + static_cast<int64_t>(m) * K + k0 + kk));
         }
+        xv[m][0] = u.x;
+        xv[m][1] = u.y;
+        xv[m][2] = u.z;
+        xv[m][3] = u.w;
+      }
 #pragma unroll
-        for (int r = 0; r < kGemvRows; ++r)
+      for (int r = 0; r < kGemvRows; ++r) {
+        uint32_t w;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(sw + r * slot_row + (kk >> 2)));
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            acc[r][m] = U8 ? dp4a_us(wq[r][e], xv[e], acc[r][m]) : dp4a_ss(wq[r][e], xv[e], acc[r][m]);
+        for (int jj = 0; jj < 4; ++jj) {
+          const uint32_t c4 = (w >> (2 * jj)) & 0x03030303u;
+#pragma unroll
+          for (int m = 0; m < MT; ++m)
+            acc[r][m] = U8 ? dp4a_us(c4, xv[m][jj], acc[r][m]) : dp4a_ss(codes_to_signed(c4), xv[m][jj], acc[r][m]);
+        }
       }
     }
     __syncwarp();
@@ -156,12 +192,12 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
           if (lane == r * MT + m && r0 + r < row_hi) {
-            const int a = U8 ? acc[r][m] - __ldg(rowsum + m) : acc[r][m];
+            const int a = acc[r][m] - rsum[m];
             const int64_t o = static_cast<int64_t>(m) * N + r0 + r;
             if (y_dtype == 2) {
               static_cast<int32_t*>(y)[o] = a;
             } else {
-              const float v = __fmul_rn(__fmul_rn(__int2float_rn(a), gamma), __ldg(a_scale + m));
+              const float v = __fmul_rn(__fmul_rn(__int2float_rn(a), gamma), asc[m]);
               if (y_dtype == 0) static_cast<float*>(y)[o] = v;
               else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
             }
@@ -174,6 +210,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __
     // Let copies still in flight land before the CTA's shared memory goes away.
     for (int j = failed_at; j < items && j < failed_at + kGemvSlots; ++j)
       mbar_wait(&bars[j % kGemvSlots], (j / kGemvSlots) & 1);
+    if (XS && warp == 0) mbar_wait(xbar, 0);
   }
 }
 
