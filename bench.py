@@ -4,9 +4,11 @@
                     [--workload NAME]
 
 One step = one pass of the whole hot path over one batch: for every linear
-of the workload, the fused RMSNorm/absmax int8 quantisation of its input and
-the W1.58A8 product with dequant epilogue (decode GEMV for M <= 8, tcgen05
-GEMM otherwise).  Weight packing (absmean ternarisation) is the offline
+of the workload, the RMSNorm/absmax int8 quantisation of its input and the
+W1.58A8 product with dequant epilogue.  Decode shapes (M <= 8) run it as one
+kernel per linear (bitnet_bitlinear_gemv); the two-kernel path
+(bitnet_quant_act + bitnet_linear_gemv) is timed alongside under
+"unfused_step".  Larger batches use bitnet_quant_act + the tcgen05 GEMM.  Weight packing (absmean ternarisation) is the offline
 step: it runs once before timing and is reported separately under "stages".
 
 Timed region: W untimed warm-up steps, then exactly K steps replayed from
@@ -306,10 +308,22 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
         fn = bl.bitnet_linear_gemv if lin.M <= 8 else bl.bitnet_linear_gemm
         fn(packs[i][0][c % COPIES], packs[i][1], b["xq"], b["a"], b["rs"], y=b["y"])
 
-    def step(c):
+    def fused(i, c):
+        # quantisation + product in one kernel (decode shapes)
+        b = bufs[i]
+        bl.bitnet_bitlinear_gemv(xs[i], packs[i][0][c % COPIES], packs[i][1], gains[i], EPS_RMS, y=b["y"])
+
+    def step_unfused(c):
         for i in range(len(lins)):
             quant(i, c)
             product(i, c)
+
+    def step_fused(c):
+        for i in range(len(lins)):
+            fused(i, c)
+
+    use_fused = all(l.M <= 8 and l.M * l.K <= 21504 for l in lins)
+    step = step_fused if use_fused else step_unfused
 
     def capture(fn_per_step, nsteps: int, start: int = 0):
         g = torch.cuda.CUDAGraph()
@@ -346,7 +360,7 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
             g_warm.replay()
     torch.cuda.synchronize(dev)
     # the timed region: exactly K steps
-    kernels_per_step = 2 * len(lins)
+    kernels_per_step = (1 if use_fused else 2) * len(lins)
     with ClockSampler(dev.index) as clocks:
         barrier(group, dev)
         torch.cuda.synchronize(dev)
@@ -377,16 +391,44 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
 
     prod_ms = per_stage(product, "product")
     quant_ms = per_stage(quant, "quant")
+    fused_ms = per_stage(fused, "fused") if use_fused else None
     prod_bytes = statistics.mean(linear_bytes(l)["product"] for l in lins)
     quant_bytes = statistics.mean(linear_bytes(l)["quant"] for l in lins)
     hbm_peak = float(peaks["hbm_gbs"])
-    src = kernel_source_hash(["gemv.cuh", "ptx.cuh"] if lins[0].M <= 8 else ["gemm.cuh", "ptx.cuh"])
-    traffic = profiled_traffic(PROFILE_SUMMARY, src) if lins[0].M <= 8 else None
-    achieved = prod_bytes / (prod_ms / 1e3) / 1e9
+    if use_fused:
+        # the dominant (only) kernel of the step: fused quantisation + GEMV;
+        # its algorithmic bytes: x in, packed W, scales, y out
+        kern, kern_ms = "gemv_kernel (fused quant + GEMV, bitnet_bitlinear_gemv)", fused_ms
+        kern_bytes = statistics.mean(linear_bytes(l)["x_in"] + l.N * l.K // 4 + 4 + linear_bytes(l)["y_out"]
+                                     for l in lins)
+        src = kernel_source_hash(["gemv.cuh", "quant.cuh", "ptx.cuh"])
+    elif lins[0].M <= 8:
+        kern, kern_ms, kern_bytes = "gemv_kernel", prod_ms, prod_bytes
+        src = kernel_source_hash(["gemv.cuh", "ptx.cuh"])
+    else:
+        kern, kern_ms, kern_bytes = "gemm_kernel", prod_ms, prod_bytes
+        src = kernel_source_hash(["gemm.cuh", "ptx.cuh"])
+    traffic = profiled_traffic(PROFILE_SUMMARY, src)
+    achieved = kern_bytes / (kern_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-                "traffic": traffic, "kernel": "gemv_kernel" if lins[0].M <= 8 else "gemm_kernel",
+                "traffic": traffic, "kernel": kern,
                 "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)" if peak_src == "measured" else
-                "fallback 6650 GB/s", "launch_us": prod_ms * 1e3, "bytes_per_launch": prod_bytes}
+                "fallback 6650 GB/s", "launch_us": kern_ms * 1e3, "bytes_per_launch": kern_bytes,
+                "how": "back-to-back launches of this kernel alone in CUDA graphs over the rotating weight copies, "
+                       "CUDA events on the launching stream; average time per launch"}
+
+    # ---- the other path over the same K steps (four-call path when the fused one is timed above)
+    unfused = None
+    if use_fused:
+        gu = capture(step_unfused, G)
+        with torch.cuda.stream(stream):
+            gu.replay()
+        torch.cuda.synchronize(dev)
+        reps = max(1, K // G)
+        ms = max_over_ranks(time_graph(gu, reps), group, dev)
+        unfused = {"value": ws * reps * G * step_bytes / (ms / 1e3) / 1e9, "unit": "GB/s",
+                   "ms_per_step": ms / (reps * G), "steps": reps * G, "kernels_per_step": 2 * len(lins),
+                   "what": "bitnet_quant_act + bitnet_linear_gemv per linear (two kernels)"}
 
     # ---- end to end through the public API with host buffers
     h2d = sum(linear_bytes(l)["x_in"] for l in lins)
@@ -398,8 +440,11 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
     def e2e_step(c):
         for i, lin in enumerate(lins):
             xs[i].copy_(xs_host[i], non_blocking=True)
-            quant(i, c)
-            product(i, c)
+            if use_fused:
+                fused(i, c)
+            else:
+                quant(i, c)
+                product(i, c)
             ys_host[i].copy_(bufs[i]["y"], non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -417,8 +462,8 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), group, dev)
     e2e = {"value": ws * k_e2e * step_bytes / (e2e_ms / 1e3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "steps": k_e2e,
-           "how": "eager Python calls of the public API per step: pinned H2D copy of every input, quant + product, "
-                  "D2H copy of every output"}
+           "how": "eager Python calls of the public API per step: pinned H2D copy of every input, the BitLinear "
+                  "call(s), D2H copy of every output"}
 
     # ---- prefill tensor-core GEMM (M = 4096), a secondary line of the same metric
     prefill = None
@@ -445,7 +490,9 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
             "ms_per_step": el_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "int8", "data": "synthetic",
             "config": {"workload": args.workload, "linears": [[l.M, l.K, l.N] for l in lins],
-                       "step": "per linear: fused quant of its input + ternary product with dequant",
+                       "step": ("per linear: one bitnet_bitlinear_gemv kernel (RMSNorm/absmax int8 quantisation of "
+                                "the input fused with the ternary GEMV and dequant)") if use_fused else
+                               "per linear: bitnet_quant_act + ternary product with dequant",
                        "l2": f"{COPIES} rotating packed-weight copies per linear "
                              f"({COPIES * sum(l.N * l.K // 4 for l in lins) / 1e6:.0f} MB > 126 MB L2)",
                        "timing": f"CUDA graphs of {G} steps, programmatic dependent launch between kernels",
@@ -455,8 +502,10 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
             "e2e": e2e,
             "gpu_launches": K * kernels_per_step,
             "clocks": clk,
+            "unfused_step": unfused,
             "stages": {"quant_us_per_launch": quant_ms * 1e3, "quant_gbs": quant_bytes / (quant_ms / 1e3) / 1e9,
                        "product_us_per_launch": prod_ms * 1e3,
+                       "fused_us_per_launch": None if fused_ms is None else fused_ms * 1e3,
                        "pack_ms": pack_ms, "pack_gbs": [l.N * l.K * 4.25 / (ms / 1e3) / 1e9
                                                         for l, ms in zip(lins, pack_ms)]},
             "prefill": prefill,

@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
             fn = getattr(L, name)
             fn.argtypes = [P, P, I64, I64, P, P, P, I64, P, I, P]
             fn.restype = I
+        L.bitnet_bitlinear_gemv.argtypes = [P, I, P, F, P, P, I64, I64, I64, P, I, P]
+        L.bitnet_bitlinear_gemv.restype = I
         L.bitnet_get_device_status.argtypes = [P]
         L.bitnet_get_device_status.restype = I
         L.bitnet_status_string.argtypes = [I]
@@ -195,6 +197,23 @@ def bitnet_linear_gemm(W_packed, gamma, x_q, a_scale, x_rowsum=None, y=None, out
     return _linear("bitnet_linear_gemm", W_packed, gamma, x_q, a_scale, x_rowsum, y, out_dtype)
 
 
+def bitnet_bitlinear_gemv(x, W_packed, gamma, rms_gain=None, rms_eps: float = 1e-5, y=None, out_dtype=None):
+    """Fused decode BitLinear (M <= 8): quantisation (with RMSNorm when
+    rms_gain is given) and the ternary product in one kernel.  Returns y."""
+    torch = _torch()
+    _need_cuda(x, rms_gain, W_packed, gamma, y)
+    M, K = x.shape
+    N = W_packed.shape[0]
+    if W_packed.shape[1] * 4 != K:
+        raise ValueError("x and W_packed disagree on K")
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype or torch.bfloat16, device=x.device)
+    st = lib().bitnet_bitlinear_gemv(_ptr(x), _dtype_code(x.dtype), _ptr(rms_gain), rms_eps, _ptr(W_packed),
+                                     _ptr(gamma), N, K, M, _ptr(y), _dtype_code(y.dtype), _stream(x.device))
+    _check("bitnet_bitlinear_gemv", st)
+    return y
+
+
 def bitnet_get_device_status(device=None) -> int:
     """Synchronises the current stream and returns (and clears) the device error status."""
     torch = _torch()
@@ -204,7 +223,11 @@ def bitnet_get_device_status(device=None) -> int:
 
 def bitlinear(x, W_packed, gamma, rms_gain=None, rms_eps: float = 1e-5, out_dtype=None):
     """One BitLinear forward: quantise x (fused RMSNorm when rms_gain is given),
-    then the ternary product with dequant.  Picks the decode kernel for M <= 8."""
+    then the ternary product with dequant.  Uses the fused decode kernel for
+    M <= 8 when the quantised rows fit its shared memory."""
+    M, K = x.shape
+    if M <= 8 and M * K <= 21504:
+        return bitnet_bitlinear_gemv(x, W_packed, gamma, rms_gain, rms_eps, out_dtype=out_dtype)
     x_q, a, rs = bitnet_quant_act(x, rms_gain, rms_eps, want_rowsum=True)
     if x.shape[0] <= 8:
         return bitnet_linear_gemv(W_packed, gamma, x_q, a, rs, out_dtype=out_dtype)

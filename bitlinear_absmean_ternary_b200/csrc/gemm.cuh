@@ -11,15 +11,16 @@
 //       32*(w%4)..+31, so thread t of warp w owns weight row 32*(w%4)+t.
 //   B = int8 activations, BN tokens x 128 K per stage, loaded by TMA into
 //       shared memory in the 128-byte swizzled K-major layout the MMA reads.
-//   D = int32 accumulator, 128 lanes x BN columns of TMEM, double-buffered.
+//   D = int32 accumulator, 128 lanes x BN columns of TMEM, double-buffered
+//       when two fit next to the A slots (BN <= 128), single otherwise.
 // Packed weights arrive by TMA too (128 rows x 32 bytes per stage, 32-byte
 // swizzle, which makes the unpack warps' 16-byte reads bank-conflict free).
 // With the per-token sums of x_q available, A holds the unsigned codes
 // c = q + 1 and the epilogue subtracts rowsum[m] (sum c*x - sum x = sum q*x).
 //
 // Persistent: one CTA per SM walks tiles t = blockIdx.x, +gridDim.x, ...
-// (weight-row tiles fastest).  Warp roles (448 threads):
-//   warp 0, lane 0   TMA producer over a STAGES-deep ring;
+// (weight-row tiles fastest).  Warp roles:
+//   warp 0 and warps 14.., lane 0   TMA producers over an S-deep ring;
 //   warp 1           TMEM allocator; lane 0 issues the MMAs;
 //   warps 2..9       unpack: two warps per TMEM lane quarter, taking
 //                    alternate stages;
@@ -43,36 +44,45 @@ namespace bitnet {
 
 constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 128;  // K bytes per stage = 4 MMAs of K = 32
-constexpr int kGemmStages = 8;
 constexpr int kGemmUnpackWarps = 8;
 constexpr int kGemmEpiWarps = 4;
-constexpr int kGemmThreads = (2 + kGemmUnpackWarps + kGemmEpiWarps) * 32;
+// TMA issue warps: one issuing thread streams a stage roughly every 270 ns
+// whatever its size, so several warps share the ring (warp p issues the
+// stages g with g % kGemmProducers == p).
+constexpr int kGemmProducers = 2;
+constexpr int kGemmThreads = (1 + kGemmProducers + kGemmUnpackWarps + kGemmEpiWarps) * 32;
 
-template <int BN>
+// BN tokens per tile, S ring stages.  TMEM holds the accumulator(s) (BN
+// columns each; two when they fit, so the epilogue of one tile overlaps the
+// MMAs of the next) and one 32-column A slot per stage.
+template <int BN, int S>
 struct GemmCfg {
   static constexpr int kXBytes = BN * kGemmBK;           // activation tile
   static constexpr int kWBytes = kGemmBM * kGemmBK / 4;  // packed weight tile
   static constexpr int kStageBytes = kXBytes + kWBytes;  // multiple of 1024
-  static constexpr int kTmemCols = 512;                  // 2 accumulators + A slots
-  static constexpr int kAcol = 2 * BN;                   // first A slot column
-  static constexpr int kBarOffset = kGemmStages * kStageBytes;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kBufs = 2 * BN + 32 * S <= kTmemCols ? 2 : 1;
+  static constexpr int kAcol = kBufs * BN;  // first A slot column
+  static constexpr int kBarOffset = S * kStageBytes;
   static constexpr int kNeeded = 1024 + kBarOffset + 256;
   // The CTA holds all 512 TMEM columns: ask for enough shared memory that a
   // second CTA never fits on the SM (228 KB), so none waits in tcgen05.alloc.
   static constexpr int kMinSmem = 233472 / 2;
   static constexpr int kSmemBytes = kNeeded > kMinSmem ? kNeeded : kMinSmem;
   static_assert(kStageBytes % 1024 == 0, "stage tiles must stay 1024-byte aligned");
-  static_assert(kAcol + kGemmStages * 32 <= kTmemCols, "TMEM budget");
-  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 128, "MMA N");
+  static_assert(kAcol + S * 32 <= kTmemCols, "TMEM budget");
+  static_assert(kNeeded <= 232448, "shared memory budget");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+  static_assert(S % kGemmProducers == 0, "each ring slot belongs to one producer");
 };
 
-template <int BN, bool U8>
+template <int BN, int S, bool U8>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                 const float* __restrict__ gamma_ptr, const float* __restrict__ a_scale,
                 const int32_t* __restrict__ rowsum, int M, int N, int K, void* __restrict__ y, int y_dtype) {
-  using C = GemmCfg<BN>;
-  constexpr int S = kGemmStages;
+  using C = GemmCfg<BN, S>;
+  constexpr int NB = C::kBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
@@ -113,7 +123,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem = *tmem_holder;
   pdl_launch_dependents();
 
-  if (warp == 0) {
+  const int prod = warp == 0 ? 0 : warp - (1 + kGemmUnpackWarps + kGemmEpiWarps);  // producer index or < 1
+  if (warp == 0 || warp >= 2 + kGemmUnpackWarps + kGemmEpiWarps) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA producer
       // The weights never depend on the previous kernel: the first ring's
@@ -121,16 +132,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int my_tiles = blockIdx.x < tiles ? (tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
       const int total = my_tiles * nk;
       const int pre = total < S ? total : S;
-      for (int g = 0; g < pre; ++g) {
+      for (int g = prod; g < pre; g += kGemmProducers) {
         const int t = blockIdx.x + (g / nk) * gridDim.x, kb = g % nk;
         mbar_arrive_expect_tx(&full[g], C::kStageBytes);
         tma_load_2d(smem + g * C::kStageBytes + C::kXBytes, &tmap_w, kb * (kGemmBK / 4), (t % n_tiles) * kGemmBM,
                     &full[g]);
       }
       pdl_wait();
-      int issued = 0;
+      int issued = prod;
       bool ok = true;
-      for (int g = 0; g < total; ++g) {
+      for (int g = prod; g < total; g += kGemmProducers) {
         const int s = g % S;
         const int t = blockIdx.x + (g / nk) * gridDim.x, kb = g % nk;
         const int n0 = (t % n_tiles) * kGemmBM, m0 = (t / n_tiles) * BN;
@@ -144,12 +155,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_load_2d(xs + C::kXBytes, &tmap_w, kb * (kGemmBK / 4), n0, &full[s]);
         }
         tma_load_2d(xs, &tmap_x, kb * kGemmBK, m0, &full[s]);
-        issued = g + 1;
+        issued = g + kGemmProducers;
       }
       if (!ok) {
         // weight tiles were requested for stages up to max(issued, pre)
         const int last = issued > pre ? issued : pre;
-        for (int g = last > S ? last - S : 0; g < last; ++g) mbar_wait(&full[g % S], (g / S) & 1);
+        for (int g = prod; g < last; g += kGemmProducers)
+          if (g + S >= last) mbar_wait(&full[g % S], (g / S) & 1);
       }
     }
   } else if (warp == 1) {
@@ -159,8 +171,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       bool ok = true;
       int g = 0, tc = 0;
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++tc) {
-        const int b = tc & 1;
-        if (!mbar_wait(&accempty[b], ((tc >> 1) & 1) ^ 1)) {
+        const int b = tc % NB;
+        if (!mbar_wait(&accempty[b], ((tc / NB) & 1) ^ 1)) {
           ok = false;
           break;
         }
@@ -224,8 +236,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const float gamma = __ldg(gamma_ptr);
     int tc = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++tc) {
-      const int b = tc & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&accfull[b], (tc >> 1) & 1))) break;
+      const int b = tc % NB;
+      if (!__all_sync(0xffffffffu, mbar_wait(&accfull[b], (tc / NB) & 1))) break;
       tc_fence_after();
       const int n = (t % n_tiles) * kGemmBM + 32 * q + lane;
       const int m0 = (t / n_tiles) * BN;

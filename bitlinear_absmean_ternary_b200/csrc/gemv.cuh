@@ -29,6 +29,7 @@
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace bitnet {
 
@@ -45,13 +46,23 @@ __host__ __device__ constexpr int gemv_smem_bytes(bool xs) {
   return kGemvRingBytes + kGemvBarBytes + (xs ? kGemvXMaxBytes : 0);
 }
 
-template <int MT, bool U8, bool XS>
+// FUSED: the kernel takes the unquantised activations x (M x K of type T)
+// and the optional RMSNorm gain instead of x_q / a_scale / rowsum, and
+// quantises every token row itself, with all 256 threads, straight into its
+// shared-memory copy of x_q (quant_row_cta: the same arithmetic and order as
+// the standalone quantisation kernel).  Every CTA repeats this small step
+// (M*K <= 21504 values, read from L2), which removes a dependent kernel
+// launch and the x_q round trip through global memory from each decode
+// linear.
+template <int MT, bool U8, bool XS, bool FUSED = false, typename T = float, int MAXC = 1>
 __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __restrict__ Wp,
                                                                const float* __restrict__ gamma_ptr, int N, int K,
                                                                const int8_t* __restrict__ xq,
                                                                const float* __restrict__ a_scale,
-                                                               const int32_t* __restrict__ rowsum, void* __restrict__ y,
-                                                               int y_dtype) {
+                                                               const int32_t* __restrict__ rowsum,
+                                                               const T* __restrict__ xin, const T* __restrict__ gain,
+                                                               float rms_eps, void* __restrict__ y, int y_dtype) {
+  static_assert(!FUSED || (XS && U8), "the fused kernel keeps x_q in shared memory and uses its row sums");
   extern __shared__ __align__(1024) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint8_t* ring = smem + warp * kGemvSlots * kGemvSlotBytes;
@@ -104,7 +115,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __
   // Everything below reads the outputs of the previous kernel.
   pdl_launch_dependents();
   pdl_wait();
-  if constexpr (XS) {
+  if constexpr (XS && !FUSED) {
     if (warp == 0 && lane == 0) {
       mbar_arrive_expect_tx(xbar, static_cast<uint32_t>(MT * K));
       bulk_copy_g2s(xs, xq, static_cast<uint32_t>(MT * K), xbar, policy_evict_last());
@@ -113,13 +124,26 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __
   const float gamma = __ldg(gamma_ptr);
   float asc[MT];
   int rsum[MT];
-#pragma unroll
-  for (int m = 0; m < MT; ++m) {
-    asc[m] = __ldg(a_scale + m);
-    rsum[m] = U8 ? __ldg(rowsum + m) : 0;
-  }
   bool xok = true;
-  if constexpr (XS) xok = __all_sync(0xffffffffu, mbar_wait(xbar, 0));
+  if constexpr (FUSED) {
+    __shared__ QuantScratch qsc;
+#pragma unroll 1
+    for (int m = 0; m < MT; ++m) {
+      float amax;
+      int sum;
+      quant_row_cta<T, MAXC>(xin + static_cast<int64_t>(m) * K, K, gain, rms_eps,
+                             reinterpret_cast<int8_t*>(xs) + m * K, qsc, amax, sum);
+      asc[m] = amax == 0.0f ? 0.0f : __fdiv_rn(amax, 127.0f);
+      rsum[m] = sum;
+    }
+  } else {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      asc[m] = __ldg(a_scale + m);
+      rsum[m] = U8 ? __ldg(rowsum + m) : 0;
+    }
+    if constexpr (XS) xok = __all_sync(0xffffffffu, mbar_wait(xbar, 0));
+  }
 
   int acc[kGemvRows][MT];
 #pragma unroll
@@ -210,7 +234,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __
     // Let copies still in flight land before the CTA's shared memory goes away.
     for (int j = failed_at; j < items && j < failed_at + kGemvSlots; ++j)
       mbar_wait(&bars[j % kGemvSlots], (j / kGemvSlots) & 1);
-    if (XS && warp == 0) mbar_wait(xbar, 0);
+    if (XS && !FUSED && warp == 0) mbar_wait(xbar, 0);
   }
 }
 

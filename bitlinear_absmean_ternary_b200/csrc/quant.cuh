@@ -2,8 +2,8 @@
 // precedes it (comrad404.com review, "Метод: как устроен BitNet b1.58":
 // 8-bit activations; RMSNorm; "normalise the input, then quantise").
 //
-// One CTA of 256 threads per token row; thread t owns the 8-element chunks
-// c = t, t+256, ... and keeps them in registers, so x is read from HBM once.
+// 256 threads per token row; thread t owns the 8-element chunks c = t,
+// t+256, ... and keeps them in registers, so x is read from HBM once.
 // The sum of squares uses the fixed order of the oracle: each thread adds
 // RN32(v*v) over its chunks in increasing k, then the halving tree
 // l += l+128, +64, +32 (shared memory), +16 .. +1 (shuffles).
@@ -51,22 +51,22 @@ struct Chunk8<float> {
 
 constexpr int kQuantThreads = 256;
 
-template <typename T, int MAXC>
-__global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(const T* __restrict__ x, int K,
-                                                                  const T* __restrict__ gain, float rms_eps,
-                                                                  int8_t* __restrict__ xq, float* __restrict__ a_out,
-                                                                  int32_t* __restrict__ rowsum_out) {
-  __shared__ float red[kQuantThreads];
-  __shared__ float bcast;
-  __shared__ int ired[kQuantThreads / 32];
+struct QuantScratch {
+  float red[kQuantThreads];
+  float bcast;
+  int ired[kQuantThreads / 32];
+};
 
+// Quantises one token row with the 256 threads of the CTA (all must call it).
+// Thread t owns the 8-element chunks c = t, t+256, ... and keeps them in
+// registers, so the row is read once.  Writes x_q through xq_row (global or
+// shared memory); returns max|h| and sum(x_q) to every thread.
+template <typename T, int MAXC>
+BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict__ gain, float rms_eps,
+                          int8_t* xq_row, QuantScratch& sc, float& amax_out, int& sum_out) {
   const int t = threadIdx.x;
   const int lane = t & 31, warp = t >> 5;
-  const int64_t m = blockIdx.x;
   const int nchunks = K >> 3;
-  const T* row = x + m * K;
-
-  pdl_wait();
 
   Chunk8<T> ch[MAXC];
 #pragma unroll
@@ -89,15 +89,15 @@ __global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(const T* __res
         }
       }
     }
-    red[t] = ss;
+    sc.red[t] = ss;
     __syncthreads();
 #pragma unroll
     for (int s = kQuantThreads / 2; s >= 32; s >>= 1) {
-      if (t < s) red[t] = __fadd_rn(red[t], red[t + s]);
+      if (t < s) sc.red[t] = __fadd_rn(sc.red[t], sc.red[t + s]);
       __syncthreads();
     }
     if (warp == 0) {
-      float p = red[lane];
+      float p = sc.red[lane];
 #pragma unroll
       for (int s = 16; s >= 1; s >>= 1) {
         const float o = __shfl_down_sync(0xffffffffu, p, s);
@@ -105,11 +105,11 @@ __global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(const T* __res
       }
       if (lane == 0) {
         const float ms = __fdiv_rn(p, static_cast<float>(K));
-        bcast = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, rms_eps)));
+        sc.bcast = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, rms_eps)));
       }
     }
     __syncthreads();
-    r = bcast;
+    r = sc.bcast;
   }
 
   // h = RN32(RN32(v * r) * g) or v; amax = max |h| (order-free).
@@ -131,28 +131,22 @@ __global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(const T* __res
 #pragma unroll
   for (int s = 16; s >= 1; s >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, s));
   __syncthreads();  // red[] reuse
-  if (lane == 0) red[warp] = amax;
+  if (lane == 0) sc.red[warp] = amax;
   __syncthreads();
-  amax = red[0];
+  amax = sc.red[0];
 #pragma unroll
-  for (int w = 1; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, red[w]);
+  for (int w = 1; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, sc.red[w]);
 
   int sum = 0;
-  if (amax == 0.0f) {
+  const float s = amax == 0.0f ? 0.0f : __fdiv_rn(127.0f, amax);
 #pragma unroll
-    for (int i = 0; i < MAXC; ++i) {
-      const int c = t + kQuantThreads * i;
-      if (c < nchunks) *reinterpret_cast<uint2*>(xq + m * K + 8 * c) = make_uint2(0u, 0u);
-    }
-  } else {
-    const float s = __fdiv_rn(127.0f, amax);
-#pragma unroll
-    for (int i = 0; i < MAXC; ++i) {
-      const int c = t + kQuantThreads * i;
-      if (c < nchunks) {
+  for (int i = 0; i < MAXC; ++i) {
+    const int c = t + kQuantThreads * i;
+    if (c < nchunks) {
+      uint32_t lo = 0, hi = 0;
+      if (amax != 0.0f) {
         Chunk8<T> g;
         if (gain != nullptr) g.load(gain + 8 * c);
-        uint32_t lo = 0, hi = 0;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const float v = ch[i].get(e);
@@ -164,26 +158,38 @@ __global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(const T* __res
           if (e < 4) lo |= b << (8 * e);
           else hi |= b << (8 * (e - 4));
         }
-        *reinterpret_cast<uint2*>(xq + m * K + 8 * c) = make_uint2(lo, hi);
       }
+      *reinterpret_cast<uint2*>(xq_row + 8 * c) = make_uint2(lo, hi);
     }
   }
-  pdl_launch_dependents();
-
-  if (rowsum_out != nullptr) {
 #pragma unroll
-    for (int s = 16; s >= 1; s >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, s);
-    if (lane == 0) ired[warp] = sum;
-  }
+  for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) sc.ired[warp] = sum;
   __syncthreads();
-  if (t == 0) {
-    a_out[m] = amax == 0.0f ? 0.0f : __fdiv_rn(amax, 127.0f);
-    if (rowsum_out != nullptr) {
-      int tot = 0;
+  int tot = 0;
 #pragma unroll
-      for (int w = 0; w < kQuantThreads / 32; ++w) tot += ired[w];
-      rowsum_out[m] = tot;
-    }
+  for (int w = 0; w < kQuantThreads / 32; ++w) tot += sc.ired[w];
+  amax_out = amax;
+  sum_out = tot;
+  __syncthreads();  // scratch reuse by the next call
+}
+
+// Standalone kernel: one CTA per token row.
+template <typename T, int MAXC>
+__global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(const T* __restrict__ x, int K,
+                                                                  const T* __restrict__ gain, float rms_eps,
+                                                                  int8_t* __restrict__ xq, float* __restrict__ a_out,
+                                                                  int32_t* __restrict__ rowsum_out) {
+  __shared__ QuantScratch sc;
+  const int64_t m = blockIdx.x;
+  pdl_wait();
+  float amax;
+  int sum;
+  quant_row_cta<T, MAXC>(x + m * K, K, gain, rms_eps, xq + m * K, sc, amax, sum);
+  pdl_launch_dependents();
+  if (threadIdx.x == 0) {
+    a_out[m] = amax == 0.0f ? 0.0f : __fdiv_rn(amax, 127.0f);
+    if (rowsum_out != nullptr) rowsum_out[m] = sum;
   }
 }
 

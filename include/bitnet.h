@@ -184,6 +184,25 @@ bitnet_status bitnet_linear_gemm(const uint8_t* W_packed, const float* gamma, in
                                  int64_t M, void* y, int y_dtype, void* stream);
 
 /*
+ * Fused decode BitLinear: bitnet_quant_act followed by bitnet_linear_gemv in
+ * one kernel launch, for M <= 8 tokens.  Every CTA quantises the M token
+ * rows itself (same arithmetic and summation order as bitnet_quant_act) into
+ * its shared memory and then runs the GEMV, so the result is identical to
+ * the two-call path while saving a dependent kernel launch and the x_q round
+ * trip through global memory per linear (the four BitLinear steps of the
+ * comrad404.com review, section "Метод", in one pass).
+ *
+ * x, x_dtype, rms_gain, rms_eps   as bitnet_quant_act.
+ * W_packed, gamma, N, K, y, y_dtype   as bitnet_linear_gemv.
+ * 1 <= M <= 8 and M * K <= 21504 (the quantised rows live in shared memory);
+ * other shapes return BITNET_ERR_UNSUPPORTED_SHAPE (use the two calls).
+ * Asynchronous.
+ */
+bitnet_status bitnet_bitlinear_gemv(const void* x, int x_dtype, const void* rms_gain, float rms_eps,
+                                    const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, int64_t M,
+                                    void* y, int y_dtype, void* stream);
+
+/*
  * Synchronises `stream`, then reports and clears the device-side error word
  * that kernels set when a bounded wait on a barrier runs out (they then skip
  * their remaining work and exit instead of hanging).  Returns BITNET_OK,

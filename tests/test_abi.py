@@ -100,6 +100,23 @@ def test_linear_rejects_bad_arguments(L, name):
         assert call(M=9) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
 
 
+def test_fused_rejects_bad_arguments(L):
+    def call(x=FAKE, dt=bl.BITNET_BF16, g=None, eps=1e-5, W=FAKE, gam=FAKE, N=8, K=64, M=1, y=FAKE,
+             yd=bl.BITNET_BF16):
+        return L.bitnet_bitlinear_gemv(x, dt, g, eps, W, gam, N, K, M, y, yd, None)
+
+    assert call(x=None) == bl.BITNET_ERR_INVALID_ARG
+    assert call(W=MIS) == bl.BITNET_ERR_INVALID_ARG
+    assert call(dt=bl.BITNET_I32) == bl.BITNET_ERR_INVALID_ARG
+    assert call(yd=9) == bl.BITNET_ERR_INVALID_ARG
+    assert call(g=FAKE, eps=0.0) == bl.BITNET_ERR_INVALID_ARG
+    assert call(M=9) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(M=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(M=2, K=21504) == bl.BITNET_ERR_UNSUPPORTED_SHAPE  # quantised rows must fit in shared memory
+    assert call(K=100) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(N=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(bl, "_lib", None)
     monkeypatch.setattr(bl, "LIB_PATH", str(tmp_path / "missing.so"))

@@ -242,6 +242,47 @@ def test_gemv_and_gemm_agree(dev, orc):
         assert torch.equal(y1, y2)
 
 
+# --------------------------------------------------------------------------- fused decode BitLinear
+
+FUSED_CASES = [
+    # M, N, K, x dtype, norm, y dtype
+    (1, 6912, 2560, "bf16", False, "bf16"),
+    (1, 2560, 6912, "bf16", True, "f32"),
+    (1, 5376, 21504, "bf16", False, "bf16"),
+    (4, 256, 256, "f32", False, "f32"),
+    (8, 300, 2688, "bf16", True, "i32"),
+    (3, 129, 64, "f32", True, "bf16"),
+    (2, 1000, 4096, "bf16", False, "bf16"),
+]
+
+
+@pytest.mark.parametrize("M,N,K,dt,norm,yt", FUSED_CASES)
+def test_fused_bitlinear_gemv_parity(dev, orc, M, N, K, dt, norm, yt):
+    import torch
+    W = synth.weights(N, K, 0.02, M + N, 1)
+    x = synth.activations(M, K, M + K, 2, "normal", 0.01, 20.0, dt)
+    x[0, :3] = 0.0
+    g = synth.gain(K, 1, 3, dt) if norm else None
+    P, G = bl.bitnet_pack_weights(_t(W, dev), EPS_W)
+    p_ref, g_ref = orc.pack_weights(W, EPS_W)
+    xq_r, a_r, _ = orc.quant_act(x, g, EPS_RMS)
+    acc_r, y_r = orc.bitlinear(p_ref, g_ref, K, xq_r, a_r)
+    out = {"bf16": torch.bfloat16, "f32": torch.float32, "i32": torch.int32}[yt]
+    xd = _x_dev(x, dt, dev)
+    gd = None if g is None else _x_dev(g, dt, dev)
+    y = bl.bitnet_bitlinear_gemv(xd, P, G, gd, EPS_RMS, out_dtype=out)
+    if yt == "i32":
+        np.testing.assert_array_equal(y.cpu().numpy(), acc_r)
+    elif yt == "f32":
+        assert ulp_diff_f32(y.cpu().numpy(), y_r).max() == 0
+    else:
+        yb = y.view(torch.int16).cpu().numpy().view(np.uint16)
+        assert ulp_diff_bf16(yb, orc.f32_to_bf16(y_r)).max() == 0
+    # identical to the two-call path
+    xq, a, rs = bl.bitnet_quant_act(xd, gd, EPS_RMS, want_rowsum=True)
+    assert torch.equal(y, bl.bitnet_linear_gemv(P, G, xq, a, rs, out_dtype=out))
+
+
 # --------------------------------------------------------------------------- whole workloads
 
 _PACKED = {}
