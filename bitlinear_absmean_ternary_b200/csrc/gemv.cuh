@@ -10,20 +10,25 @@
 // instructions per four weights.
 //
 // Work split: CTA c owns the contiguous rows [N*c/G, N*(c+1)/G) (G = grid,
-// one CTA per SM); its warps take groups of 4 consecutive rows round-robin.
-// A group is streamed in items of up to 4096 weights per row (4 KB): lane 0
-// of the warp issues the bulk asynchronous copies of an item into a 2-slot
-// ring of shared memory owned by that warp.  The activations x_q (M*K bytes)
-// are copied into shared memory once per CTA when they fit.  Lane l handles
-// 16 consecutive weights of each of the 4 rows per 512-weight step, so the
-// warp's loads of codes (4 bytes per lane) and of activations (16 bytes per
-// lane) are contiguous and free of bank conflicts, and each activation load
-// serves 4 rows.  Lane partial sums are reduced with warp shuffles.
+// one CTA per SM).  Its rows are cut into groups of 4 and K into equal
+// chunks of at most 2560 weights; an item is one (group, chunk) pair, at most
+// 4 x 640 bytes of packed codes, and item j goes to warp j % 16, so short and
+// long rows both spread over all 16 warps.  Lane 0 of each warp streams the
+// warp's items with bulk asynchronous copies (L2 evict-first) into a 2-slot
+// ring of shared memory it owns.  The activations x_q (M*K bytes) sit in
+// shared memory, copied once per CTA.  Lane l handles 16 consecutive weights
+// of each of the 4 rows per 512-weight step, so the warp's loads of codes
+// (4 bytes per lane) and of activations (16 bytes per lane) are contiguous
+// and free of bank conflicts, and each activation load serves 4 rows.  A
+// warp reduces its partial sums with one redux per row and token and adds
+// them to the row's shared-memory accumulator (integer atomics: exact and
+// order-free); the rows' outputs are dequantised and stored once all items
+// of a wave of up to 256 rows are in.
 //
 // The first weight items are requested before waiting on the previous
 // kernel (programmatic dependent launch), because the weights never depend
-// on it; under 100 KB of shared memory per CTA lets the next kernel's CTA sit
-// on the same SM and do the same.
+// on it; about 110 KB of shared memory per CTA lets the next kernel's CTA
+// sit on the same SM and do the same.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -33,35 +38,42 @@
 
 namespace bitnet {
 
-constexpr int kGemvWarps = 8;
-constexpr int kGemvRows = 4;                                 // rows per group
-constexpr int kGemvSlots = 2;                                // ring depth per warp
-constexpr int kGemvSlotBytes = 4096;                         // one item: 4 rows x 1 KB
-constexpr int kGemvKChunk = kGemvSlotBytes * 4 / kGemvRows;  // 4096 weights per row per item
+constexpr int kGemvWarps = 16;
+constexpr int kGemvThreads = kGemvWarps * 32;
+constexpr int kGemvRows = 4;                                   // rows per group
+constexpr int kGemvSlots = 2;                                  // ring depth per warp
+constexpr int kGemvKChunkMax = 2560;                           // weights per row per item
+constexpr int kGemvSlotBytes = kGemvRows * kGemvKChunkMax / 4;  // 2560 bytes
 constexpr int kGemvRingBytes = kGemvWarps * kGemvSlots * kGemvSlotBytes;
-constexpr int kGemvXMaxBytes = 21504;  // x_q is staged in shared memory when M*K fits
-constexpr int kGemvBarBytes = 256;
+constexpr int kGemvBarBytes = 512;
+constexpr int kGemvWaveRows = 256;                             // rows accumulated in shared memory at a time
+constexpr int kGemvXMaxBytes = 21504;                          // x_q is staged in shared memory when M*K fits
 
-__host__ __device__ constexpr int gemv_smem_bytes(bool xs) {
-  return kGemvRingBytes + kGemvBarBytes + (xs ? kGemvXMaxBytes : 0);
+__host__ __device__ constexpr int gemv_smem_bytes(int mt, int k, bool xs) {
+  return kGemvRingBytes + kGemvBarBytes + kGemvWaveRows * mt * 4 + (xs ? ((mt * k + 15) / 16) * 16 : 0);
+}
+
+// Equal K-chunks of at most kGemvKChunkMax weights, multiples of 64.
+__host__ __device__ constexpr int gemv_kchunk(int K) {
+  return ((K + (K + kGemvKChunkMax - 1) / kGemvKChunkMax - 1) / ((K + kGemvKChunkMax - 1) / kGemvKChunkMax) + 63) /
+         64 * 64;
 }
 
 // FUSED: the kernel takes the unquantised activations x (M x K of type T)
 // and the optional RMSNorm gain instead of x_q / a_scale / rowsum, and
-// quantises every token row itself, with all 256 threads, straight into its
-// shared-memory copy of x_q (quant_row_cta: the same arithmetic and order as
-// the standalone quantisation kernel).  Every CTA repeats this small step
-// (M*K <= 21504 values, read from L2), which removes a dependent kernel
-// launch and the x_q round trip through global memory from each decode
-// linear.
+// quantises every token row itself straight into its shared-memory copy of
+// x_q (quant_row_cta: the same arithmetic and order as the standalone
+// quantisation kernel).  Every CTA repeats this small step (M*K <= 21504
+// values, read from L2), which removes a dependent kernel launch and the x_q
+// round trip through global memory from each decode linear.
 template <int MT, bool U8, bool XS, bool FUSED = false, typename T = float, int MAXC = 1>
-__global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __restrict__ Wp,
-                                                               const float* __restrict__ gamma_ptr, int N, int K,
-                                                               const int8_t* __restrict__ xq,
-                                                               const float* __restrict__ a_scale,
-                                                               const int32_t* __restrict__ rowsum,
-                                                               const T* __restrict__ xin, const T* __restrict__ gain,
-                                                               float rms_eps, void* __restrict__ y, int y_dtype) {
+__global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint8_t* __restrict__ Wp,
+                                                            const float* __restrict__ gamma_ptr, int N, int K,
+                                                            const int8_t* __restrict__ xq,
+                                                            const float* __restrict__ a_scale,
+                                                            const int32_t* __restrict__ rowsum,
+                                                            const T* __restrict__ xin, const T* __restrict__ gain,
+                                                            float rms_eps, void* __restrict__ y, int y_dtype) {
   static_assert(!FUSED || (XS && U8), "the fused kernel keeps x_q in shared memory and uses its row sums");
   extern __shared__ __align__(1024) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -69,15 +81,16 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __
   uint64_t* all_bars = reinterpret_cast<uint64_t*>(smem + kGemvRingBytes);
   uint64_t* bars = all_bars + warp * kGemvSlots;
   uint64_t* xbar = all_bars + kGemvWarps * kGemvSlots;
-  uint8_t* xs = smem + kGemvRingBytes + kGemvBarBytes;
+  int* accs = reinterpret_cast<int*>(smem + kGemvRingBytes + kGemvBarBytes);  // [kGemvWaveRows][MT]
+  uint8_t* xs = smem + kGemvRingBytes + kGemvBarBytes + kGemvWaveRows * MT * 4;
 
   const int64_t row_lo = static_cast<int64_t>(N) * blockIdx.x / gridDim.x;
   const int64_t row_hi = static_cast<int64_t>(N) * (blockIdx.x + 1) / gridDim.x;
-  const int ngroups = static_cast<int>((row_hi - row_lo + kGemvRows - 1) / kGemvRows);
-  const int my_groups = ngroups > warp ? (ngroups - warp + kGemvWarps - 1) / kGemvWarps : 0;
-  const int kchunk = K < kGemvKChunk ? K : kGemvKChunk;
+  const int nrows = static_cast<int>(row_hi - row_lo);
+  const int ngroups = (nrows + kGemvRows - 1) / kGemvRows;
+  const int kchunk = gemv_kchunk(K);
   const int nkc = (K + kchunk - 1) / kchunk;
-  const int items = my_groups * nkc;
+  const int items = ngroups * nkc;  // item j -> (group j / nkc, chunk j % nkc), done by warp j % kGemvWarps
   const int64_t row_bytes = K >> 2;
   const int slot_row = kchunk >> 2;  // bytes per row inside a slot
 
@@ -86,19 +99,21 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __
     if (warp == 0) mbar_init(xbar, 1);
     fence_barrier_init();
   }
+  for (int i = threadIdx.x; i < kGemvWaveRows * MT; i += kGemvThreads) accs[i] = 0;
   __syncthreads();
 
   const uint64_t policy = policy_evict_first();
-  // Issue item j into ring slot j % kGemvSlots (lane 0 only).
-  auto issue = [&](int j) {
+  // Issue this warp's k-th item (item j = warp + k * kGemvWarps) into slot k % kGemvSlots (lane 0 only).
+  auto issue = [&](int k) {
+    const int j = warp + k * kGemvWarps;
     const int gi = j / nkc, kc = j - gi * nkc;
-    const int64_t r0 = row_lo + static_cast<int64_t>(warp + gi * kGemvWarps) * kGemvRows;
+    const int64_t r0 = row_lo + static_cast<int64_t>(gi) * kGemvRows;
     const int64_t left = row_hi - r0;
     const int nr = left < kGemvRows ? static_cast<int>(left) : kGemvRows;
     const int k0 = kc * kchunk;
     const int len = min(kchunk, K - k0) >> 2;  // bytes per row
-    uint64_t* bar = &bars[j % kGemvSlots];
-    uint8_t* dst = ring + (j % kGemvSlots) * kGemvSlotBytes;
+    uint64_t* bar = &bars[k % kGemvSlots];
+    uint8_t* dst = ring + (k % kGemvSlots) * kGemvSlotBytes;
     mbar_arrive_expect_tx(bar, static_cast<uint32_t>(nr * len));
     if (len == row_bytes) {
       // whole rows: the group's rows are contiguous in memory, one copy
@@ -109,8 +124,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __
                       policy);
     }
   };
+  const int my_items = items > warp ? (items - warp + kGemvWarps - 1) / kGemvWarps : 0;
   if (lane == 0)
-    for (int j = 0; j < kGemvSlots && j < items; ++j) issue(j);
+    for (int k = 0; k < kGemvSlots && k < my_items; ++k) issue(k);
 
   // Everything below reads the outputs of the previous kernel.
   pdl_launch_dependents();
@@ -145,95 +161,100 @@ __global__ void __launch_bounds__(kGemvWarps * 32) gemv_kernel(const uint8_t* __
     if constexpr (XS) xok = __all_sync(0xffffffffu, mbar_wait(xbar, 0));
   }
 
-  int acc[kGemvRows][MT];
+  // Waves of up to kGemvWaveRows rows (kGemvWaveRows / 4 groups).
+  constexpr int kWaveGroups = kGemvWaveRows / kGemvRows;
+  const int nwaves = (ngroups + kWaveGroups - 1) / kWaveGroups;
+  int k = 0;  // this warp's item counter (ring position)
+  int failed_at = -1;
+  for (int wv = 0; wv < nwaves; ++wv) {
+    const int j_end = min(items, (wv + 1) * kWaveGroups * nkc);
+    for (; xok && failed_at < 0 && warp + k * kGemvWarps < j_end; ++k) {
+      const int j = warp + k * kGemvWarps;
+      const int slot = k % kGemvSlots;
+      // Every lane acquires the barrier itself; the warp leaves together if any gave up.
+      const bool got = mbar_wait(&bars[slot], (k / kGemvSlots) & 1);
+      if (!__all_sync(0xffffffffu, got)) {
+        failed_at = k;
+        break;
+      }
+      const int gi = j / nkc, kc = j - gi * nkc;
+      const int k0 = kc * kchunk;
+      const int len = min(kchunk, K - k0);  // weights per row in this item
+      const uint32_t sw = smem_addr(ring + slot * kGemvSlotBytes);
+      int acc[kGemvRows][MT];
 #pragma unroll
-  for (int r = 0; r < kGemvRows; ++r)
+      for (int r = 0; r < kGemvRows; ++r)
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[r][m] = 0;
-
-  int failed_at = xok ? -1 : 0;
-  for (int j = 0; xok && j < items; ++j) {
-    const int slot = j % kGemvSlots;
-    // Every lane acquires the barrier itself; the warp leaves together if any gave up.
-    const bool got = mbar_wait(&bars[slot], (j / kGemvSlots) & 1);
-    if (!__all_sync(0xffffffffu, got)) {
-      failed_at = j;
-      break;
-    }
-    const int gi = j / nkc, kc = j - gi * nkc;
-    const int k0 = kc * kchunk;
-    const int len = min(kchunk, K - k0);  // weights per row in this item
-    const uint32_t sw = smem_addr(ring + slot * kGemvSlotBytes);
+        for (int m = 0; m < MT; ++m) acc[r][m] = 0;
 #pragma unroll 1
-    for (int kk = lane * 16; kk < len; kk += 512) {
-      // This lane: weights k0+kk .. k0+kk+15 of the 4 rows.
-      uint32_t xv[MT][4];
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        uint4 u;
-        if constexpr (XS) {
-          u = lds128(smem_addr(xs) + m * K + k0 + kk);
-        } else {
-          u = __ldg(reinterpret_cast<const uint4*>(xq + static_cast<int64_t>(m) * K + k0 + kk));
-        }
-        xv[m][0] = u.x;
-        xv[m][1] = u.y;
-        xv[m][2] = u.z;
-        xv[m][3] = u.w;
-      }
-#pragma unroll
-      for (int r = 0; r < kGemvRows; ++r) {
-        uint32_t w;
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(sw + r * slot_row + (kk >> 2)));
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const uint32_t c4 = (w >> (2 * jj)) & 0x03030303u;
-#pragma unroll
-          for (int m = 0; m < MT; ++m)
-            acc[r][m] = U8 ? dp4a_us(c4, xv[m][jj], acc[r][m]) : dp4a_ss(codes_to_signed(c4), xv[m][jj], acc[r][m]);
-        }
-      }
-    }
-    __syncwarp();
-    if (lane == 0 && j + kGemvSlots < items) {
-      fence_proxy_async_smem();
-      issue(j + kGemvSlots);
-    }
-    if (kc == nkc - 1) {
-      // Row group finished: reduce over lanes, dequantise, store.
-#pragma unroll
-      for (int r = 0; r < kGemvRows; ++r)
+      for (int kk = lane * 16; kk < len; kk += 512) {
+        // This lane: weights k0+kk .. k0+kk+15 of the 4 rows.
+        uint32_t xv[MT][4];
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-          int v = acc[r][m];
-#pragma unroll
-          for (int s = 16; s >= 1; s >>= 1) v += __shfl_xor_sync(0xffffffffu, v, s);
-          acc[r][m] = v;
-        }
-      const int64_t r0 = row_lo + static_cast<int64_t>(warp + gi * kGemvWarps) * kGemvRows;
-#pragma unroll
-      for (int r = 0; r < kGemvRows; ++r)
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-          if (lane == r * MT + m && r0 + r < row_hi) {
-            const int a = acc[r][m] - rsum[m];
-            const int64_t o = static_cast<int64_t>(m) * N + r0 + r;
-            if (y_dtype == 2) {
-              static_cast<int32_t*>(y)[o] = a;
-            } else {
-              const float v = __fmul_rn(__fmul_rn(__int2float_rn(a), gamma), asc[m]);
-              if (y_dtype == 0) static_cast<float*>(y)[o] = v;
-              else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
-            }
+          uint4 u;
+          if constexpr (XS) {
+            u = lds128(smem_addr(xs) + m * K + k0 + kk);
+          } else {
+            u = __ldg(reinterpret_cast<const uint4*>(xq + static_cast<int64_t>(m) * K + k0 + kk));
           }
-          acc[r][m] = 0;
+          xv[m][0] = u.x;
+          xv[m][1] = u.y;
+          xv[m][2] = u.z;
+          xv[m][3] = u.w;
+        }
+#pragma unroll
+        for (int r = 0; r < kGemvRows; ++r) {
+          uint32_t w;
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w) : "r"(sw + r * slot_row + (kk >> 2)));
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            const uint32_t c4 = (w >> (2 * jj)) & 0x03030303u;
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+              acc[r][m] = U8 ? dp4a_us(c4, xv[m][jj], acc[r][m]) : dp4a_ss(codes_to_signed(c4), xv[m][jj], acc[r][m]);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0 && k + kGemvSlots < my_items) {
+        fence_proxy_async_smem();
+        issue(k + kGemvSlots);
+      }
+      // Item partial sums -> the rows' shared accumulators.
+      const int wrow0 = (gi - wv * kWaveGroups) * kGemvRows;  // row of the group inside the wave
+      const int grow0 = gi * kGemvRows;                       // row of the group inside the CTA
+#pragma unroll
+      for (int r = 0; r < kGemvRows; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const int v = __reduce_add_sync(0xffffffffu, acc[r][m]);
+          if (lane == r * MT + m && grow0 + r < nrows) atomicAdd(&accs[(wrow0 + r) * MT + m], v);
         }
     }
+    // Wave finished: dequantise and store its rows, then clear the accumulators.
+    __syncthreads();
+    const int wrows = min(kGemvWaveRows, nrows - wv * kGemvWaveRows);
+    for (int i = threadIdx.x; i < wrows * MT; i += kGemvThreads) {
+      const int rr = i / MT, m = i - rr * MT;
+      const int a = accs[i] - rsum[m];
+      const int64_t o = static_cast<int64_t>(m) * N + row_lo + wv * kGemvWaveRows + rr;
+      if (y_dtype == 2) {
+        static_cast<int32_t*>(y)[o] = a;
+      } else {
+        const float v = __fmul_rn(__fmul_rn(__int2float_rn(a), gamma), asc[m]);
+        if (y_dtype == 0) static_cast<float*>(y)[o] = v;
+        else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
+      }
+      accs[i] = 0;
+    }
+    __syncthreads();
   }
-  if (failed_at >= 0 && lane == 0) {
+  if ((failed_at >= 0 || !xok) && lane == 0) {
     // Let copies still in flight land before the CTA's shared memory goes away.
-    for (int j = failed_at; j < items && j < failed_at + kGemvSlots; ++j)
-      mbar_wait(&bars[j % kGemvSlots], (j / kGemvSlots) & 1);
+    const int from = failed_at >= 0 ? failed_at : 0;
+    for (int kk = from; kk < my_items && kk < from + kGemvSlots; ++kk)
+      mbar_wait(&bars[kk % kGemvSlots], (kk / kGemvSlots) & 1);
     if (XS && !FUSED && warp == 0) mbar_wait(xbar, 0);
   }
 }

@@ -54,24 +54,46 @@ constexpr int kQuantThreads = 256;
 struct QuantScratch {
   float red[kQuantThreads];
   float bcast;
-  int ired[kQuantThreads / 32];
+  int ired[32];
 };
 
-// Quantises one token row with the 256 threads of the CTA (all must call it).
-// Thread t owns the 8-element chunks c = t, t+256, ... and keeps them in
-// registers, so the row is read once.  Writes x_q through xq_row (global or
-// shared memory); returns max|h| and sum(x_q) to every thread.
+// RNE of an fp32 value to a signed byte with saturation to [-128, 127]; for
+// |v| <= 127 * (1 + 2^-24), as h * (127 / amax) always is, this equals
+// clamp(RNE(v), -127, 127).
+BN_DEV uint32_t f32_to_s8_rne(float v) {
+  uint32_t r;
+  asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(r) : "f"(v));
+  return r;
+}
+
+// Four signed bytes (low byte of each argument) packed into a word, byte 0 = a.
+BN_DEV uint32_t pack4_s8(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Quantises one token row with the threads of the CTA.  Every thread must
+// call it (it holds CTA-wide barriers).  Thread t owns the 8-element chunks
+// c = t, t+nt, ... (nt = all threads without RMSNorm, the first 256 with it)
+// and keeps them in registers, so the row is read once.  Writes x_q through
+// xq_row (global or shared memory); returns max|h| and sum(x_q) to every
+// thread.
 template <typename T, int MAXC>
 BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict__ gain, float rms_eps,
                           int8_t* xq_row, QuantScratch& sc, float& amax_out, int& sum_out) {
   const int t = threadIdx.x;
   const int lane = t & 31, warp = t >> 5;
-  const int nchunks = K >> 3;
+  // Without RMSNorm nothing depends on which thread owns which chunk (max and
+  // integer sums are order-free), so every thread of the CTA takes part; with
+  // it, the first 256 threads keep the fixed ownership the summation order is
+  // defined on.
+  const int nt = gain == nullptr ? static_cast<int>(blockDim.x) : kQuantThreads;
+  const bool act = t < nt;
+  const int nchunks = act ? (K >> 3) : 0;  // threads beyond nt own no chunk
 
   Chunk8<T> ch[MAXC];
 #pragma unroll
   for (int i = 0; i < MAXC; ++i) {
-    const int c = t + kQuantThreads * i;
+    const int c = t + nt * i;
     if (c < nchunks) ch[i].load(row + 8 * c);
   }
 
@@ -89,7 +111,7 @@ BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict_
         }
       }
     }
-    sc.red[t] = ss;
+    if (act) sc.red[t] = ss;
     __syncthreads();
 #pragma unroll
     for (int s = kQuantThreads / 2; s >= 32; s >>= 1) {
@@ -116,7 +138,7 @@ BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict_
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < MAXC; ++i) {
-    const int c = t + kQuantThreads * i;
+    const int c = t + nt * i;
     if (c < nchunks) {
       Chunk8<T> g;
       if (gain != nullptr) g.load(gain + 8 * c);
@@ -131,44 +153,43 @@ BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict_
 #pragma unroll
   for (int s = 16; s >= 1; s >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, s));
   __syncthreads();  // red[] reuse
-  if (lane == 0) sc.red[warp] = amax;
+  if (act && lane == 0) sc.red[warp] = amax;
   __syncthreads();
+  const int nw = nt >> 5;
   amax = sc.red[0];
-#pragma unroll
-  for (int w = 1; w < kQuantThreads / 32; ++w) amax = fmaxf(amax, sc.red[w]);
+  for (int w = 1; w < nw; ++w) amax = fmaxf(amax, sc.red[w]);
 
   int sum = 0;
   const float s = amax == 0.0f ? 0.0f : __fdiv_rn(127.0f, amax);
 #pragma unroll
   for (int i = 0; i < MAXC; ++i) {
-    const int c = t + kQuantThreads * i;
+    const int c = t + nt * i;
     if (c < nchunks) {
       uint32_t lo = 0, hi = 0;
       if (amax != 0.0f) {
         Chunk8<T> g;
         if (gain != nullptr) g.load(gain + 8 * c);
+        uint32_t q[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const float v = ch[i].get(e);
           const float h = gain != nullptr ? __fmul_rn(__fmul_rn(v, r), g.get(e)) : v;
-          int q = __float2int_rn(__fmul_rn(h, s));
-          q = q < -127 ? -127 : (q > 127 ? 127 : q);
-          sum += q;
-          const uint32_t b = static_cast<uint32_t>(q) & 0xFFu;
-          if (e < 4) lo |= b << (8 * e);
-          else hi |= b << (8 * (e - 4));
+          q[e] = f32_to_s8_rne(__fmul_rn(h, s));
         }
+        lo = pack4_s8(q[0], q[1], q[2], q[3]);
+        hi = pack4_s8(q[4], q[5], q[6], q[7]);
+        sum = __dp4a(static_cast<int>(lo), 0x01010101, sum);
+        sum = __dp4a(static_cast<int>(hi), 0x01010101, sum);
       }
       *reinterpret_cast<uint2*>(xq_row + 8 * c) = make_uint2(lo, hi);
     }
   }
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane == 0) sc.ired[warp] = sum;
+  if (act && lane == 0) sc.ired[warp] = sum;
   __syncthreads();
   int tot = 0;
-#pragma unroll
-  for (int w = 0; w < kQuantThreads / 32; ++w) tot += sc.ired[w];
+  for (int w = 0; w < nw; ++w) tot += sc.ired[w];
   amax_out = amax;
   sum_out = tot;
   __syncthreads();  // scratch reuse by the next call
