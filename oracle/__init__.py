@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_bitlinear_sampled.restype = ctypes.c_int
         L.oracle_f32_to_bf16.argtypes = [P, I64, P]
         L.oracle_f32_to_bf16.restype = None
+        L.oracle_relu2_gate.argtypes = [P, P, I64, P]
+        L.oracle_relu2_gate.restype = None
         _lib = L
     return _lib
 
@@ -182,3 +184,44 @@ def f32_to_bf16(y: np.ndarray) -> np.ndarray:
     out = np.empty(y.shape, dtype=np.uint16)
     lib().oracle_f32_to_bf16(_p(y), y.size, _p(out))
     return out
+
+
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> the fp32 values they stand for (exact)."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def relu2_gate(u: np.ndarray, g: np.ndarray) -> np.ndarray:
+    """RN32(RN32(r*r)*u) with r = max(g, +0): the squared-ReLU gate of the FFN."""
+    u = _f32(u)
+    g = _f32(g)
+    assert u.shape == g.shape
+    out = np.empty_like(u)
+    lib().oracle_relu2_gate(_p(u), _p(g), u.size, _p(out))
+    return out
+
+
+def bitlinear_forward(x: np.ndarray, packed: np.ndarray, gamma, gain=None, rms_eps: float = 1e-5):
+    """One BitLinear on fp32 token rows x (M x K): optional RMSNorm, absmax int8
+    quantisation, exact ternary product, dequant.  Returns (acc int32, y fp32)."""
+    x = _f32(x)
+    xq, a, _ = quant_act(x, gain, rms_eps)
+    return bitlinear(packed, gamma, x.shape[1], xq, a)
+
+
+def ffn(x: np.ndarray, up, gate, down, gain_in=None, eps_in: float = 1e-5, gain_sub=None, eps_sub: float = 1e-5):
+    """Feed-forward block of BitNet b1.58 built from BitLinears.
+
+    up, gate: (packed F x D/4, gamma); down: (packed D x F/4, gamma).  x: M x D
+    fp32 values (bf16 values in the block).  Steps: u = BitLinear_up(x) and
+    g = BitLinear_gate(x), both normalising x with gain_in; h = bf16 of the
+    squared-ReLU gate relu2_gate(u, g) (the down projection's input, stored
+    as bf16 like every activation of the block); y = BitLinear_down(h),
+    normalising h with gain_sub (the sub-layer norm).
+    Returns (h bf16 bits M x F, acc_down int32 M x D, y fp32 M x D)."""
+    _, u = bitlinear_forward(x, up[0], up[1], gain_in, eps_in)
+    _, g = bitlinear_forward(x, gate[0], gate[1], gain_in, eps_in)
+    h_bits = f32_to_bf16(relu2_gate(u, g))
+    acc, y = bitlinear_forward(bf16_to_f32(h_bits), down[0], down[1], gain_sub, eps_sub)
+    return h_bits, acc, y

@@ -241,6 +241,21 @@ int oracle_bitlinear_sampled(const uint8_t* packed, float gamma, int64_t N, int6
   return 0;
 }
 
+// Squared-ReLU gating of the feed-forward block: the FFN of BitNet b1.58
+// uses a squared ReLU as its activation ([Explainer, "Zrób to sam": squared
+// ReLU in the FFN, subln normalisation, no biases]; kripta.biz 2B4T news:
+// ReLU^2 in the FFN layers).  The gate branch goes through the activation
+// and multiplies the up branch elementwise:
+//   out[i] = RN32(RN32(r * r) * u[i]),  r = g[i] if g[i] > 0, else +0.
+// u and g are the fp32 outputs of the up and gate BitLinears.
+void oracle_relu2_gate(const float* u, const float* g, int64_t n, float* out) {
+  for (int64_t i = 0; i < n; ++i) {
+    const float r = g[i] > 0.0f ? g[i] : 0.0f;
+    const float sq = r * r;
+    out[i] = sq * u[i];
+  }
+}
+
 // fp32 -> bf16, round half to even, as bit patterns (NaN -> quiet NaN).
 void oracle_f32_to_bf16(const float* y, int64_t n, uint16_t* out) {
   for (int64_t i = 0; i < n; ++i) {
