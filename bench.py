@@ -470,6 +470,11 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
     if not args.no_prefill and lins[0].M <= 8:
         prefill = bench_prefill(torch, bl, dev, stream, peaks, peak_src, group)
 
+    # ---- the one-launch decode FFN block (up, gate, squared-ReLU gating, down), a secondary line
+    ffn_block = None
+    if not args.no_ffn and lins[0].M <= 8:
+        ffn_block = bench_ffn_block(torch, bl, dev, stream, peaks, peak_src, group)
+
     # ---- CPU oracle baseline (rank 0, N = 1)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
@@ -509,12 +514,79 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
                        "pack_ms": pack_ms, "pack_gbs": [l.N * l.K * 4.25 / (ms / 1e3) / 1e9
                                                         for l, ms in zip(lins, pack_ms)]},
             "prefill": prefill,
+            "ffn_block": ffn_block,
         }
         print(json.dumps(line), flush=True)
     if group:
         import torch.distributed as dist
         del g_main, g_rem
         dist.destroy_process_group()
+
+
+def bench_ffn_block(torch, bl, dev, stream, peaks, peak_src, group, name="ffn_block_m1_2p5b"):
+    """The one-launch decode FFN (bitnet_bitlinear_ffn_gemv: up and gate, squared-ReLU gating, sub-norm, down)
+    back to back in CUDA graphs over rotating weight copies, beside the same three BitLinears as separate
+    fused launches (without the gating step)."""
+    blk = synth.FFN_BLOCKS[name]
+    P = {}
+    for which in ("up", "gate", "down"):
+        W = torch.from_numpy(blk.make_w(which, 0)).to(dev)
+        P[which] = bl.bitnet_pack_weights(W, EPS_W)
+        del W
+    copies = max(2, int(2 * 126e6 // blk.weight_bytes) + 1)
+    cps = [[P[w][0]] + [P[w][0].clone() for _ in range(copies - 1)] for w in ("up", "gate", "down")]
+    bf = lambda a: torch.from_numpy(synth.f32_to_bf16_bits(a).view(np.int16).copy()).to(dev).view(torch.bfloat16)
+    x = bf(blk.make_x(0))
+    gi, gs = (bf(g) for g in blk.make_gains(0))
+    h = torch.empty((blk.M, blk.F), dtype=torch.bfloat16, device=dev)
+    u = torch.empty((blk.M, blk.F), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((blk.M, blk.D), dtype=torch.bfloat16, device=dev)
+    sync = torch.zeros(bl.BITNET_FFN_SYNC_BYTES, dtype=torch.uint8, device=dev)
+    G = P["up"][1], P["gate"][1], P["down"][1]
+
+    def ffn(c):
+        bl.bitnet_bitlinear_ffn_gemv(x, cps[0][c % copies], G[0], cps[1][c % copies], G[1], cps[2][c % copies],
+                                     G[2], gi, EPS_RMS, gs, EPS_RMS, h=h, y=y, sync=sync)
+
+    def three(c):
+        bl.bitnet_bitlinear_gemv(x, cps[0][c % copies], G[0], gi, EPS_RMS, y=u)
+        bl.bitnet_bitlinear_gemv(x, cps[1][c % copies], G[1], gi, EPS_RMS, y=h)
+        bl.bitnet_bitlinear_gemv(h, cps[2][c % copies], G[2], gs, EPS_RMS, y=y)
+
+    def timed(fn, per=64, reps=40):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for c in range(per):
+                fn(c)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                g.replay()
+        torch.cuda.synchronize(dev)
+        barrier(group, dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(group, dev)
+        return max_over_ranks(e0.elapsed_time(e1), group, dev) / (per * reps)
+
+    ms = timed(ffn)
+    ms3 = timed(three)
+    status = bl.bitnet_get_device_status()
+    nbytes = blk.weight_bytes + 2 * blk.M * blk.D + 2 * (blk.D + blk.F) + 12 + 2 * blk.M * blk.F + 2 * blk.M * blk.D
+    gbs = nbytes / (ms / 1e3) / 1e9
+    hbm = float(peaks["hbm_gbs"])
+    traffic = profiled_traffic(os.path.join(ROOT, "profiles", "ffn_block_m1_2p5b.md"),
+                               kernel_source_hash(["ffn.cuh", "gemv.cuh", "quant.cuh", "ptx.cuh"]))
+    return {"workload": name, "M": blk.M, "D": blk.D, "F": blk.F, "us_per_ffn": ms * 1e3, "gbs": gbs,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "traffic": traffic, "bytes_per_launch": nbytes,
+                         "peak_source": f"{peak_src} hbm_gbs"},
+            "three_fused_launches_us": ms3 * 1e3, "weight_copies": copies, "device_status": status,
+            "timing": "CUDA graphs of 64 launches over rotating weight copies, CUDA events, per launch"}
 
 
 def bench_prefill(torch, bl, dev, stream, peaks, peak_src, group):
@@ -573,6 +645,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-prefill", action="store_true", help="skip the secondary prefill GEMM measurement")
+    ap.add_argument("--no-ffn", action="store_true", help="skip the secondary one-launch FFN block measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

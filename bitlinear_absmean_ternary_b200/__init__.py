@@ -28,6 +28,8 @@ BITNET_F32 = 0
 BITNET_BF16 = 1
 BITNET_I32 = 2
 
+BITNET_FFN_SYNC_BYTES = 64
+
 _lib = None
 
 
@@ -58,6 +60,8 @@ def lib() -> ctypes.CDLL:
             fn.restype = I
         L.bitnet_bitlinear_gemv.argtypes = [P, I, P, F, P, P, I64, I64, I64, P, I, P]
         L.bitnet_bitlinear_gemv.restype = I
+        L.bitnet_bitlinear_ffn_gemv.argtypes = [P, I, I64, I64, I64, P, F, P, P, P, P, P, F, P, P, P, P, I, P, P]
+        L.bitnet_bitlinear_ffn_gemv.restype = I
         L.bitnet_get_device_status.argtypes = [P]
         L.bitnet_get_device_status.restype = I
         L.bitnet_status_string.argtypes = [I]
@@ -212,6 +216,33 @@ def bitnet_bitlinear_gemv(x, W_packed, gamma, rms_gain=None, rms_eps: float = 1e
                                      _ptr(gamma), N, K, M, _ptr(y), _dtype_code(y.dtype), _stream(x.device))
     _check("bitnet_bitlinear_gemv", st)
     return y
+
+
+def bitnet_bitlinear_ffn_gemv(x, W_up, gamma_up, W_gate, gamma_gate, W_down, gamma_down, rms_gain_in=None,
+                              rms_eps_in: float = 1e-5, rms_gain_sub=None, rms_eps_sub: float = 1e-5, h=None, y=None,
+                              out_dtype=None, sync=None):
+    """Decode FFN block (M <= 8) in one launch: u, g = BitLinear_up/gate(x),
+    h = bf16 squared-ReLU gate, y = BitLinear_down(h).  x: M x D bf16.
+    sync: BITNET_FFN_SYNC_BYTES zeroed device bytes reused across calls on one
+    stream (allocated per call when None).  Returns (h, y)."""
+    torch = _torch()
+    _need_cuda(x, W_up, gamma_up, W_gate, gamma_gate, W_down, gamma_down, rms_gain_in, rms_gain_sub, h, y, sync)
+    M, D = x.shape
+    F = W_up.shape[0]
+    if tuple(W_up.shape) != (F, D // 4) or tuple(W_gate.shape) != (F, D // 4) or tuple(W_down.shape) != (D, F // 4):
+        raise ValueError("W_up/W_gate must be F x D/4 and W_down D x F/4 packed bytes")
+    if h is None:
+        h = torch.empty((M, F), dtype=torch.bfloat16, device=x.device)
+    if y is None:
+        y = torch.empty((M, D), dtype=out_dtype or torch.bfloat16, device=x.device)
+    if sync is None:
+        sync = torch.zeros(BITNET_FFN_SYNC_BYTES, dtype=torch.uint8, device=x.device)
+    st = lib().bitnet_bitlinear_ffn_gemv(_ptr(x), _dtype_code(x.dtype), M, D, F, _ptr(rms_gain_in), rms_eps_in,
+                                         _ptr(W_up), _ptr(gamma_up), _ptr(W_gate), _ptr(gamma_gate),
+                                         _ptr(rms_gain_sub), rms_eps_sub, _ptr(W_down), _ptr(gamma_down), _ptr(h),
+                                         _ptr(y), _dtype_code(y.dtype), _ptr(sync), _stream(x.device))
+    _check("bitnet_bitlinear_ffn_gemv", st)
+    return h, y
 
 
 def bitnet_get_device_status(device=None) -> int:

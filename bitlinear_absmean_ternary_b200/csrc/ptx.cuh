@@ -307,4 +307,59 @@ BN_DEV int4 ld_shared_cluster_v4(uint32_t cluster_addr) {
   return v;
 }
 
+// ------------------------------------------------------- grid-wide barrier
+
+BN_DEV uint64_t ld_acquire_gpu_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+BN_DEV uint64_t atom_add_release_gpu_u64(uint64_t* p, uint64_t v) {
+  uint64_t old;
+  asm volatile("atom.add.release.gpu.global.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+  return old;
+}
+
+// Barrier over every CTA of a cooperative launch of G CTAs, on a 64-bit
+// arrival counter that only ever grows.  A launch finds the counter at a
+// multiple of G (it starts at 0 and every completed barrier adds G), so a
+// CTA's own arrival returns base + (CTAs that arrived before it), from which
+// it knows the target base + G; it then waits until the counter reaches it.
+// One release atomic per CTA and acquire polls: no step of the barrier
+// waits on another CTA's atomic round trip.  Consecutive launches on one
+// stream may share the counter (a launch reaches its barrier only after the
+// previous launch completed).  Every thread of every CTA must call it.
+// Gives up after kWaitLimitNs, flags the device error word and returns
+// false; the counter is then no longer a multiple of G and must be reset.
+// NT: the first NT threads of each CTA take part (named barrier 1), or all
+// threads when NT == 0.
+template <int NT = 0>
+BN_DEV bool grid_barrier(uint64_t* counter, int* flag_smem) {
+  if constexpr (NT == 0) __syncthreads();
+  else asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+  if (threadIdx.x == 0) {
+    bool ok = true;
+    const uint64_t G = static_cast<uint64_t>(gridDim.x) * gridDim.y * gridDim.z;
+    // release: this CTA's writes, ordered before it by the CTA barrier above
+    const uint64_t old = atom_add_release_gpu_u64(counter, 1);
+    const uint64_t target = (old / G + 1) * G;
+    if (old + 1 != target) {
+      const uint64_t t0 = global_timer_ns();
+      for (uint32_t i = 1; ld_acquire_gpu_u64(counter) < target; ++i) {
+        if ((i & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+          flag_timeout();
+          ok = false;
+          break;
+        }
+      }
+    }
+    __threadfence();
+    *flag_smem = ok ? 1 : 0;
+  }
+  if constexpr (NT == 0) __syncthreads();
+  else asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+  return *flag_smem != 0;
+}
+
 }  // namespace bitnet

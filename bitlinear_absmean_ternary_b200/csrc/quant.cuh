@@ -22,6 +22,8 @@ template <>
 struct Chunk8<__nv_bfloat16> {
   uint4 u;
   BN_DEV void load(const __nv_bfloat16* p) { u = __ldg(reinterpret_cast<const uint4*>(p)); }
+  // For data written earlier in the same kernel by other CTAs: L2 only.
+  BN_DEV void load_cg(const __nv_bfloat16* p) { u = __ldcg(reinterpret_cast<const uint4*>(p)); }
   BN_DEV float get(int e) const {
     const uint32_t w = e < 2 ? u.x : (e < 4 ? u.y : (e < 6 ? u.z : u.w));
     return __uint_as_float((e & 1) ? (w & 0xFFFF0000u) : (w << 16));
@@ -34,6 +36,10 @@ struct Chunk8<float> {
   BN_DEV void load(const float* p) {
     a = __ldg(reinterpret_cast<const float4*>(p));
     b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  }
+  BN_DEV void load_cg(const float* p) {
+    a = __ldcg(reinterpret_cast<const float4*>(p));
+    b = __ldcg(reinterpret_cast<const float4*>(p) + 1);
   }
   BN_DEV float get(int e) const {
     switch (e) {
@@ -52,9 +58,9 @@ struct Chunk8<float> {
 constexpr int kQuantThreads = 256;
 
 struct QuantScratch {
-  float red[kQuantThreads];
-  float bcast;
-  int ired[32];
+  float red[kQuantThreads];  // per-thread sums of squares (the first 256 threads)
+  float amx[32];             // per-warp max|h|
+  int ired[32];              // per-warp sums of x_q
 };
 
 // RNE of an fp32 value to a signed byte with saturation to [-128, 127]; for
@@ -71,31 +77,75 @@ BN_DEV uint32_t pack4_s8(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
+BN_DEV void prefetch_l1(const void* p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
+
+// Barrier over the first NT threads of the CTA (named barrier 1), or over
+// the whole CTA when NT == 0.
+template <int NT>
+BN_DEV void sync_threads() {
+  if constexpr (NT == 0) __syncthreads();
+  else asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
+}
+
 // Quantises one token row with the threads of the CTA.  Every thread must
 // call it (it holds CTA-wide barriers).  Thread t owns the 8-element chunks
 // c = t, t+nt, ... (nt = all threads without RMSNorm, the first 256 with it)
 // and keeps them in registers, so the row is read once.  Writes x_q through
-// xq_row (global or shared memory); returns max|h| and sum(x_q) to every
-// thread.
-template <typename T, int MAXC>
+// xq_row (global or shared memory; complete and visible to the whole CTA on
+// return); returns max|h| and sum(x_q) to every thread.  COHERENT reads the
+// row through L2 only, for a row that other CTAs of the same kernel wrote.
+//
+// The work is a chain of dependent steps, so the code keeps the chain short:
+// the row and the gain are requested together at the start (one memory
+// round trip), and each of the three reductions (sum of squares, max|h|,
+// sum of x_q) costs one CTA barrier.  For the sum of squares every warp
+// evaluates the same fixed tree from the 256 per-thread sums in shared
+// memory -- level 128, 64 and 32 pairings, then shuffles 16 .. 1 -- so each
+// warp obtains the norm itself, with the oracle's order of additions.
+// Consecutive calls may reuse the scratch: every write to a scratch array
+// comes after a barrier that all readers of its previous contents passed.
+// NT: the threads taking part are the first NT of the CTA (synchronised by
+// named barrier 1), or all of them when NT == 0.
+template <typename T, int MAXC, bool COHERENT = false, int NT = 0>
 BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict__ gain, float rms_eps,
                           int8_t* xq_row, QuantScratch& sc, float& amax_out, int& sum_out) {
   const int t = threadIdx.x;
   const int lane = t & 31, warp = t >> 5;
+  const int nthreads = NT == 0 ? static_cast<int>(blockDim.x) : NT;
+  const int nwarps = nthreads >> 5;
   // Without RMSNorm nothing depends on which thread owns which chunk (max and
   // integer sums are order-free), so every thread of the CTA takes part; with
   // it, the first 256 threads keep the fixed ownership the summation order is
   // defined on.
-  const int nt = gain == nullptr ? static_cast<int>(blockDim.x) : kQuantThreads;
-  const bool act = t < nt;
-  const int nchunks = act ? (K >> 3) : 0;  // threads beyond nt own no chunk
+  const int nt = gain == nullptr ? nthreads : kQuantThreads;
+  const int nchunks = t < nt ? (K >> 3) : 0;  // threads beyond nt own no chunk
+  // The gain stays in registers when that is cheap, else it is prefetched
+  // into L1 and read again there.
+  constexpr bool kGainRegs = sizeof(Chunk8<T>) * MAXC <= 64;
 
   Chunk8<T> ch[MAXC];
+  Chunk8<T> gch[kGainRegs ? MAXC : 1];
 #pragma unroll
   for (int i = 0; i < MAXC; ++i) {
     const int c = t + nt * i;
-    if (c < nchunks) ch[i].load(row + 8 * c);
+    if (c < nchunks) {
+      if constexpr (COHERENT) ch[i].load_cg(row + 8 * c);
+      else ch[i].load(row + 8 * c);
+      if (gain != nullptr) {
+        if constexpr (kGainRegs) gch[i].load(gain + 8 * c);
+        else prefetch_l1(gain + 8 * c);
+      }
+    }
   }
+  auto gain_chunk = [&](int i, int c) {
+    if constexpr (kGainRegs) {
+      return gch[i];
+    } else {
+      Chunk8<T> g;
+      g.load(gain + 8 * c);
+      return g;
+    }
+  };
 
   float r = 1.0f;
   if (gain != nullptr) {
@@ -111,27 +161,19 @@ BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict_
         }
       }
     }
-    if (act) sc.red[t] = ss;
-    __syncthreads();
+    if (t < kQuantThreads) sc.red[t] = ss;
+    sync_threads<NT>();
+    const float* R = sc.red;
+    float p = __fadd_rn(__fadd_rn(__fadd_rn(R[lane], R[lane + 128]), __fadd_rn(R[lane + 64], R[lane + 192])),
+                        __fadd_rn(__fadd_rn(R[lane + 32], R[lane + 160]), __fadd_rn(R[lane + 96], R[lane + 224])));
 #pragma unroll
-    for (int s = kQuantThreads / 2; s >= 32; s >>= 1) {
-      if (t < s) sc.red[t] = __fadd_rn(sc.red[t], sc.red[t + s]);
-      __syncthreads();
+    for (int s = 16; s >= 1; s >>= 1) {
+      const float o = __shfl_down_sync(0xffffffffu, p, s);
+      if (lane < s) p = __fadd_rn(p, o);
     }
-    if (warp == 0) {
-      float p = sc.red[lane];
-#pragma unroll
-      for (int s = 16; s >= 1; s >>= 1) {
-        const float o = __shfl_down_sync(0xffffffffu, p, s);
-        if (lane < s) p = __fadd_rn(p, o);
-      }
-      if (lane == 0) {
-        const float ms = __fdiv_rn(p, static_cast<float>(K));
-        sc.bcast = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, rms_eps)));
-      }
-    }
-    __syncthreads();
-    r = sc.bcast;
+    p = __shfl_sync(0xffffffffu, p, 0);
+    const float ms = __fdiv_rn(p, static_cast<float>(K));
+    r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, rms_eps)));
   }
 
   // h = RN32(RN32(v * r) * g) or v; amax = max |h| (order-free).
@@ -141,7 +183,7 @@ BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict_
     const int c = t + nt * i;
     if (c < nchunks) {
       Chunk8<T> g;
-      if (gain != nullptr) g.load(gain + 8 * c);
+      if (gain != nullptr) g = gain_chunk(i, c);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const float v = ch[i].get(e);
@@ -152,12 +194,11 @@ BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict_
   }
 #pragma unroll
   for (int s = 16; s >= 1; s >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, s));
-  __syncthreads();  // red[] reuse
-  if (act && lane == 0) sc.red[warp] = amax;
-  __syncthreads();
-  const int nw = nt >> 5;
-  amax = sc.red[0];
-  for (int w = 1; w < nw; ++w) amax = fmaxf(amax, sc.red[w]);
+  if (lane == 0) sc.amx[warp] = amax;
+  sync_threads<NT>();
+  amax = lane < nwarps ? sc.amx[lane] : 0.0f;
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, s));
 
   int sum = 0;
   const float s = amax == 0.0f ? 0.0f : __fdiv_rn(127.0f, amax);
@@ -168,7 +209,7 @@ BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict_
       uint32_t lo = 0, hi = 0;
       if (amax != 0.0f) {
         Chunk8<T> g;
-        if (gain != nullptr) g.load(gain + 8 * c);
+        if (gain != nullptr) g = gain_chunk(i, c);
         uint32_t q[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -186,13 +227,13 @@ BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict_
   }
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (act && lane == 0) sc.ired[warp] = sum;
-  __syncthreads();
-  int tot = 0;
-  for (int w = 0; w < nw; ++w) tot += sc.ired[w];
+  if (lane == 0) sc.ired[warp] = sum;
+  sync_threads<NT>();
+  int tot = lane < nwarps ? sc.ired[lane] : 0;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
   amax_out = amax;
   sum_out = tot;
-  __syncthreads();  // scratch reuse by the next call
 }
 
 // Standalone kernel: one CTA per token row.

@@ -212,3 +212,40 @@ WORKLOADS = {
         Linear("down", m, 21504, 5376, 0.01, outlier_frac=0.005, outlier_scale=30.0, w_id=101, x_id=102)]
        for m in (1, 16, 2048)},
 }
+
+
+@dataclasses.dataclass(frozen=True)
+class FfnBlock:
+    """Feed-forward block of three BitLinears: up and gate (D -> F), squared-ReLU
+    gating, down (F -> D), with an RMSNorm gain on each BitLinear input."""
+    name: str
+    M: int
+    D: int
+    F: int
+    w_sigma: float
+    outlier_frac: float = 0.0
+    outlier_scale: float = 1.0
+    ids: tuple = (1, 2, 3, 4, 5, 6)  # up, gate, down, x, gain_in, gain_sub
+
+    def make_w(self, which: str, seed: int = 0) -> np.ndarray:
+        i = {"up": 0, "gate": 1, "down": 2}[which]
+        N, K = (self.D, self.F) if which == "down" else (self.F, self.D)
+        return weights(N, K, self.w_sigma, seed, self.ids[i])
+
+    def make_x(self, seed: int = 0) -> np.ndarray:
+        return activations(self.M, self.D, seed, self.ids[3], "normal", self.outlier_frac, self.outlier_scale, "bf16")
+
+    def make_gains(self, seed: int = 0):
+        return gain(self.D, seed, self.ids[4], "bf16"), gain(self.F, seed, self.ids[5], "bf16")
+
+    @property
+    def weight_bytes(self) -> int:
+        return 3 * self.F * self.D // 4
+
+
+FFN_BLOCKS = {
+    # the 2.5B-class FFN (up/gate 2560 -> 6912, down 6912 -> 2560) at decode, 1% outlier channels x20
+    "ffn_block_m1_2p5b": FfnBlock("ffn_block_m1_2p5b", 1, 2560, 6912, 0.02, 0.01, 20.0, (51, 55, 61, 52, 53, 63)),
+    # the 27B-class FFN (up/gate 5376 -> 21504, down 21504 -> 5376), 0.5% outlier channels x30
+    "ffn_block_m1_27b": FfnBlock("ffn_block_m1_27b", 1, 5376, 21504, 0.01, 0.005, 30.0, (91, 95, 101, 92, 93, 103)),
+}

@@ -202,6 +202,62 @@ bitnet_status bitnet_bitlinear_gemv(const void* x, int x_dtype, const void* rms_
                                     const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, int64_t M,
                                     void* y, int y_dtype, void* stream);
 
+/* Bytes of the grid-barrier workspace that bitnet_bitlinear_ffn_gemv takes. */
+#define BITNET_FFN_SYNC_BYTES 64
+
+/*
+ * Decode feed-forward block of BitNet b1.58 for M <= 8 tokens, in one
+ * launch.  The block is three BitLinears with squared-ReLU gating
+ * (inferownia.pl, "BitNet b1.58: era 1-bitowych LLM-ów", section "Zrób to
+ * sam": squared ReLU in the FFN, subln normalisation, no biases; kripta.biz
+ * BitNet b1.58 2B4T news: ReLU^2 in the FFN layers); each BitLinear
+ * normalises and quantises its input, multiplies by the ternary weights and
+ * rescales (comrad404.com review, section "Метод"):
+ *
+ *   u = BitLinear(x; W_up, gamma_up, rms_gain_in)      fp32, as bitnet_bitlinear_gemv
+ *   g = BitLinear(x; W_gate, gamma_gate, rms_gain_in)  fp32
+ *   h = bf16_RNE(RN32(RN32(r * r) * u)),  r = g if g > 0, else +0
+ *   y = BitLinear(h; W_down, gamma_down, rms_gain_sub) y_dtype
+ *
+ * Results are identical to two bitnet_bitlinear_gemv calls with F32 output,
+ * the gating step, and a third bitnet_bitlinear_gemv on h.
+ *
+ * x            [in]  M x D bf16 token rows (x_dtype must be BITNET_BF16).
+ * M, D, F      [in]  1 <= M <= 8; D (hidden) and F (FFN width) positive
+ *                    multiples of 64, each <= 24576; shapes whose working set
+ *                    does not fit one SM's shared memory (roughly M * max(D, F)
+ *                    above 140000 bytes) return BITNET_ERR_UNSUPPORTED_SHAPE.
+ * rms_gain_in  [in]  D bf16 RMSNorm gain of x, or NULL for no norm; rms_eps_in
+ *                    finite and > 0 when given.
+ * W_up, W_gate [in]  F x D/4 packed (bitnet_pack_weights of F x D matrices),
+ *                    gamma_up, gamma_gate their scales (device float[1]).
+ * rms_gain_sub [in]  F bf16 RMSNorm gain of h (the sub-layer norm), or NULL;
+ *                    rms_eps_sub finite and > 0 when given.
+ * W_down       [in]  D x F/4 packed, gamma_down its scale.
+ * h            [out] M x F bf16: the down projection's input.
+ * y            [out] M x D of dtype y_dtype (BITNET_F32, BITNET_BF16, or
+ *                    BITNET_I32 for the raw int32 accumulator of W_down).
+ * sync         [in,out] BITNET_FFN_SYNC_BYTES bytes of device memory, 8-byte
+ *                    aligned, zero-filled by the caller before the first call
+ *                    (its first 8 bytes count barrier arrivals).  Calls in one
+ *                    stream may share it; calls that can run at the same time
+ *                    (other streams) must not.  The call leaves it ready for
+ *                    the next call, except after a BITNET_ERR_TIMEOUT, when it
+ *                    must be zero-filled again.
+ * Pointers: x, gains, W_*, h, y 16-byte aligned; gammas 4-byte aligned; h
+ * and y must not overlap the inputs.
+ * The kernel is a cooperative launch of one CTA per SM (its CTAs wait for
+ * one another once, between the gating and the down projection; that wait is
+ * bounded and reports BITNET_ERR_TIMEOUT through bitnet_get_device_status).
+ * Asynchronous.
+ */
+bitnet_status bitnet_bitlinear_ffn_gemv(const void* x, int x_dtype, int64_t M, int64_t D, int64_t F,
+                                        const void* rms_gain_in, float rms_eps_in, const uint8_t* W_up,
+                                        const float* gamma_up, const uint8_t* W_gate, const float* gamma_gate,
+                                        const void* rms_gain_sub, float rms_eps_sub, const uint8_t* W_down,
+                                        const float* gamma_down, void* h, void* y, int y_dtype, void* sync,
+                                        void* stream);
+
 /*
  * Synchronises `stream`, then reports and clears the device-side error word
  * that kernels set when a bounded wait on a barrier runs out (they then skip

@@ -117,6 +117,29 @@ def test_fused_rejects_bad_arguments(L):
     assert call(N=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
 
 
+def test_ffn_rejects_bad_arguments(L):
+    def call(x=FAKE, dt=bl.BITNET_BF16, M=1, D=64, F=128, gi=None, ei=1e-5, Wu=FAKE, gu=FAKE, Wg=FAKE, gg=FAKE,
+             gs=None, es=1e-5, Wd=FAKE, gd=FAKE, h=FAKE, y=FAKE, yd=bl.BITNET_BF16, sync=FAKE):
+        return L.bitnet_bitlinear_ffn_gemv(x, dt, M, D, F, gi, ei, Wu, gu, Wg, gg, gs, es, Wd, gd, h, y, yd, sync,
+                                           None)
+
+    for kw in ({"x": None}, {"Wu": None}, {"gg": None}, {"Wd": None}, {"h": None}, {"y": None}, {"sync": None}):
+        assert call(**kw) == bl.BITNET_ERR_INVALID_ARG, kw
+    for kw in ({"x": MIS}, {"Wg": MIS}, {"h": MIS}, {"gi": MIS}, {"sync": FAKE + 4}, {"gd": FAKE + 2}):
+        assert call(**kw) == bl.BITNET_ERR_INVALID_ARG, kw
+    assert call(dt=bl.BITNET_F32) == bl.BITNET_ERR_INVALID_ARG  # bf16 activations only
+    assert call(yd=7) == bl.BITNET_ERR_INVALID_ARG
+    assert call(gi=FAKE, ei=0.0) == bl.BITNET_ERR_INVALID_ARG
+    assert call(gs=FAKE, es=float("inf")) == bl.BITNET_ERR_INVALID_ARG
+    assert call(M=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(M=9) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(D=96) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(F=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(F=24576 + 64) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    # the quantised rows of h (8 x 24576 bytes) do not fit beside a 2-slot ring
+    assert call(M=8, F=24576) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(bl, "_lib", None)
     monkeypatch.setattr(bl, "LIB_PATH", str(tmp_path / "missing.so"))
