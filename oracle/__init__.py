@@ -62,6 +62,14 @@ def lib() -> ctypes.CDLL:
         L.oracle_f32_to_bf16.restype = None
         L.oracle_relu2_gate.argtypes = [P, P, I64, P]
         L.oracle_relu2_gate.restype = None
+        L.oracle_b3_padded_k.argtypes = [I64]
+        L.oracle_b3_padded_k.restype = I64
+        L.oracle_pack_codes_b3.argtypes = [P, I64, I64, P]
+        L.oracle_pack_codes_b3.restype = None
+        L.oracle_unpack_codes_b3.argtypes = [P, I64, I64, P]
+        L.oracle_unpack_codes_b3.restype = I64
+        L.oracle_bitlinear_b3.argtypes = [P, F, I64, I64, P, P, I64, P, P]
+        L.oracle_bitlinear_b3.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -225,3 +233,46 @@ def ffn(x: np.ndarray, up, gate, down, gain_in=None, eps_in: float = 1e-5, gain_
     h_bits = f32_to_bf16(relu2_gate(u, g))
     acc, y = bitlinear_forward(bf16_to_f32(h_bits), down[0], down[1], gain_sub, eps_sub)
     return h_bits, acc, y
+
+
+def b3_padded_k(K: int) -> int:
+    return int(lib().oracle_b3_padded_k(K))
+
+
+def pack_codes_b3(q: np.ndarray) -> np.ndarray:
+    """Base-3 packing of ternary codes (N x K int8) -> N x b3_padded_k(K)/5 bytes."""
+    q = np.ascontiguousarray(q, dtype=np.int8)
+    N, K = q.shape
+    out = np.empty((N, b3_padded_k(K) // 5), dtype=np.uint8)
+    lib().oracle_pack_codes_b3(_p(q), N, K, _p(out))
+    return out
+
+
+def unpack_codes_b3(packed: np.ndarray, K: int):
+    """Returns (q int8 N x K, number of invalid bytes or non-zero padded codes)."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    N = packed.shape[0]
+    q = np.empty((N, K), dtype=np.int8)
+    bad = lib().oracle_unpack_codes_b3(_p(packed), N, K, _p(q))
+    return q, int(bad)
+
+
+def pack_weights_b3(W: np.ndarray, eps: float):
+    """Absmean ternarisation + base-3 packing.  Returns (packed, gamma)."""
+    q, g = ternarize(W, eps)
+    return pack_codes_b3(q), g
+
+
+def bitlinear_b3(packed: np.ndarray, gamma, K: int, xq: np.ndarray, a: np.ndarray):
+    """The BitLinear product against base-3 packed weights.  Returns (acc int32, y fp32)."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    xq = np.ascontiguousarray(xq, dtype=np.int8)
+    a = _f32(a)
+    N = packed.shape[0]
+    M = xq.shape[0]
+    acc = np.empty((M, N), dtype=np.int32)
+    y = np.empty((M, N), dtype=np.float32)
+    st = lib().oracle_bitlinear_b3(_p(packed), np.float32(gamma), N, K, _p(xq), _p(a), M, _p(acc), _p(y))
+    if st != 0:
+        raise ValueError(f"oracle_bitlinear_b3 status {st}")
+    return acc, y

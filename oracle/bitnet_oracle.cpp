@@ -241,6 +241,67 @@ int oracle_bitlinear_sampled(const uint8_t* packed, float gamma, int64_t N, int6
   return 0;
 }
 
+// Base-3 storage of the ternary codes ([Explainer, "Skąd te 1,58 bita": a
+// ternary weight carries log2(3) ~ 1.58 bits of information; Habr repost,
+// "Когда - три лучше двух": log2(3) bits per parameter).  Five codes
+// c = q + 1 in {0,1,2} fit in one byte as a base-3 number (3^5 = 243 <= 256),
+// 1.6 bits per weight.  Layout (this library's own): a row is padded with
+// zero weights to Kp = ceil(K/80)*80 and stored as Kp/80 groups of 16 bytes;
+// byte i of group g is sum_{t=0..4} c[80g + 16t + i] * 3^t.
+int64_t oracle_b3_padded_k(int64_t K) { return (K + 79) / 80 * 80; }
+
+void oracle_pack_codes_b3(const int8_t* q, int64_t N, int64_t K, uint8_t* packed) {
+  const int64_t Kp = oracle_b3_padded_k(K), rb = Kp / 5;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t g = 0; g < Kp / 80; ++g)
+      for (int i = 0; i < 16; ++i) {
+        int v = 0, p3 = 1;
+        for (int t = 0; t < 5; ++t) {
+          const int64_t k = 80 * g + 16 * t + i;
+          const int c = k < K ? q[n * K + k] + 1 : 1;
+          v += c * p3;
+          p3 *= 3;
+        }
+        packed[n * rb + 16 * g + i] = static_cast<uint8_t>(v);
+      }
+}
+
+// Inverse of oracle_pack_codes_b3 for the first K weights of each row;
+// returns the number of bytes above 242 (not a valid base-3 group) plus the
+// number of padded positions whose code is not 1 (q = 0).
+int64_t oracle_unpack_codes_b3(const uint8_t* packed, int64_t N, int64_t K, int8_t* q) {
+  const int64_t Kp = oracle_b3_padded_k(K), rb = Kp / 5;
+  int64_t bad = 0;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t g = 0; g < Kp / 80; ++g)
+      for (int i = 0; i < 16; ++i) {
+        int v = packed[n * rb + 16 * g + i];
+        if (v > 242) ++bad;
+        for (int t = 0; t < 5; ++t) {
+          const int c = v % 3;
+          v /= 3;
+          const int64_t k = 80 * g + 16 * t + i;
+          if (k < K) q[n * K + k] = static_cast<int8_t>(c - 1);
+          else if (c != 1) ++bad;
+        }
+      }
+  return bad;
+}
+
+// The BitLinear product against base-3 packed weights: the same exact dot
+// product and dequant as oracle_bitlinear, on the decoded codes.
+int oracle_bitlinear_b3(const uint8_t* packed, float gamma, int64_t N, int64_t K,
+                        const int8_t* xq, const float* a, int64_t M, int32_t* acc, float* y) {
+  const int64_t rb = oracle_b3_padded_k(K) / 5;
+  std::vector<int8_t> q(static_cast<size_t>(K));
+  for (int64_t n = 0; n < N; ++n) {
+    if (oracle_unpack_codes_b3(packed + n * rb, 1, K, q.data()) != 0) return 2;
+    for (int64_t m = 0; m < M; ++m)
+      if (oracle_dot(q.data(), xq + m * K, K, gamma, a[m], &acc[m * N + n], &y[m * N + n]) != 0) return 1;
+  }
+  return 0;
+}
+
 // Squared-ReLU gating of the feed-forward block: the FFN of BitNet b1.58
 // uses a squared ReLU as its activation ([Explainer, "Zrób to sam": squared
 // ReLU in the FFN, subln normalisation, no biases]; kripta.biz 2B4T news:
