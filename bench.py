@@ -470,6 +470,11 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
     if not args.no_prefill and lins[0].M <= 8:
         prefill = bench_prefill(torch, bl, dev, stream, peaks, peak_src, group)
 
+    # ---- the decode step on base-3 packed weights, a secondary line
+    decode_b3 = None
+    if not args.no_b3 and use_fused and all(l.M * ((l.K + 79) // 80 * 80) <= 24000 for l in lins):
+        decode_b3 = bench_b3(torch, bl, dev, stream, lins, xs, gains, peaks, peak_src, group, el_ms / K)
+
     # ---- the one-launch decode FFN block (up, gate, squared-ReLU gating, down), a secondary line
     ffn_block = None
     if not args.no_ffn and lins[0].M <= 8:
@@ -515,12 +520,57 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
                                                         for l, ms in zip(lins, pack_ms)]},
             "prefill": prefill,
             "ffn_block": ffn_block,
+            "decode_b3": decode_b3,
         }
         print(json.dumps(line), flush=True)
     if group:
         import torch.distributed as dist
         del g_main, g_rem
         dist.destroy_process_group()
+
+
+def bench_b3(torch, bl, dev, stream, lins, xs, gains, peaks, peak_src, group, two_bit_step_ms):
+    """The decode step with base-3 packed weights (bitnet_bitlinear_gemv_b3, five codes per byte): same
+    linears, inputs, weight rotation and graphs as the 2-bit step; GB/s on the base-3 byte count."""
+    packs = []
+    for lin in lins:
+        W = torch.from_numpy(lin.make_w(0)).to(dev)
+        P, G = bl.bitnet_pack_weights_b3(W, EPS_W)
+        del W
+        packs.append(([P] + [P.clone() for _ in range(COPIES - 1)], G))
+    ys = [torch.empty((l.M, l.N), dtype=torch.bfloat16 if l.y_dtype == "bf16" else torch.float32, device=dev)
+          for l in lins]
+
+    def step(c):
+        for i in range(len(lins)):
+            bl.bitnet_bitlinear_gemv_b3(xs[i], packs[i][0][c % COPIES], packs[i][1], gains[i], EPS_RMS, y=ys[i])
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for c in range(GRAPH_STEPS):
+            step(c)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            g.replay()
+    torch.cuda.synchronize(dev)
+    reps = 40
+    barrier(group, dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(group, dev)
+    ms = max_over_ranks(e0.elapsed_time(e1), group, dev) / (reps * GRAPH_STEPS)
+    b3_bytes = sum(l.N * bl.bitnet_b3_row_bytes(l.K) for l in lins)
+    step_bytes = b3_bytes + sum(linear_bytes(l)["x_in"] + 4 + linear_bytes(l)["y_out"] for l in lins)
+    gbs = step_bytes / (ms / 1e3) / 1e9
+    return {"us_per_step": ms * 1e3, "gbs": gbs, "frac": gbs / float(peaks["hbm_gbs"]),
+            "weight_bytes_per_step": b3_bytes, "two_bit_us_per_step": two_bit_step_ms * 1e3,
+            "device_status": bl.bitnet_get_device_status(),
+            "timing": f"CUDA graphs of {GRAPH_STEPS} steps over {COPIES} rotating weight copies, per step"}
 
 
 def bench_ffn_block(torch, bl, dev, stream, peaks, peak_src, group, name="ffn_block_m1_2p5b"):
@@ -646,6 +696,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-prefill", action="store_true", help="skip the secondary prefill GEMM measurement")
     ap.add_argument("--no-ffn", action="store_true", help="skip the secondary one-launch FFN block measurement")
+    ap.add_argument("--no-b3", action="store_true", help="skip the secondary base-3 decode measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

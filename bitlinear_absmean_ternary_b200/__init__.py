@@ -62,6 +62,12 @@ def lib() -> ctypes.CDLL:
         L.bitnet_bitlinear_gemv.restype = I
         L.bitnet_bitlinear_ffn_gemv.argtypes = [P, I, I64, I64, I64, P, F, P, P, P, P, P, F, P, P, P, P, I, P, P]
         L.bitnet_bitlinear_ffn_gemv.restype = I
+        L.bitnet_b3_row_bytes.argtypes = [I64]
+        L.bitnet_b3_row_bytes.restype = ctypes.c_size_t
+        L.bitnet_pack_weights_b3.argtypes = [P, I64, I64, F, P, P, P, ctypes.c_size_t, P]
+        L.bitnet_pack_weights_b3.restype = I
+        L.bitnet_bitlinear_gemv_b3.argtypes = [P, I, P, F, P, P, I64, I64, I64, P, I, P]
+        L.bitnet_bitlinear_gemv_b3.restype = I
         L.bitnet_get_device_status.argtypes = [P]
         L.bitnet_get_device_status.restype = I
         L.bitnet_status_string.argtypes = [I]
@@ -243,6 +249,49 @@ def bitnet_bitlinear_ffn_gemv(x, W_up, gamma_up, W_gate, gamma_gate, W_down, gam
                                          _ptr(y), _dtype_code(y.dtype), _ptr(sync), _stream(x.device))
     _check("bitnet_bitlinear_ffn_gemv", st)
     return h, y
+
+
+def bitnet_b3_row_bytes(K: int) -> int:
+    return int(lib().bitnet_b3_row_bytes(K))
+
+
+def bitnet_pack_weights_b3(W, eps: float = 1e-5, W_b3=None, gamma=None, workspace=None):
+    """Absmean ternarisation + base-3 packing (5 codes per byte) of fp32 W (N x K).
+    Returns (W_b3 uint8 N x bitnet_b3_row_bytes(K), gamma float32 [1]).  Synchronises."""
+    torch = _torch()
+    _need_cuda(W)
+    N, K = W.shape
+    rb = bitnet_b3_row_bytes(K)
+    if rb == 0:
+        raise ValueError("K must be a positive multiple of 64")
+    if W_b3 is None:
+        W_b3 = torch.empty((N, rb), dtype=torch.uint8, device=W.device)
+    if gamma is None:
+        gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    nbytes = bitnet_pack_workspace_bytes(N, K)
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=W.device)
+    _need_cuda(W_b3, gamma, workspace)
+    st = lib().bitnet_pack_weights_b3(_ptr(W), N, K, eps, _ptr(W_b3), _ptr(gamma), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(W.device))
+    _check("bitnet_pack_weights_b3", st)
+    return W_b3, gamma
+
+
+def bitnet_bitlinear_gemv_b3(x, W_b3, gamma, rms_gain=None, rms_eps: float = 1e-5, y=None, out_dtype=None):
+    """Fused decode BitLinear (M <= 8) on base-3 packed weights.  Returns y (M x N)."""
+    torch = _torch()
+    _need_cuda(x, rms_gain, W_b3, gamma, y)
+    M, K = x.shape
+    N = W_b3.shape[0]
+    if W_b3.shape[1] != bitnet_b3_row_bytes(K):
+        raise ValueError("x and W_b3 disagree on K")
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype or torch.bfloat16, device=x.device)
+    st = lib().bitnet_bitlinear_gemv_b3(_ptr(x), _dtype_code(x.dtype), _ptr(rms_gain), rms_eps, _ptr(W_b3),
+                                        _ptr(gamma), N, K, M, _ptr(y), _dtype_code(y.dtype), _stream(x.device))
+    _check("bitnet_bitlinear_gemv_b3", st)
+    return y
 
 
 def bitnet_get_device_status(device=None) -> int:

@@ -14,6 +14,7 @@
 #include "ffn.cuh"
 #include "gemm.cuh"
 #include "gemv.cuh"
+#include "gemv_b3.cuh"
 #include "pack.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
@@ -400,6 +401,50 @@ int ffn_slots(int M, int D, int F, int G) {
   return sl >= 2 ? sl : 0;
 }
 
+// Fused decode BitLinear on base-3 packed weights.
+constexpr int kGemvB3XMaxBytes = 24000;  // M * Kp: the quantised, zero-padded token rows in shared memory
+
+template <int MT, typename T, int MAXC>
+cudaError_t launch_b3_t(const void* x, const void* gain, float eps, const uint8_t* Wp, const float* gamma, int N,
+                        int K, void* y, int yd, cudaStream_t s) {
+  static bool done[kMaxDevices] = {};
+  auto kern = gemv_b3_kernel<MT, T, MAXC>;
+  const cudaError_t e = set_smem(kern, gemv_b3_smem_bytes(MT, kGemvB3XMaxBytes / MT), done);
+  if (e != cudaSuccess) return e;
+  const int64_t groups = (N + kGemvRows - 1) / kGemvRows;
+  const int grid = static_cast<int>(groups < sm_count() ? groups : sm_count());
+  return launch_pdl(kern, dim3(grid), dim3(kGemvThreads), gemv_b3_smem_bytes(MT, b3_padded_k(K)), s, Wp, gamma, N,
+                    K, static_cast<const T*>(x), static_cast<const T*>(gain), eps, y, yd);
+}
+
+template <int MT, typename T>
+cudaError_t launch_b3_c(const void* x, const void* gain, float eps, const uint8_t* Wp, const float* gamma, int N,
+                        int K, void* y, int yd, cudaStream_t s) {
+  const int per_thread = (K / 8 + kQuantThreads - 1) / kQuantThreads;
+  if (per_thread <= 2) return launch_b3_t<MT, T, 2>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+  if (per_thread <= 4) return launch_b3_t<MT, T, 4>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+  if constexpr (sizeof(T) == 2) {
+    if (per_thread <= 12) return launch_b3_t<MT, T, 12>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <typename T>
+cudaError_t launch_b3(int M, const void* x, const void* gain, float eps, const uint8_t* Wp, const float* gamma,
+                      int N, int K, void* y, int yd, cudaStream_t s) {
+  switch (M) {
+    case 1: return launch_b3_c<1, T>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+    case 2: return launch_b3_c<2, T>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+    case 3: return launch_b3_c<3, T>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+    case 4: return launch_b3_c<4, T>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+    case 5: return launch_b3_c<5, T>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+    case 6: return launch_b3_c<6, T>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+    case 7: return launch_b3_c<7, T>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+    case 8: return launch_b3_c<8, T>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 bitnet_status check_linear(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K, const int8_t* xq,
                            const float* a, const int32_t* rs, int64_t M, void* y, int yd) {
   if (Wp == nullptr || gamma == nullptr || xq == nullptr || a == nullptr || y == nullptr) return BITNET_ERR_INVALID_ARG;
@@ -478,6 +523,60 @@ bitnet_status bitnet_pack_weights(const float* W, int64_t N, int64_t K, float ep
     return BITNET_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return BITNET_ERR_CUDA;
   return host_flag != 0 ? BITNET_ERR_NONFINITE : BITNET_OK;
+}
+
+size_t bitnet_b3_row_bytes(int64_t K) {
+  if (!valid_k(K)) return 0;
+  return static_cast<size_t>((K + 79) / 80 * 80 / 5);
+}
+
+bitnet_status bitnet_pack_weights_b3(const float* W, int64_t N, int64_t K, float eps, uint8_t* W_b3, float* gamma,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (W == nullptr || W_b3 == nullptr || gamma == nullptr || workspace == nullptr) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(W_b3, 16) || !aligned(gamma, 4) || !aligned(workspace, 16))
+    return BITNET_ERR_INVALID_ARG;
+  if (!std::isfinite(eps) || !(eps > 0.0f)) return BITNET_ERR_INVALID_ARG;
+  if (!valid_k(K) || K > kGemvB3XMaxBytes || N < 1 || N > (int64_t{1} << 31) || N * K > (int64_t{1} << 40))
+    return BITNET_ERR_UNSUPPORTED_SHAPE;
+  if (workspace_bytes < bitnet_pack_workspace_bytes(N, K)) return BITNET_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  double* rowsum = static_cast<double*>(workspace);
+  float* d = reinterpret_cast<float*>(rowsum + N);
+  unsigned int* flag = reinterpret_cast<unsigned int*>(d + 1);
+
+  if (cudaMemsetAsync(flag, 0, sizeof(unsigned int), s) != cudaSuccess) return BITNET_ERR_CUDA;
+  const int blocks1 = static_cast<int>(std::min<int64_t>((N + 7) / 8, int64_t{sm_count()} * 8));
+  pack_rowsum_kernel<<<blocks1, 256, 0, s>>>(W, N, K, rowsum, flag);
+  pack_gamma_kernel<<<1, 32, 0, s>>>(rowsum, N, K, eps, gamma, d);
+  const int rb = static_cast<int>(bitnet_b3_row_bytes(K));
+  const int blocks3 = static_cast<int>(std::min<int64_t>((N * rb + 255) / 256, int64_t{sm_count()} * 16));
+  pack_codes_b3_kernel<<<blocks3, 256, 0, s>>>(W, N, static_cast<int>(K), rb, d, W_b3);
+  if (cudaGetLastError() != cudaSuccess) return BITNET_ERR_CUDA;
+  unsigned int host_flag = 0;
+  if (cudaMemcpyAsync(&host_flag, flag, sizeof(host_flag), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BITNET_ERR_CUDA;
+  return host_flag != 0 ? BITNET_ERR_NONFINITE : BITNET_OK;
+}
+
+bitnet_status bitnet_bitlinear_gemv_b3(const void* x, int x_dtype, const void* rms_gain, float rms_eps,
+                                       const uint8_t* W_b3, const float* gamma, int64_t N, int64_t K, int64_t M,
+                                       void* y, int y_dtype, void* stream) {
+  if (x == nullptr || W_b3 == nullptr || gamma == nullptr || y == nullptr) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(rms_gain, 16) || !aligned(W_b3, 16) || !aligned(y, 16) || !aligned(gamma, 4))
+    return BITNET_ERR_INVALID_ARG;
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
+  if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16 && y_dtype != BITNET_I32) return BITNET_ERR_INVALID_ARG;
+  if (rms_gain != nullptr && (!std::isfinite(rms_eps) || !(rms_eps > 0.0f))) return BITNET_ERR_INVALID_ARG;
+  if (!valid_k(K) || N < 1 || N > INT32_MAX || M < 1 || M > 8) return BITNET_ERR_UNSUPPORTED_SHAPE;
+  const int64_t kp = (K + 79) / 80 * 80;
+  if (M * kp > kGemvB3XMaxBytes || (x_dtype == BITNET_F32 && K > 8192)) return BITNET_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int n = static_cast<int>(N), k = static_cast<int>(K), m = static_cast<int>(M);
+  const cudaError_t e = x_dtype == BITNET_BF16
+                            ? launch_b3<__nv_bfloat16>(m, x, rms_gain, rms_eps, W_b3, gamma, n, k, y, y_dtype, s)
+                            : launch_b3<float>(m, x, rms_gain, rms_eps, W_b3, gamma, n, k, y, y_dtype, s);
+  return from_cuda(e);
 }
 
 bitnet_status bitnet_pack_weights_noalloc(const float* W, int64_t N, int64_t K, float eps, uint8_t* W_packed,

@@ -82,4 +82,38 @@ __global__ void __launch_bounds__(256) pack_codes_kernel(const float* __restrict
   }
 }
 
+// Base-3 storage: five codes c = q + 1 per byte as a base-3 number (a
+// ternary weight holds log2(3) ~ 1.58 bits: inferownia.pl, "Skąd te 1,58
+// bita"), 1.6 bits per weight.  A row is padded with zero weights (c = 1) to
+// Kp = ceil(K/80)*80 and stored as groups of 16 bytes; byte i of group g is
+// sum_t c[80g + 16t + i] * 3^t.  One thread per packed byte; q uses the same
+// operations as pack_codes_kernel.
+__global__ void __launch_bounds__(256) pack_codes_b3_kernel(const float* __restrict__ W, int64_t N, int K,
+                                                            int row_bytes, const float* __restrict__ d_ptr,
+                                                            uint8_t* __restrict__ packed) {
+  const float d = *d_ptr;
+  const int64_t total = N * row_bytes;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total; idx += stride) {
+    const int64_t n = idx / row_bytes;
+    const int j = static_cast<int>(idx - n * row_bytes);
+    const int g = j >> 4, i = j & 15;
+    const float* row = W + n * K;
+    int v = 0, p3 = 1;
+#pragma unroll
+    for (int t = 0; t < 5; ++t) {
+      const int k = 80 * g + 16 * t + i;
+      int c = 1;
+      if (k < K) {
+        int q = __float2int_rn(__fdiv_rn(__ldg(row + k), d));
+        q = q < -1 ? -1 : (q > 1 ? 1 : q);
+        c = q + 1;
+      }
+      v += c * p3;
+      p3 *= 3;
+    }
+    packed[idx] = static_cast<uint8_t>(v);
+  }
+}
+
 }  // namespace bitnet

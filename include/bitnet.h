@@ -202,6 +202,34 @@ bitnet_status bitnet_bitlinear_gemv(const void* x, int x_dtype, const void* rms_
                                     const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, int64_t M,
                                     void* y, int y_dtype, void* stream);
 
+/*
+ * Base-3 storage of the ternary codes, 1.6 bits per weight (a ternary weight
+ * holds log2(3) ~ 1.58 bits: inferownia.pl, "BitNet b1.58: era 1-bitowych
+ * LLM-ów", section "Skąd te 1,58 bita"; Habr repost on juhe.plus, section
+ * "Когда - три лучше двух").  Five codes c = q + 1 form one byte as a base-3
+ * number.  A row is padded with zero weights to Kp = ceil(K/80)*80 and stored
+ * as Kp/80 groups of 16 bytes; byte i of group g = sum_{t=0..4} c[80g+16t+i]
+ * 3^t.  Rows are contiguous, bitnet_b3_row_bytes(K) = Kp/5 bytes each
+ * (K = 2560: 512 bytes; K = 6912: 1392 bytes), 20% fewer than the 2-bit
+ * layout when K is a multiple of 80.
+ *
+ * bitnet_b3_row_bytes: bytes per packed row, 0 for an unsupported K.
+ * bitnet_pack_weights_b3: as bitnet_pack_weights (same gamma, same codes,
+ *   same workspace and errors; K <= 24000), writing N x bitnet_b3_row_bytes(K)
+ *   bytes to W_b3.  Synchronises.
+ * bitnet_bitlinear_gemv_b3: as bitnet_bitlinear_gemv (fused quantisation and
+ *   product for M <= 8 tokens) on base-3 packed weights; requires
+ *   M * Kp <= 24000 (and K <= 8192 for fp32 x).  Results identical to
+ *   bitnet_bitlinear_gemv on the 2-bit packing of the same matrix.
+ *   Asynchronous.
+ */
+size_t bitnet_b3_row_bytes(int64_t K);
+bitnet_status bitnet_pack_weights_b3(const float* W, int64_t N, int64_t K, float eps, uint8_t* W_b3, float* gamma,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+bitnet_status bitnet_bitlinear_gemv_b3(const void* x, int x_dtype, const void* rms_gain, float rms_eps,
+                                       const uint8_t* W_b3, const float* gamma, int64_t N, int64_t K, int64_t M,
+                                       void* y, int y_dtype, void* stream);
+
 /* Bytes of the grid-barrier workspace that bitnet_bitlinear_ffn_gemv takes. */
 #define BITNET_FFN_SYNC_BYTES 64
 

@@ -140,6 +140,29 @@ def test_ffn_rejects_bad_arguments(L):
     assert call(M=8, F=24576) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
 
 
+def test_b3_rejects_bad_arguments(L):
+    assert bl.bitnet_b3_row_bytes(2560) == 512 and bl.bitnet_b3_row_bytes(6912) == 1392
+    assert bl.bitnet_b3_row_bytes(64) == 16 and bl.bitnet_b3_row_bytes(100) == 0
+    assert L.bitnet_pack_weights_b3(None, 4, 64, 1e-5, FAKE, FAKE, FAKE, 1 << 20, None) == bl.BITNET_ERR_INVALID_ARG
+    assert L.bitnet_pack_weights_b3(FAKE, 4, 64, 0.0, FAKE, FAKE, FAKE, 1 << 20, None) == bl.BITNET_ERR_INVALID_ARG
+    assert L.bitnet_pack_weights_b3(FAKE, 4, 96, 1e-5, FAKE, FAKE, FAKE, 1 << 20, None) == \
+        bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert L.bitnet_pack_weights_b3(FAKE, 4, 64, 1e-5, FAKE, FAKE, FAKE, 8, None) == bl.BITNET_ERR_INVALID_ARG
+
+    def call(x=FAKE, dt=bl.BITNET_BF16, g=None, eps=1e-5, W=FAKE, gam=FAKE, N=8, K=64, M=1, y=FAKE,
+             yd=bl.BITNET_BF16):
+        return L.bitnet_bitlinear_gemv_b3(x, dt, g, eps, W, gam, N, K, M, y, yd, None)
+
+    assert call(x=None) == bl.BITNET_ERR_INVALID_ARG
+    assert call(W=MIS) == bl.BITNET_ERR_INVALID_ARG
+    assert call(dt=bl.BITNET_I32) == bl.BITNET_ERR_INVALID_ARG
+    assert call(g=FAKE, eps=-1.0) == bl.BITNET_ERR_INVALID_ARG
+    assert call(M=9) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(K=100) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(M=2, K=21504) == bl.BITNET_ERR_UNSUPPORTED_SHAPE  # 2 x 21520 padded rows > 24000
+    assert call(dt=bl.BITNET_F32, K=8192 + 64) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(bl, "_lib", None)
     monkeypatch.setattr(bl, "LIB_PATH", str(tmp_path / "missing.so"))
