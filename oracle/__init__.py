@@ -276,3 +276,51 @@ def bitlinear_b3(packed: np.ndarray, gamma, K: int, xq: np.ndarray, a: np.ndarra
     if st != 0:
         raise ValueError(f"oracle_bitlinear_b3 status {st}")
     return acc, y
+
+
+# ----------------------------------------------------------------------------
+# Straight-through estimator (STE) backward of the BitLinear.
+#
+# Training keeps full-precision latent weights and lets the forward use the
+# rounded ones (Habr repost on juhe.plus, section "А откуда взялась сама
+# идея?": the precise values accumulate the small updates, the computation
+# uses the coarse ones); the rounding step has a zero derivative almost
+# everywhere, so the backward pass treats it as absent and passes the
+# gradient straight through (same page, section "Когда - три лучше двух":
+# forward with the real rounding, backward as if it were not there).  The forward used W_hat = gamma * q and x_hat[m] = a[m] *
+# x_q[m] (y = x_hat W_hat^T), so with the quantisers treated as identities:
+#   dX[m, k] = sum_n dY[m, n] * gamma * q[n, k]     (gradient at the quantiser input)
+#   dW[n, k] = sum_m dY[m, n] * a[m] * x_q[m, k]    (gradient reaching the latent W)
+# Reading of the precision: dY is bf16 (bf16 training); dX = RN32(gamma * S)
+# with S the exact sum; the weight-gradient product takes bf16 operands, so
+# its left operand is dYs = bf16_RNE(RN32(dY * a[m])) and dW = RN32(exact sum
+# of dYs * x_q).  The sums use numpy's fp64 matmul as a primitive: every
+# product and partial sum here is exact in fp64 for |dY| below 2^60.
+
+
+def ste_backward_input(dY: np.ndarray, packed: np.ndarray, gamma, K: int) -> np.ndarray:
+    """dX = RN32(gamma * (dY @ q)), dY: M x N fp32 values (bf16 values in use)."""
+    q, bad = unpack_codes(packed, K)
+    if bad:
+        raise ValueError("packed weights hold an illegal code")
+    S = np.asarray(dY, np.float64) @ q.astype(np.float64)
+    return (np.float32(gamma).astype(np.float64) * S).astype(np.float32)
+
+
+def ste_scale_grad(dY: np.ndarray, a: np.ndarray) -> np.ndarray:
+    """dYs = bf16_RNE(RN32(dY[m, n] * a[m])) as bf16 bit patterns."""
+    dY = _f32(dY)
+    a = _f32(a)
+    return f32_to_bf16((dY * a[:, None]).astype(np.float32))
+
+
+def ste_backward_weight(dY: np.ndarray, xq: np.ndarray, a: np.ndarray) -> np.ndarray:
+    """dW = RN32(sum_m dYs[m, n] * x_q[m, k]) with dYs = ste_scale_grad(dY, a); N x K fp32."""
+    dYs = bf16_to_f32(ste_scale_grad(dY, a)).astype(np.float64)
+    return (dYs.T @ np.asarray(xq, np.float64)).astype(np.float32)
+
+
+def ste_backward_weight_exact(dY: np.ndarray, xq: np.ndarray, a: np.ndarray) -> np.ndarray:
+    """The same sum without the bf16 rounding of the left operand, in fp64."""
+    x_hat = np.asarray(xq, np.float64) * np.asarray(a, np.float64)[:, None]
+    return np.asarray(dY, np.float64).T @ x_hat
