@@ -470,6 +470,11 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
     if not args.no_prefill and lins[0].M <= 8:
         prefill = bench_prefill(torch, bl, dev, stream, peaks, peak_src, group)
 
+    # ---- STE backward GEMMs at the prefill shapes, a secondary line
+    ste = None
+    if not args.no_ste and lins[0].M <= 8:
+        ste = bench_ste(torch, bl, dev, stream, peaks, peak_src, group)
+
     # ---- the decode step on base-3 packed weights, a secondary line
     decode_b3 = None
     if not args.no_b3 and use_fused and all(l.M * ((l.K + 79) // 80 * 80) <= 24000 for l in lins):
@@ -521,6 +526,7 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
             "prefill": prefill,
             "ffn_block": ffn_block,
             "decode_b3": decode_b3,
+            "ste_backward": ste,
         }
         print(json.dumps(line), flush=True)
     if group:
@@ -571,6 +577,57 @@ def bench_b3(torch, bl, dev, stream, lins, xs, gains, peaks, peak_src, group, tw
             "weight_bytes_per_step": b3_bytes, "two_bit_us_per_step": two_bit_step_ms * 1e3,
             "device_status": bl.bitnet_get_device_status(),
             "timing": f"CUDA graphs of {GRAPH_STEPS} steps over {COPIES} rotating weight copies, per step"}
+
+
+def bench_ste(torch, bl, dev, stream, peaks, peak_src, group):
+    """Straight-through-estimator backward GEMMs (tcgen05 kind::f16, bf16 operands, fp32 accumulation) at the
+    prefill shapes, M = 4096 tokens: input gradient dX = gamma dY q and weight gradient dW = bf16(dY a)^T x_q,
+    per-launch CUDA-event time with L2 flushed (256 MB write) before each launch."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    bf16_peak = float(peaks["bf16_tflops"])
+    out, tot_flop, tot_ms = {}, 0, 0.0
+    for lin in synth.WORKLOADS["prefill_m4096_2p5b_ffn"]:
+        M, N, K = lin.M, lin.N, lin.K
+        W = torch.from_numpy(lin.make_w(0)).to(dev)
+        P, G = bl.bitnet_pack_weights(W, EPS_W)
+        del W
+        x = torch.from_numpy(synth.f32_to_bf16_bits(lin.make_x(0)).view(np.int16).copy()).to(dev).view(torch.bfloat16)
+        dY = torch.from_numpy(synth.f32_to_bf16_bits(synth.activations(M, N, 0, 99, "normal", 0.0, 1.0, "bf16"))
+                              .view(np.int16).copy()).to(dev).view(torch.bfloat16)
+        with torch.cuda.stream(stream):
+            xq, a, _ = bl.bitnet_quant_act(x, None, EPS_RMS)
+            dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+            dW = torch.empty((N, K), dtype=torch.float32, device=dev)
+            ws = torch.empty(bl.bitnet_ste_weight_workspace_bytes(M, N), dtype=torch.uint8, device=dev)
+            tx, tw = [], []
+            for it in range(13):
+                flush.zero_()
+                e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                e0.record(stream)
+                bl.bitnet_ste_backward_input(P, G, dY, dX=dX)
+                e1.record(stream)
+                flush.zero_()
+                e2.record(stream)
+                e3 = torch.cuda.Event(enable_timing=True)
+                bl.bitnet_ste_backward_weight(dY, xq, a, dW=dW, workspace=ws)
+                e3.record(stream)
+                torch.cuda.synchronize(dev)
+                if it >= 3:
+                    tx.append(e0.elapsed_time(e1))
+                    tw.append(e2.elapsed_time(e3))
+        flop = 2 * M * N * K
+        msx = max_over_ranks(statistics.median(tx), group, dev)
+        msw = max_over_ranks(statistics.median(tw), group, dev)
+        out[f"K{K}_N{N}"] = {"dx_us": msx * 1e3, "dx_tflops": flop / (msx / 1e3) / 1e12,
+                             "dw_us": msw * 1e3, "dw_tflops": flop / (msw / 1e3) / 1e12}
+        tot_flop += 2 * flop
+        tot_ms += msx + msw
+    tf = tot_flop / (tot_ms / 1e3) / 1e12
+    return {"workload": "prefill_m4096_2p5b_ffn", "tflops": tf, "unit": "TFLOP/s",
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": bf16_peak, "unit": "TFLOP/s",
+                         "frac": tf / bf16_peak, "peak_source": f"{peak_src} bf16_tflops"},
+            "per_shape": out, "device_status": bl.bitnet_get_device_status(),
+            "timing": "median of 10 single launches, L2 flushed before each; dW includes its dY*a transpose pre-pass"}
 
 
 def bench_ffn_block(torch, bl, dev, stream, peaks, peak_src, group, name="ffn_block_m1_2p5b"):
@@ -697,6 +754,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true", help="skip the secondary prefill GEMM measurement")
     ap.add_argument("--no-ffn", action="store_true", help="skip the secondary one-launch FFN block measurement")
     ap.add_argument("--no-b3", action="store_true", help="skip the secondary base-3 decode measurement")
+    ap.add_argument("--no-ste", action="store_true", help="skip the secondary STE backward GEMM measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

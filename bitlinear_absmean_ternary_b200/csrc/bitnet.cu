@@ -18,6 +18,7 @@
 #include "pack.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
+#include "ste_gemm.cuh"
 
 namespace {
 
@@ -109,6 +110,20 @@ bool make_map_u8(CUtensorMap* map, const void* base, uint64_t cols, uint64_t row
   const cuuint32_t box[2] = {box_cols, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D bf16 tensor [rows][cols] with row pitch `pitch` bytes, box {box_cols, box_rows}.
+bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t pitch,
+                   uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -445,6 +460,21 @@ cudaError_t launch_b3(int M, const void* x, const void* gain, float eps, const u
   }
 }
 
+// STE backward GEMMs (ste_gemm.cuh): persistent, one CTA per SM.
+template <int MODE>
+cudaError_t launch_ste(const CUtensorMap& mb, const CUtensorMap& ma, const float* scale, int R, int C, int J,
+                       void* out, int od, cudaStream_t s) {
+  static bool done[kMaxDevices] = {};
+  const cudaError_t e = set_smem(ste_gemm_kernel<MODE>, SteCfg<MODE>::kSmemBytes, done);
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = static_cast<int64_t>((R + kSteBM - 1) / kSteBM) * ((C + kSteBN - 1) / kSteBN);
+  const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
+  return launch_pdl(ste_gemm_kernel<MODE>, dim3(grid), dim3(kGemmThreads), SteCfg<MODE>::kSmemBytes, s, mb, ma,
+                    scale, R, C, J, out, od);
+}
+
+int64_t ste_padded_m(int64_t M) { return (M + kSteBJ - 1) / kSteBJ * kSteBJ; }
+
 bitnet_status check_linear(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K, const int8_t* xq,
                            const float* a, const int32_t* rs, int64_t M, void* y, int yd) {
   if (Wp == nullptr || gamma == nullptr || xq == nullptr || a == nullptr || y == nullptr) return BITNET_ERR_INVALID_ARG;
@@ -722,6 +752,59 @@ bitnet_status bitnet_bitlinear_ffn_gemv(const void* x, int x_dtype, int64_t M, i
   const int per_thread = ((d > f ? d : f) / 8 + kQuantThreads - 1) / kQuantThreads;
   const cudaError_t e = per_thread <= 4 ? launch_ffn_c<4>(m, a, G, smem, s) : launch_ffn_c<12>(m, a, G, smem, s);
   return from_cuda(e);
+}
+
+bitnet_status bitnet_ste_backward_input(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K,
+                                        const void* dY, int64_t M, void* dX, int dx_dtype, void* stream) {
+  if (W_packed == nullptr || gamma == nullptr || dY == nullptr || dX == nullptr) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(W_packed, 16) || !aligned(dY, 16) || !aligned(dX, 16) || !aligned(gamma, 4))
+    return BITNET_ERR_INVALID_ARG;
+  if (dx_dtype != BITNET_F32 && dx_dtype != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
+  if (!valid_k(K) || N < 8 || N % 8 != 0 || N > INT32_MAX || M < 1 || M > INT32_MAX)
+    return BITNET_ERR_UNSUPPORTED_SHAPE;
+  CUtensorMap mb, ma;
+  if (!make_map_bf16(&mb, dY, static_cast<uint64_t>(N), static_cast<uint64_t>(M), static_cast<uint64_t>(N) * 2,
+                     kSteBox, kSteBN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_u8(&ma, W_packed, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4),
+                   kSteBM / 4, kSteBJ, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return BITNET_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return from_cuda(launch_ste<0>(mb, ma, gamma, static_cast<int>(K), static_cast<int>(M), static_cast<int>(N), dX,
+                                 dx_dtype, s));
+}
+
+size_t bitnet_ste_weight_workspace_bytes(int64_t M, int64_t N) {
+  if (M < 1 || N < 1) return 0;
+  return static_cast<size_t>(N) * static_cast<size_t>(ste_padded_m(M)) * 2;
+}
+
+bitnet_status bitnet_ste_backward_weight(const void* dY, const int8_t* x_q, const float* a_scale, int64_t M,
+                                         int64_t N, int64_t K, void* dW, int dw_dtype, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  if (dY == nullptr || x_q == nullptr || a_scale == nullptr || dW == nullptr || workspace == nullptr)
+    return BITNET_ERR_INVALID_ARG;
+  if (!aligned(dY, 16) || !aligned(x_q, 16) || !aligned(dW, 16) || !aligned(workspace, 16) || !aligned(a_scale, 4))
+    return BITNET_ERR_INVALID_ARG;
+  if (dw_dtype != BITNET_F32 && dw_dtype != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
+  if (!valid_k(K) || N < 8 || N % 8 != 0 || N > INT32_MAX || M < 1 || M > INT32_MAX)
+    return BITNET_ERR_UNSUPPORTED_SHAPE;
+  if (workspace_bytes < bitnet_ste_weight_workspace_bytes(M, N)) return BITNET_ERR_INVALID_ARG;
+  const int64_t Mp = ste_padded_m(M);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  __nv_bfloat16* dyst = static_cast<__nv_bfloat16*>(workspace);
+  const dim3 pgrid(static_cast<unsigned>((N + 31) / 32), static_cast<unsigned>(Mp / 32));
+  cudaError_t e = launch_pdl(ste_scale_transpose_kernel, pgrid, dim3(256), 0, s,
+                             static_cast<const __nv_bfloat16*>(dY), a_scale, static_cast<int>(M), static_cast<int>(N),
+                             static_cast<int>(Mp), dyst);
+  if (e != cudaSuccess) return BITNET_ERR_CUDA;
+  CUtensorMap mb, ma;
+  if (!make_map_bf16(&mb, dyst, static_cast<uint64_t>(Mp), static_cast<uint64_t>(N), static_cast<uint64_t>(Mp) * 2,
+                     kSteBox, kSteBN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_u8(&ma, x_q, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(K), kSteBM,
+                   kSteBJ, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return BITNET_ERR_CUDA;
+  return from_cuda(launch_ste<1>(mb, ma, nullptr, static_cast<int>(K), static_cast<int>(N), static_cast<int>(Mp),
+                                 dW, dw_dtype, s));
 }
 
 bitnet_status bitnet_get_device_status(void* stream) {

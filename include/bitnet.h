@@ -230,6 +230,34 @@ bitnet_status bitnet_bitlinear_gemv_b3(const void* x, int x_dtype, const void* r
                                        const uint8_t* W_b3, const float* gamma, int64_t N, int64_t K, int64_t M,
                                        void* y, int y_dtype, void* stream);
 
+/*
+ * Backward pass of the BitLinear with the straight-through estimator.
+ * Training keeps precise latent weights and computes with the rounded ones,
+ * and the backward pass lets the gradient through the rounding as if it were
+ * absent (Habr repost on juhe.plus, sections "А откуда взялась сама идея?"
+ * and "Когда - три лучше двух").  The forward used W_hat = gamma * q and
+ * x_hat[m] = a_scale[m] * x_q[m]; both products run on the tensor cores
+ * (tcgen05 kind::f16: bf16 operands, fp32 accumulation).
+ *
+ * bitnet_ste_backward_input: dX[m][k] = RN32(gamma * sum_n dY[m][n] q[n][k])
+ *   up to the order of the fp32 accumulation.  W_packed, gamma, N, K as for
+ *   the forward (N x K/4 packed codes); dY: M x N bf16, row-major; dX: M x K
+ *   of dx_dtype (BITNET_F32 or BITNET_BF16).  N a multiple of 8.
+ * bitnet_ste_backward_weight: dW[n][k] = sum_m dYs[m][n] x_q[m][k] with
+ *   dYs = bf16_RNE(RN32(dY[m][n] * a_scale[m])) (the product's bf16 left
+ *   operand), up to the order of the fp32 accumulation.  dY: M x N bf16; x_q,
+ *   a_scale: the forward's quantised activations (M x K int8, M fp32); dW:
+ *   N x K of dw_dtype.  workspace: bitnet_ste_weight_workspace_bytes(M, N)
+ *   device bytes (dYs transposed, padded to a multiple of 64 tokens).
+ * Pointers 16-byte aligned (gamma, a_scale 4-byte).  Asynchronous.
+ */
+bitnet_status bitnet_ste_backward_input(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K,
+                                        const void* dY, int64_t M, void* dX, int dx_dtype, void* stream);
+size_t bitnet_ste_weight_workspace_bytes(int64_t M, int64_t N);
+bitnet_status bitnet_ste_backward_weight(const void* dY, const int8_t* x_q, const float* a_scale, int64_t M,
+                                         int64_t N, int64_t K, void* dW, int dw_dtype, void* workspace,
+                                         size_t workspace_bytes, void* stream);
+
 /* Bytes of the grid-barrier workspace that bitnet_bitlinear_ffn_gemv takes. */
 #define BITNET_FFN_SYNC_BYTES 64
 

@@ -163,6 +163,31 @@ def test_b3_rejects_bad_arguments(L):
     assert call(dt=bl.BITNET_F32, K=8192 + 64) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
 
 
+def test_ste_rejects_bad_arguments(L):
+    assert bl.bitnet_ste_weight_workspace_bytes(100, 16) == 16 * 128 * 2
+    assert bl.bitnet_ste_weight_workspace_bytes(0, 16) == 0
+
+    def dx(W=FAKE, g=FAKE, N=64, K=64, dY=FAKE, M=8, out=FAKE, od=bl.BITNET_F32):
+        return L.bitnet_ste_backward_input(W, g, N, K, dY, M, out, od, None)
+
+    assert dx(W=None) == bl.BITNET_ERR_INVALID_ARG
+    assert dx(dY=MIS) == bl.BITNET_ERR_INVALID_ARG
+    assert dx(od=bl.BITNET_I32) == bl.BITNET_ERR_INVALID_ARG
+    assert dx(N=60) == bl.BITNET_ERR_UNSUPPORTED_SHAPE   # dY rows must be 16-byte multiples
+    assert dx(K=96) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert dx(M=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+
+    def dw(dY=FAKE, xq=FAKE, a=FAKE, M=8, N=64, K=64, out=FAKE, od=bl.BITNET_F32, ws=FAKE, wsb=1 << 20):
+        return L.bitnet_ste_backward_weight(dY, xq, a, M, N, K, out, od, ws, wsb, None)
+
+    assert dw(a=None) == bl.BITNET_ERR_INVALID_ARG
+    assert dw(xq=MIS) == bl.BITNET_ERR_INVALID_ARG
+    assert dw(od=9) == bl.BITNET_ERR_INVALID_ARG
+    assert dw(wsb=16) == bl.BITNET_ERR_INVALID_ARG
+    assert dw(N=12) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert dw(K=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(bl, "_lib", None)
     monkeypatch.setattr(bl, "LIB_PATH", str(tmp_path / "missing.so"))
