@@ -598,13 +598,14 @@ def bench_ste(torch, bl, dev, stream, peaks, peak_src, group):
             xq, a, _ = bl.bitnet_quant_act(x, None, EPS_RMS)
             dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
             dW = torch.empty((N, K), dtype=torch.float32, device=dev)
-            ws = torch.empty(bl.bitnet_ste_weight_workspace_bytes(M, N), dtype=torch.uint8, device=dev)
+            ws = torch.empty(bl.bitnet_ste_weight_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
+            wsx = torch.empty(bl.bitnet_ste_input_workspace_bytes(N, K), dtype=torch.uint8, device=dev)
             tx, tw = [], []
             for it in range(13):
                 flush.zero_()
                 e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
                 e0.record(stream)
-                bl.bitnet_ste_backward_input(P, G, dY, dX=dX)
+                bl.bitnet_ste_backward_input(P, G, dY, dX=dX, workspace=wsx)
                 e1.record(stream)
                 flush.zero_()
                 e2.record(stream)
@@ -627,7 +628,8 @@ def bench_ste(torch, bl, dev, stream, peaks, peak_src, group):
             "roofline": {"bound": "tensor", "achieved": tf, "peak": bf16_peak, "unit": "TFLOP/s",
                          "frac": tf / bf16_peak, "peak_source": f"{peak_src} bf16_tflops"},
             "per_shape": out, "device_status": bl.bitnet_get_device_status(),
-            "timing": "median of 10 single launches, L2 flushed before each; dW includes its dY*a transpose pre-pass"}
+            "timing": "median of 10 single calls, L2 flushed before each; each call includes its operand "
+                      "expansion pre-passes (codes to bf16 for dX; dY*a and x_q transposed to bf16 for dW)"}
 
 
 def bench_ffn_block(torch, bl, dev, stream, peaks, peak_src, group, name="ffn_block_m1_2p5b"):

@@ -68,9 +68,11 @@ def lib() -> ctypes.CDLL:
         L.bitnet_pack_weights_b3.restype = I
         L.bitnet_bitlinear_gemv_b3.argtypes = [P, I, P, F, P, P, I64, I64, I64, P, I, P]
         L.bitnet_bitlinear_gemv_b3.restype = I
-        L.bitnet_ste_backward_input.argtypes = [P, P, I64, I64, P, I64, P, I, P]
+        L.bitnet_ste_input_workspace_bytes.argtypes = [I64, I64]
+        L.bitnet_ste_input_workspace_bytes.restype = ctypes.c_size_t
+        L.bitnet_ste_backward_input.argtypes = [P, P, I64, I64, P, I64, P, I, P, ctypes.c_size_t, P]
         L.bitnet_ste_backward_input.restype = I
-        L.bitnet_ste_weight_workspace_bytes.argtypes = [I64, I64]
+        L.bitnet_ste_weight_workspace_bytes.argtypes = [I64, I64, I64]
         L.bitnet_ste_weight_workspace_bytes.restype = ctypes.c_size_t
         L.bitnet_ste_backward_weight.argtypes = [P, P, P, I64, I64, I64, P, I, P, ctypes.c_size_t, P]
         L.bitnet_ste_backward_weight.restype = I
@@ -300,24 +302,31 @@ def bitnet_bitlinear_gemv_b3(x, W_b3, gamma, rms_gain=None, rms_eps: float = 1e-
     return y
 
 
-def bitnet_ste_backward_input(W_packed, gamma, dY, dX=None, out_dtype=None):
+def bitnet_ste_input_workspace_bytes(N: int, K: int) -> int:
+    return int(lib().bitnet_ste_input_workspace_bytes(N, K))
+
+
+def bitnet_ste_backward_input(W_packed, gamma, dY, dX=None, out_dtype=None, workspace=None):
     """STE input gradient dX = gamma * dY q (M x K), dY: M x N bf16."""
     torch = _torch()
-    _need_cuda(W_packed, gamma, dY, dX)
+    _need_cuda(W_packed, gamma, dY, dX, workspace)
     M, N = dY.shape
     K = W_packed.shape[1] * 4
     if W_packed.shape[0] != N:
         raise ValueError("dY and W_packed disagree on N")
     if dX is None:
         dX = torch.empty((M, K), dtype=out_dtype or torch.float32, device=dY.device)
+    if workspace is None:
+        workspace = torch.empty(bitnet_ste_input_workspace_bytes(N, K), dtype=torch.uint8, device=dY.device)
     st = lib().bitnet_ste_backward_input(_ptr(W_packed), _ptr(gamma), N, K, _ptr(dY), M, _ptr(dX),
-                                         _dtype_code(dX.dtype), _stream(dY.device))
+                                         _dtype_code(dX.dtype), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(dY.device))
     _check("bitnet_ste_backward_input", st)
     return dX
 
 
-def bitnet_ste_weight_workspace_bytes(M: int, N: int) -> int:
-    return int(lib().bitnet_ste_weight_workspace_bytes(M, N))
+def bitnet_ste_weight_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().bitnet_ste_weight_workspace_bytes(M, N, K))
 
 
 def bitnet_ste_backward_weight(dY, x_q, a_scale, dW=None, out_dtype=None, workspace=None):
@@ -330,9 +339,8 @@ def bitnet_ste_backward_weight(dY, x_q, a_scale, dW=None, out_dtype=None, worksp
         raise ValueError("dY and x_q disagree on M")
     if dW is None:
         dW = torch.empty((N, K), dtype=out_dtype or torch.float32, device=dY.device)
-    nbytes = bitnet_ste_weight_workspace_bytes(M, N)
     if workspace is None:
-        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dY.device)
+        workspace = torch.empty(bitnet_ste_weight_workspace_bytes(M, N, K), dtype=torch.uint8, device=dY.device)
     st = lib().bitnet_ste_backward_weight(_ptr(dY), _ptr(x_q), _ptr(a_scale), M, N, K, _ptr(dW),
                                           _dtype_code(dW.dtype), _ptr(workspace),
                                           workspace.numel() * workspace.element_size(), _stream(dY.device))

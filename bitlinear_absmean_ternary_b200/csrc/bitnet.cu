@@ -461,19 +461,22 @@ cudaError_t launch_b3(int M, const void* x, const void* gain, float eps, const u
 }
 
 // STE backward GEMMs (ste_gemm.cuh): persistent, one CTA per SM.
-template <int MODE>
-cudaError_t launch_ste(const CUtensorMap& mb, const CUtensorMap& ma, const float* scale, int R, int C, int J,
+constexpr int kSteBN = 256;
+constexpr int kSteStages = 2;
+
+cudaError_t launch_ste(const CUtensorMap& ma, const CUtensorMap& mb, const float* scale, int R, int C, int J,
                        void* out, int od, cudaStream_t s) {
+  using Cfg = SteCfg<kSteBN, kSteStages>;
   static bool done[kMaxDevices] = {};
-  const cudaError_t e = set_smem(ste_gemm_kernel<MODE>, SteCfg<MODE>::kSmemBytes, done);
+  auto kern = ste_gemm_kernel<kSteBN, kSteStages>;
+  const cudaError_t e = set_smem(kern, Cfg::kSmemBytes, done);
   if (e != cudaSuccess) return e;
   const int64_t tiles = static_cast<int64_t>((R + kSteBM - 1) / kSteBM) * ((C + kSteBN - 1) / kSteBN);
   const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-  return launch_pdl(ste_gemm_kernel<MODE>, dim3(grid), dim3(kGemmThreads), SteCfg<MODE>::kSmemBytes, s, mb, ma,
-                    scale, R, C, J, out, od);
+  return launch_pdl(kern, dim3(grid), dim3(kSteThreads), Cfg::kSmemBytes, s, ma, mb, scale, R, C, J, out, od);
 }
 
-int64_t ste_padded_m(int64_t M) { return (M + kSteBJ - 1) / kSteBJ * kSteBJ; }
+int64_t ste_pad(int64_t n) { return (n + kStePad - 1) / kStePad * kStePad; }
 
 bitnet_status check_linear(const uint8_t* Wp, const float* gamma, int64_t N, int64_t K, const int8_t* xq,
                            const float* a, const int32_t* rs, int64_t M, void* y, int yd) {
@@ -754,28 +757,43 @@ bitnet_status bitnet_bitlinear_ffn_gemv(const void* x, int x_dtype, int64_t M, i
   return from_cuda(e);
 }
 
+size_t bitnet_ste_input_workspace_bytes(int64_t N, int64_t K) {
+  if (N < 1 || !valid_k(K)) return 0;
+  return static_cast<size_t>(K) * static_cast<size_t>(ste_pad(N)) * 2;
+}
+
 bitnet_status bitnet_ste_backward_input(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K,
-                                        const void* dY, int64_t M, void* dX, int dx_dtype, void* stream) {
-  if (W_packed == nullptr || gamma == nullptr || dY == nullptr || dX == nullptr) return BITNET_ERR_INVALID_ARG;
-  if (!aligned(W_packed, 16) || !aligned(dY, 16) || !aligned(dX, 16) || !aligned(gamma, 4))
+                                        const void* dY, int64_t M, void* dX, int dx_dtype, void* workspace,
+                                        size_t workspace_bytes, void* stream) {
+  if (W_packed == nullptr || gamma == nullptr || dY == nullptr || dX == nullptr || workspace == nullptr)
+    return BITNET_ERR_INVALID_ARG;
+  if (!aligned(W_packed, 16) || !aligned(dY, 16) || !aligned(dX, 16) || !aligned(workspace, 16) ||
+      !aligned(gamma, 4))
     return BITNET_ERR_INVALID_ARG;
   if (dx_dtype != BITNET_F32 && dx_dtype != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
   if (!valid_k(K) || N < 8 || N % 8 != 0 || N > INT32_MAX || M < 1 || M > INT32_MAX)
     return BITNET_ERR_UNSUPPORTED_SHAPE;
-  CUtensorMap mb, ma;
-  if (!make_map_bf16(&mb, dY, static_cast<uint64_t>(N), static_cast<uint64_t>(M), static_cast<uint64_t>(N) * 2,
-                     kSteBox, kSteBN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_u8(&ma, W_packed, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4),
-                   kSteBM / 4, kSteBJ, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return BITNET_ERR_CUDA;
+  if (workspace_bytes < bitnet_ste_input_workspace_bytes(N, K)) return BITNET_ERR_INVALID_ARG;
+  const int64_t Np = ste_pad(N);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return from_cuda(launch_ste<0>(mb, ma, gamma, static_cast<int>(K), static_cast<int>(M), static_cast<int>(N), dX,
-                                 dx_dtype, s));
+  __nv_bfloat16* wt = static_cast<__nv_bfloat16*>(workspace);
+  const dim3 pgrid(static_cast<unsigned>(Np / 64), static_cast<unsigned>(K / 64));
+  if (launch_pdl(ste_expand_wt_kernel, pgrid, dim3(256), 0, s, W_packed, static_cast<int>(N), static_cast<int>(K),
+                 static_cast<int>(Np), wt) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  CUtensorMap ma, mb;
+  if (!make_map_bf16(&ma, wt, static_cast<uint64_t>(Np), static_cast<uint64_t>(K), static_cast<uint64_t>(Np) * 2,
+                     kSteBox, kSteBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_bf16(&mb, dY, static_cast<uint64_t>(N), static_cast<uint64_t>(M), static_cast<uint64_t>(N) * 2,
+                     kSteBox, kSteBN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return BITNET_ERR_CUDA;
+  return from_cuda(launch_ste(ma, mb, gamma, static_cast<int>(K), static_cast<int>(M), static_cast<int>(Np), dX,
+                              dx_dtype, s));
 }
 
-size_t bitnet_ste_weight_workspace_bytes(int64_t M, int64_t N) {
-  if (M < 1 || N < 1) return 0;
-  return static_cast<size_t>(N) * static_cast<size_t>(ste_padded_m(M)) * 2;
+size_t bitnet_ste_weight_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || N < 1 || !valid_k(K)) return 0;
+  return (static_cast<size_t>(N) + static_cast<size_t>(K)) * static_cast<size_t>(ste_pad(M)) * 2;
 }
 
 bitnet_status bitnet_ste_backward_weight(const void* dY, const int8_t* x_q, const float* a_scale, int64_t M,
@@ -788,23 +806,27 @@ bitnet_status bitnet_ste_backward_weight(const void* dY, const int8_t* x_q, cons
   if (dw_dtype != BITNET_F32 && dw_dtype != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
   if (!valid_k(K) || N < 8 || N % 8 != 0 || N > INT32_MAX || M < 1 || M > INT32_MAX)
     return BITNET_ERR_UNSUPPORTED_SHAPE;
-  if (workspace_bytes < bitnet_ste_weight_workspace_bytes(M, N)) return BITNET_ERR_INVALID_ARG;
-  const int64_t Mp = ste_padded_m(M);
+  if (workspace_bytes < bitnet_ste_weight_workspace_bytes(M, N, K)) return BITNET_ERR_INVALID_ARG;
+  const int64_t Mp = ste_pad(M);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  __nv_bfloat16* dyst = static_cast<__nv_bfloat16*>(workspace);
-  const dim3 pgrid(static_cast<unsigned>((N + 31) / 32), static_cast<unsigned>(Mp / 32));
-  cudaError_t e = launch_pdl(ste_scale_transpose_kernel, pgrid, dim3(256), 0, s,
-                             static_cast<const __nv_bfloat16*>(dY), a_scale, static_cast<int>(M), static_cast<int>(N),
-                             static_cast<int>(Mp), dyst);
-  if (e != cudaSuccess) return BITNET_ERR_CUDA;
-  CUtensorMap mb, ma;
-  if (!make_map_bf16(&mb, dyst, static_cast<uint64_t>(Mp), static_cast<uint64_t>(N), static_cast<uint64_t>(Mp) * 2,
-                     kSteBox, kSteBN, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map_u8(&ma, x_q, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(K), kSteBM,
-                   kSteBJ, CU_TENSOR_MAP_SWIZZLE_NONE))
+  __nv_bfloat16* dyst = static_cast<__nv_bfloat16*>(workspace);  // [N][Mp]
+  __nv_bfloat16* xt = dyst + N * Mp;                              // [K][Mp]
+  const dim3 g1(static_cast<unsigned>((N + 31) / 32), static_cast<unsigned>(Mp / 32));
+  if (launch_pdl(ste_scale_transpose_kernel, g1, dim3(256), 0, s, static_cast<const __nv_bfloat16*>(dY), a_scale,
+                 static_cast<int>(M), static_cast<int>(N), static_cast<int>(Mp), dyst) != cudaSuccess)
     return BITNET_ERR_CUDA;
-  return from_cuda(launch_ste<1>(mb, ma, nullptr, static_cast<int>(K), static_cast<int>(N), static_cast<int>(Mp),
-                                 dW, dw_dtype, s));
+  const dim3 g2(static_cast<unsigned>(Mp / 64), static_cast<unsigned>(K / 64));
+  if (launch_pdl(ste_expand_xt_kernel, g2, dim3(256), 0, s, x_q, static_cast<int>(M), static_cast<int>(K),
+                 static_cast<int>(Mp), xt) != cudaSuccess)
+    return BITNET_ERR_CUDA;
+  CUtensorMap ma, mb;
+  if (!make_map_bf16(&ma, xt, static_cast<uint64_t>(Mp), static_cast<uint64_t>(K), static_cast<uint64_t>(Mp) * 2,
+                     kSteBox, kSteBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_bf16(&mb, dyst, static_cast<uint64_t>(Mp), static_cast<uint64_t>(N), static_cast<uint64_t>(Mp) * 2,
+                     kSteBox, kSteBN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return BITNET_ERR_CUDA;
+  return from_cuda(launch_ste(ma, mb, nullptr, static_cast<int>(K), static_cast<int>(N), static_cast<int>(Mp), dW,
+                              dw_dtype, s));
 }
 
 bitnet_status bitnet_get_device_status(void* stream) {

@@ -10,23 +10,20 @@
 //   MODE 1 (weight gradient): dW[n, k] = sum_m dYs[m, n] x_q[m, k],
 //                             dYs = bf16(dY[m, n] * a[m]) (a pre-pass writes it transposed)
 //
-// Both are D[r, c] = sum_j A[r, j] B[c, j] with output rows r = k (a stage
-// carries 128 contraction elements, 8 MMAs, to amortise the stage handoff): a tile is
-// 128 values of k (the MMA's M, one TMEM lane each) by BN = 128 columns
-// (m for dX, n for dW), so that the epilogue's 32 lanes store 32 consecutive
-// k of one output row.
-//   A (128 x 128 per stage) is built in tensor memory by converter warps from
-//     a tile that TMA brings into shared memory with the contraction index j
-//     along its rows: MODE 0 packed weight rows n (32 bytes = 128 codes of k
-//     each; code -> bf16 -1/0/+1 through one byte permute per pair),
-//     MODE 1 int8 activation rows m (128 bytes of k; exact int8 -> bf16).
-//   B (BN x 128 per stage, two 64-wide boxes) is bf16, K-major (j
-//     contiguous), loaded by TMA in the 128-byte swizzled layout: MODE 0 dY as stored ([M][N]), MODE 1 the
-//     pre-pass output dYs^T ([N][M padded]).
-// Warp roles, barriers and bounded waits follow the int8 GEMM (gemm.cuh):
-// two TMA producer warps, an MMA warp that also allocates TMEM, eight
-// converter warps (two per TMEM lane quarter, alternate stages), four
-// epilogue warps; the accumulator is double-buffered in TMEM.
+// Both are D[r, c] = sum_j A[r, j] B[c, j] with output rows r = k, on a plain
+// bf16 GEMM whose operands both come from shared memory by TMA (128-byte
+// swizzled, K-major): expansion pre-passes first write the ternary codes
+// transposed as bf16 -1/0/+1 (MODE 0: WT[k][n]) or the int8 activations
+// transposed as exact bf16 (MODE 1: XT[k][m]), and dY * a transposed and
+// rounded to bf16 (MODE 1: dYs^T[n][m]).  Training GEMMs are bound by the
+// tensor pipe, so expanding each operand once beats re-expanding a weight
+// tile for every tile of tokens inside the GEMM (an in-GEMM expansion into
+// tensor memory kept the integer pipe 80% busy and the tensor pipe 30%).
+// Tile: 128 rows k (TMEM lanes) x BN columns (m for dX, n for dW), 128
+// contraction elements (8 MMAs) per stage; the epilogue's 32 lanes store 32
+// consecutive k of one output row.  Warps: two TMA producers (alternate
+// stages), one MMA issuer that also allocates TMEM, four epilogue warps; the
+// fp32 accumulator is double-buffered in TMEM; every wait is bounded.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -36,28 +33,28 @@
 
 namespace bitnet {
 
-constexpr int kSteBM = 128;   // output rows (k) per tile
-constexpr int kSteBN = 128;   // output columns per tile
-constexpr int kSteBJ = 128;   // contraction elements per stage (8 MMAs of K = 16)
-constexpr int kSteBox = 64;   // bf16 per 128-byte swizzled B box
-constexpr int kSteStages = 4;
+constexpr int kSteBM = 128;  // output rows (k) per tile
+constexpr int kSteBJ = 128;  // contraction elements per stage (8 MMAs of K = 16)
+constexpr int kSteBox = 64;  // bf16 per 128-byte swizzled box
+constexpr int kStePad = 64;  // contraction lengths of the expanded operands are padded to this
+constexpr int kSteEpiWarps = 4;
+constexpr int kSteThreads = (3 + kSteEpiWarps) * 32;  // producer, MMA, 4 epilogue, producer
 
-template <int MODE>
+// BN output columns per tile, S ring stages.  TMEM holds two accumulators of
+// BN fp32 columns.
+template <int BN, int S>
 struct SteCfg {
-  static constexpr int kBSub = kSteBN * 128;                      // one B box: bf16 [BN][64]
-  static constexpr int kBBytes = kBSub * (kSteBJ / kSteBox);
-  static constexpr int kARow = MODE == 0 ? kSteBM / 4 : kSteBM;   // source bytes per contraction row
-  static constexpr int kABytes = kSteBJ * kARow;                  // [BJ rows j][kARow]
-  static constexpr int kStageBytes = kBBytes + kABytes;
-  static constexpr int kAslot = kSteBJ / 2;  // TMEM columns per A slot (two bf16 per column)
-  static constexpr int kTmemCols = 512;
-  static constexpr int kAcol = 2 * kSteBN;   // two accumulator buffers first
-  static constexpr int kBarOffset = kSteStages * kStageBytes;
+  static constexpr int kASub = kSteBM * 128;                // one A box: bf16 [128][64]
+  static constexpr int kBSub = BN * 128;                    // one B box: bf16 [BN][64]
+  static constexpr int kBoxes = kSteBJ / kSteBox;           // boxes per operand per stage
+  static constexpr int kStageBytes = kBoxes * (kASub + kBSub);
+  static constexpr int kTmemCols = 2 * BN <= 256 ? 256 : 512;
+  static constexpr int kBarOffset = S * kStageBytes;
   static constexpr int kSmemBytes = 1024 + kBarOffset + 256;
   static_assert(kStageBytes % 1024 == 0, "stage tiles must stay 1024-byte aligned");
-  static_assert(kAcol + kSteStages * kAslot <= kTmemCols, "TMEM budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(kSteStages % kGemmProducers == 0, "each ring slot belongs to one producer");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+  static_assert(S % 2 == 0 || S == 3, "ring");
 };
 
 // Instruction descriptor for kind::f16 with bf16 A and B (both K-major) and
@@ -68,38 +65,37 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// D (tmem) [+]= A (tmem) x B (smem descriptor), kind::f16, fp32 accumulate.
-BN_DEV void mma_bf16_tmemA(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+// D (tmem) [+]= A (smem descriptor) x B (smem descriptor), kind::f16, fp32 accumulate.
+BN_DEV void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
-// R output rows (k), C output columns, J contraction length.  out is [C][R]
-// row-major (fp32 or bf16); scale_ptr: gamma (MODE 0) or null (scale 1).
-template <int MODE>
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    ste_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_a,
+// D[r][c] = sum_j A[r][j] B[c][j] for R output rows, C columns, contraction J;
+// A [R][J] and B [C][J] bf16 row-major (j contiguous) behind the tensor maps.
+// out is [C][R] row-major (fp32 or bf16), times *scale_ptr when given.
+template <int BN, int S>
+__global__ void __launch_bounds__(kSteThreads, 1)
+    ste_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                     const float* __restrict__ scale_ptr, int R, int C, int J, void* __restrict__ out, int out_dtype) {
-  using Cfg = SteCfg<MODE>;
-  constexpr int S = kSteStages;
+  using Cfg = SteCfg<BN, S>;
   constexpr int NB = 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::kBarOffset);
   uint64_t* empty = full + S;
-  uint64_t* afull = empty + S;
-  uint64_t* accfull = afull + S;
+  uint64_t* accfull = empty + S;
   uint64_t* accempty = accfull + 2;
   uint64_t* done = accempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int r_tiles = (R + kSteBM - 1) / kSteBM;
-  const int tiles = r_tiles * ((C + kSteBN - 1) / kSteBN);
+  const int tiles = r_tiles * ((C + BN - 1) / BN);
   const int nk = (J + kSteBJ - 1) / kSteBJ;
   const int cid = blockIdx.x, ncl = gridDim.x;
   const int my_tiles = cid < tiles ? (tiles - cid + ncl - 1) / ncl : 0;
@@ -109,16 +105,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
-      mbar_init(&afull[s], 4);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accfull[b], 1);
-      mbar_init(&accempty[b], kGemmEpiWarps);
+      mbar_init(&accempty[b], kSteEpiWarps);
     }
     mbar_init(done, 1);
     fence_barrier_init();
-    tma_prefetch_desc(&tmap_b);
     tma_prefetch_desc(&tmap_a);
+    tma_prefetch_desc(&tmap_b);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, Cfg::kTmemCols);
@@ -130,17 +125,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem = *tmem_holder;
   pdl_launch_dependents();
 
-  const int prod = warp == 0 ? 0 : warp - (1 + kGemmUnpackWarps + kGemmEpiWarps);
-  if (warp == 0 || warp >= 2 + kGemmUnpackWarps + kGemmEpiWarps) {
+  if (warp == 0 || warp == 2 + kSteEpiWarps) {
     if (lane == 0) {
-      // ------------------------------------------------------------ TMA producers
-      pdl_wait();  // dY and x_q come from earlier kernels
+      // ------------------------------------------------------------ TMA producers (stage g by producer g % 2)
+      const int prod = warp == 0 ? 0 : 1;
+      pdl_wait();  // the operands come from earlier kernels
       int issued = prod;
       bool ok = true;
-      for (int g = prod; g < total; g += kGemmProducers) {
+      for (int g = prod; g < total; g += 2) {
         const int s = g % S;
         const int t = cid + (g / nk) * ncl, kb = g % nk;
-        const int r0 = (t % r_tiles) * kSteBM, c0 = (t / r_tiles) * kSteBN;
+        const int r0 = (t % r_tiles) * kSteBM, c0 = (t / r_tiles) * BN;
         uint8_t* st = smem + s * Cfg::kStageBytes;
         if (g >= S && !mbar_wait(&empty[s], ((g / S) & 1) ^ 1)) {
           ok = false;
@@ -148,20 +143,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
 #pragma unroll
-        for (int i = 0; i < kSteBJ / kSteBox; ++i)
-          tma_load_2d(st + i * Cfg::kBSub, &tmap_b, kb * kSteBJ + i * kSteBox, c0, &full[s]);
-        tma_load_2d(st + Cfg::kBBytes, &tmap_a, MODE == 0 ? r0 / 4 : r0, kb * kSteBJ, &full[s]);
-        issued = g + kGemmProducers;
+        for (int i = 0; i < Cfg::kBoxes; ++i) {
+          tma_load_2d(st + i * Cfg::kASub, &tmap_a, kb * kSteBJ + i * kSteBox, r0, &full[s]);
+          tma_load_2d(st + Cfg::kBoxes * Cfg::kASub + i * Cfg::kBSub, &tmap_b, kb * kSteBJ + i * kSteBox, c0,
+                      &full[s]);
+        }
+        issued = g + 2;
       }
       if (!ok) {
-        for (int g = prod; g < issued; g += kGemmProducers)
+        for (int g = prod; g < issued; g += 2)
           if (g + S >= issued) mbar_wait(&full[g % S], (g / S) & 1);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = idesc_bf16(kSteBM, kSteBN);
+      constexpr uint32_t idesc = idesc_bf16(kSteBM, BN);
       bool ok = true;
       int g = 0, tc = 0;
       for (int t = cid; ok && t < tiles; t += ncl, ++tc) {
@@ -171,21 +168,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t dcol = tmem + b * kSteBN;
+        const uint32_t dcol = tmem + b * BN;
         for (int kb = 0; kb < nk; ++kb, ++g) {
           const int s = g % S;
-          const uint32_t ph = (g / S) & 1;
-          if (!mbar_wait(&full[s], ph) || !mbar_wait(&afull[s], ph)) {
+          if (!mbar_wait(&full[s], (g / S) & 1)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t baddr = smem_addr(smem + s * Cfg::kStageBytes);
+          const uint32_t abase = smem_addr(smem + s * Cfg::kStageBytes);
+          const uint32_t bbase = abase + Cfg::kBoxes * Cfg::kASub;
 #pragma unroll
           for (int kk = 0; kk < kSteBJ / 16; ++kk)
-            mma_bf16_tmemA(dcol, tmem + Cfg::kAcol + Cfg::kAslot * s + 8 * kk,
-                           smem_desc_k_sw128(baddr + (kk >> 2) * Cfg::kBSub + 32 * (kk & 3)), idesc,
-                           (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16_ss(dcol, smem_desc_k_sw128(abase + (kk >> 2) * Cfg::kASub + 32 * (kk & 3)),
+                        smem_desc_k_sw128(bbase + (kk >> 2) * Cfg::kBSub + 32 * (kk & 3)), idesc,
+                        (kb > 0 || kk > 0) ? 1u : 0u);
           tc_commit(&empty[s]);
         }
         if (ok) tc_commit(&accfull[b]);
@@ -193,56 +190,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_commit(done);
       mbar_wait(done, 0);
     }
-  } else if (warp < kGemmFirstEpiWarp) {
-    // ------------------------------------------------------------ converters
-    const int q = warp & 3;
-    const int par = (warp - 2) >> 2;  // stages with g % 2 == par
-    const int r = 32 * q + lane;      // output row (k - r0) of this thread = its TMEM lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
-    // MODE 0: weight k0 + r sits in 32-bit word r / 16 of a 32-byte packed row, at bit 8 (r % 4) + 2 ((r / 4) % 4)
-    const uint32_t woff = MODE == 0 ? static_cast<uint32_t>(r >> 4) * 4u : static_cast<uint32_t>(r & ~3);
-    const uint32_t sh = MODE == 0 ? 8u * (r & 3) + 2u * ((r >> 2) & 3) : 8u * (r & 3);
-    for (int g = par; g < total; g += 2) {
-      const int s = g % S;
-      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (g / S) & 1))) break;
-      const uint32_t src = smem_addr(smem + s * Cfg::kStageBytes + Cfg::kBBytes) + woff;
-#pragma unroll
-      for (int h = 0; h < kSteBJ / 64; ++h) {  // 64 contraction elements -> 32 TMEM columns per pass
-        uint32_t v[32];
-#pragma unroll
-        for (int p = 0; p < 32; ++p) {
-          const int j = 64 * h + 2 * p;
-          uint32_t w0, w1;
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w0) : "r"(src + j * Cfg::kARow));
-          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w1) : "r"(src + (j + 1) * Cfg::kARow));
-          if constexpr (MODE == 0) {
-            // codes c in {0,1,2} -> bf16 of q = c - 1: bytes (0x80,0xBF), (0,0), (0x80,0x3F) at pool
-            // positions (2c, 2c+1) of {0x0000BF80, 0x00003F80}
-            uint32_t c0, c1;
-            asm("bfe.u32 %0, %1, %2, 2;" : "=r"(c0) : "r"(w0), "r"(sh));
-            asm("bfe.u32 %0, %1, %2, 2;" : "=r"(c1) : "r"(w1), "r"(sh));
-            v[p] = __byte_perm(0x0000BF80u, 0x00003F80u, 0x1010u + 0x22u * c0 + 0x2200u * c1);
-          } else {
-            // signed byte -> float exactly: the bits of 1.5 * 2^23 plus x are the float 1.5 * 2^23 + x
-            // (unit spacing in [2^23, 2^24)), minus 1.5 * 2^23; |x| <= 127 leaves the low 16 bits of the
-            // float zero, so its high half is the bf16 value
-            int x0, x1;
-            asm("bfe.s32 %0, %1, %2, 8;" : "=r"(x0) : "r"(w0), "r"(sh));
-            asm("bfe.s32 %0, %1, %2, 8;" : "=r"(x1) : "r"(w1), "r"(sh));
-            const float f0 = __fsub_rn(__int_as_float(0x4B400000 + x0), 12582912.0f);
-            const float f1 = __fsub_rn(__int_as_float(0x4B400000 + x1), 12582912.0f);
-            v[p] = __byte_perm(__float_as_uint(f0), __float_as_uint(f1), 0x7632);
-          }
-        }
-        tmem_st_32x32b_x32(lane_base + Cfg::kAcol + Cfg::kAslot * s + 32 * h, v);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&afull[s]);
-    }
   } else {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (warps 2 .. 5)
     const int q = warp & 3;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
     const float scale = scale_ptr != nullptr ? __ldg(scale_ptr) : 1.0f;
@@ -252,11 +201,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(&accfull[b], (tc / NB) & 1))) break;
       tc_fence_after();
       const int k = (t % r_tiles) * kSteBM + 32 * q + lane;
-      const int c0 = (t / r_tiles) * kSteBN;
+      const int c0 = (t / r_tiles) * BN;
 #pragma unroll 1
-      for (int cc = 0; cc < kSteBN; cc += 32) {
+      for (int cc = 0; cc < BN; cc += 32) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(lane_base + b * kSteBN + cc, v);
+        tmem_ld_32x32b_x32(lane_base + b * BN + cc, v);
         tmem_ld_wait();
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
@@ -282,6 +231,51 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, Cfg::kTmemCols);
   }
+}
+
+// Expansion of the ternary codes for the input gradient: WT[k][n] = q[n][k]
+// as bf16 (-1, 0, +1) for n < N, 0 for N <= n < Np.  One 64 x 64 tile per
+// CTA through shared memory: packed words of 16 codes read along k, bf16
+// rows written along n.
+__global__ void __launch_bounds__(256) ste_expand_wt_kernel(const uint8_t* __restrict__ Wp, int N, int K, int Np,
+                                                            __nv_bfloat16* __restrict__ wt) {
+  __shared__ int8_t tile[64][65];  // [n][k]
+  pdl_wait();
+  const int n0 = blockIdx.x * 64, k0 = blockIdx.y * 64;
+  {
+    const int n = threadIdx.x >> 2, w = threadIdx.x & 3;  // 64 rows x 4 words of 16 codes
+    uint32_t word = 0x55555555u;  // code 1 (q = 0) in every field: padding rows
+    if (n0 + n < N && k0 + 16 * w < K)
+      word = __ldg(reinterpret_cast<const uint32_t*>(Wp + static_cast<int64_t>(n0 + n) * (K / 4) + k0 / 4) + w);
+#pragma unroll
+    for (int e = 0; e < 16; ++e)  // weight 16w + e: byte e % 4, bits 2 (e / 4)
+      tile[n][16 * w + e] = static_cast<int8_t>(((word >> (8 * (e & 3) + 2 * (e >> 2))) & 3u) - 1);
+  }
+  __syncthreads();
+  pdl_launch_dependents();
+  const int nn = threadIdx.x & 63, kr = threadIdx.x >> 6;  // 64 n x 4 rows of k per pass
+  for (int k = kr; k < 64; k += 4)
+    if (k0 + k < K && n0 + nn < Np)
+      wt[static_cast<int64_t>(k0 + k) * Np + n0 + nn] = __float2bfloat16_rn(static_cast<float>(tile[nn][k]));
+}
+
+// Expansion of the activations for the weight gradient: XT[k][m] = x_q[m][k]
+// as bf16 (exact) for m < M, 0 for M <= m < Mp.
+__global__ void __launch_bounds__(256) ste_expand_xt_kernel(const int8_t* __restrict__ xq, int M, int K, int Mp,
+                                                            __nv_bfloat16* __restrict__ xt) {
+  __shared__ int8_t tile[64][65];  // [m][k]
+  pdl_wait();
+  const int m0 = blockIdx.x * 64, k0 = blockIdx.y * 64;
+  for (int i = threadIdx.x; i < 64 * 64; i += 256) {
+    const int m = i >> 6, k = i & 63;
+    tile[m][k] = (m0 + m < M && k0 + k < K) ? xq[static_cast<int64_t>(m0 + m) * K + k0 + k] : int8_t{0};
+  }
+  __syncthreads();
+  pdl_launch_dependents();
+  const int mm = threadIdx.x & 63, kr = threadIdx.x >> 6;
+  for (int k = kr; k < 64; k += 4)
+    if (k0 + k < K && m0 + mm < Mp)
+      xt[static_cast<int64_t>(k0 + k) * Mp + m0 + mm] = __float2bfloat16_rn(static_cast<float>(tile[mm][k]));
 }
 
 // Pre-pass of the weight gradient: dYsT[n][m] = bf16_RNE(RN32(dY[m][n] * a[m]))

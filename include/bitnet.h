@@ -237,23 +237,27 @@ bitnet_status bitnet_bitlinear_gemv_b3(const void* x, int x_dtype, const void* r
  * absent (Habr repost on juhe.plus, sections "А откуда взялась сама идея?"
  * and "Когда - три лучше двух").  The forward used W_hat = gamma * q and
  * x_hat[m] = a_scale[m] * x_q[m]; both products run on the tensor cores
- * (tcgen05 kind::f16: bf16 operands, fp32 accumulation).
+ * (tcgen05 kind::f16: bf16 operands, fp32 accumulation) after short
+ * pre-passes that write the operands as bf16 into the caller's workspace.
  *
  * bitnet_ste_backward_input: dX[m][k] = RN32(gamma * sum_n dY[m][n] q[n][k])
  *   up to the order of the fp32 accumulation.  W_packed, gamma, N, K as for
  *   the forward (N x K/4 packed codes); dY: M x N bf16, row-major; dX: M x K
- *   of dx_dtype (BITNET_F32 or BITNET_BF16).  N a multiple of 8.
+ *   of dx_dtype (BITNET_F32 or BITNET_BF16).  N a multiple of 8.  workspace:
+ *   bitnet_ste_input_workspace_bytes(N, K) device bytes (q transposed as bf16).
  * bitnet_ste_backward_weight: dW[n][k] = sum_m dYs[m][n] x_q[m][k] with
  *   dYs = bf16_RNE(RN32(dY[m][n] * a_scale[m])) (the product's bf16 left
  *   operand), up to the order of the fp32 accumulation.  dY: M x N bf16; x_q,
  *   a_scale: the forward's quantised activations (M x K int8, M fp32); dW:
- *   N x K of dw_dtype.  workspace: bitnet_ste_weight_workspace_bytes(M, N)
- *   device bytes (dYs transposed, padded to a multiple of 64 tokens).
+ *   N x K of dw_dtype.  workspace: bitnet_ste_weight_workspace_bytes(M, N, K)
+ *   device bytes (dYs and x_q transposed as bf16, tokens padded to 64).
  * Pointers 16-byte aligned (gamma, a_scale 4-byte).  Asynchronous.
  */
+size_t bitnet_ste_input_workspace_bytes(int64_t N, int64_t K);
 bitnet_status bitnet_ste_backward_input(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K,
-                                        const void* dY, int64_t M, void* dX, int dx_dtype, void* stream);
-size_t bitnet_ste_weight_workspace_bytes(int64_t M, int64_t N);
+                                        const void* dY, int64_t M, void* dX, int dx_dtype, void* workspace,
+                                        size_t workspace_bytes, void* stream);
+size_t bitnet_ste_weight_workspace_bytes(int64_t M, int64_t N, int64_t K);
 bitnet_status bitnet_ste_backward_weight(const void* dY, const int8_t* x_q, const float* a_scale, int64_t M,
                                          int64_t N, int64_t K, void* dW, int dw_dtype, void* workspace,
                                          size_t workspace_bytes, void* stream);

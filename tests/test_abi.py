@@ -164,15 +164,19 @@ def test_b3_rejects_bad_arguments(L):
 
 
 def test_ste_rejects_bad_arguments(L):
-    assert bl.bitnet_ste_weight_workspace_bytes(100, 16) == 16 * 128 * 2
-    assert bl.bitnet_ste_weight_workspace_bytes(0, 16) == 0
+    assert bl.bitnet_ste_weight_workspace_bytes(100, 16, 64) == (16 + 64) * 128 * 2
+    assert bl.bitnet_ste_weight_workspace_bytes(0, 16, 64) == 0
+    assert bl.bitnet_ste_input_workspace_bytes(100, 64) == 64 * 128 * 2
+    assert bl.bitnet_ste_input_workspace_bytes(100, 96) == 0
 
-    def dx(W=FAKE, g=FAKE, N=64, K=64, dY=FAKE, M=8, out=FAKE, od=bl.BITNET_F32):
-        return L.bitnet_ste_backward_input(W, g, N, K, dY, M, out, od, None)
+    def dx(W=FAKE, g=FAKE, N=64, K=64, dY=FAKE, M=8, out=FAKE, od=bl.BITNET_F32, ws=FAKE, wsb=1 << 20):
+        return L.bitnet_ste_backward_input(W, g, N, K, dY, M, out, od, ws, wsb, None)
 
     assert dx(W=None) == bl.BITNET_ERR_INVALID_ARG
+    assert dx(ws=None) == bl.BITNET_ERR_INVALID_ARG
     assert dx(dY=MIS) == bl.BITNET_ERR_INVALID_ARG
     assert dx(od=bl.BITNET_I32) == bl.BITNET_ERR_INVALID_ARG
+    assert dx(wsb=64) == bl.BITNET_ERR_INVALID_ARG
     assert dx(N=60) == bl.BITNET_ERR_UNSUPPORTED_SHAPE   # dY rows must be 16-byte multiples
     assert dx(K=96) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
     assert dx(M=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE

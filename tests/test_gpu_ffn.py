@@ -140,3 +140,29 @@ def test_ffn_shared_sync_words_repeat_and_graph_capture(dev, orc):
     G = torch.cuda.get_device_properties(dev).multi_processor_count
     assert count == 13 * G  # 1 + 4 eager launches and 2 replays of 4, one barrier of G arrivals each
     assert bl.bitnet_get_device_status() == bl.BITNET_OK
+
+
+def test_ffn_barrier_timeout_is_reported_and_context_survives(dev, orc):
+    """Failure detection without a fault: start the barrier's arrival counter at
+    1 instead of 0.  The CTA that arrives last then computes a target one
+    barrier further on that no arrival will reach, gives up after the bounded
+    wait (about 2 s), flags the device error word and returns; the host reads
+    BITNET_ERR_TIMEOUT and the context stays usable: after re-zeroing the
+    counter the next call is correct again."""
+    import torch
+    M, D, F = 1, 256, 512
+    x, gi, gs, dv, ref = _make(orc, dev, M, D, F, True, True, seed=21)
+    h_r, _, y_r = orc.ffn(x, ref["up"], ref["gate"], ref["down"], gi, EPS_RMS, gs, EPS_RMS)
+    args = (_bf16_dev(x, dev), *dv["up"], *dv["gate"], *dv["down"], _bf16_dev(gi, dev), EPS_RMS,
+            _bf16_dev(gs, dev), EPS_RMS)
+    assert bl.bitnet_get_device_status() == bl.BITNET_OK
+    sync = torch.zeros(bl.BITNET_FFN_SYNC_BYTES, dtype=torch.uint8, device=dev)
+    sync[0] = 1  # arrival counter = 1: not a multiple of the CTA count
+    bl.bitnet_bitlinear_ffn_gemv(*args, sync=sync, out_dtype=torch.float32)
+    assert bl.bitnet_get_device_status() == bl.BITNET_ERR_TIMEOUT
+    assert bl.bitnet_get_device_status() == bl.BITNET_OK  # the status was read and cleared
+    sync.zero_()
+    h, y = bl.bitnet_bitlinear_ffn_gemv(*args, sync=sync, out_dtype=torch.float32)
+    assert bl.bitnet_get_device_status() == bl.BITNET_OK
+    np.testing.assert_array_equal(_bits(h), h_r)
+    np.testing.assert_array_equal(y.cpu().numpy().view(np.uint32), y_r.view(np.uint32))
