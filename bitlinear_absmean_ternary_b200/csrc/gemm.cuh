@@ -57,7 +57,7 @@ namespace bitnet {
 constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 256;  // K bytes per stage = 8 MMAs of K = 32
 constexpr int kGemmUnpackWarps = 8;
-constexpr int kGemmEpiWarps = 4;
+constexpr int kGemmEpiWarps = 8;  // two per TMEM lane quarter, each draining half of the columns
 // TMA issue warps: one issuing thread streams a stage roughly every 270 ns
 // whatever its size, so two warps share the ring (warp p issues the stages g
 // with g % kGemmProducers == p).
@@ -276,7 +276,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
     pdl_wait();  // a_scale and rowsum come from the previous kernel
     const float gamma = __ldg(gamma_ptr);
-    constexpr int CW = BN < 32 ? BN : 32;
+    constexpr int EH = BN >= 64 ? 2 : 1;      // column halves per tile (one per warp of a quarter)
+    constexpr int CW = BN / EH < 32 ? BN / EH : 32;
+    const int half = (warp - kGemmFirstEpiWarp) >> 2;
+    const int col_lo = half * (BN / EH), col_hi = half < EH ? (half + 1) * (BN / EH) : col_lo;
     int tc = 0;
     for (int t = cid; t < tiles; t += ncl, ++tc) {
       const int b = tc % NB;
@@ -289,7 +292,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int r = 32 * q + lane;  // accumulator row (TMEM lane) this thread drains
         if (tc > 0 && !__all_sync(0xffffffffu, mbar_wait_cluster(consumed, (tc - 1) & 1))) break;
 #pragma unroll 1
-        for (int cc = 0; cc < BN; cc += CW) {
+        for (int cc = col_lo; cc < col_hi; cc += CW) {
           uint32_t v[CW];
           if constexpr (CW == 32) {
             tmem_ld_32x32b_x32(lane_base + b * BN + cc, v);
@@ -353,7 +356,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // ---- one CTA per tile: dequantise straight from TMEM
         const int n = n0 + 32 * q + lane;
 #pragma unroll 1
-        for (int cc = 0; cc < BN; cc += CW) {
+        for (int cc = col_lo; cc < col_hi; cc += CW) {
           uint32_t v[CW];
           if constexpr (CW == 32) {
             tmem_ld_32x32b_x32(lane_base + b * BN + cc, v);
