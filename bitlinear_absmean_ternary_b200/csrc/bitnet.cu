@@ -462,7 +462,7 @@ cudaError_t launch_b3(int M, const void* x, const void* gain, float eps, const u
 
 // STE backward GEMMs (ste_gemm.cuh): persistent, one CTA per SM.
 constexpr int kSteBN = 256;
-constexpr int kSteStages = 2;
+constexpr int kSteStages = 4;
 
 cudaError_t launch_ste(const CUtensorMap& ma, const CUtensorMap& mb, const float* scale, int R, int C, int J,
                        void* out, int od, cudaStream_t s) {

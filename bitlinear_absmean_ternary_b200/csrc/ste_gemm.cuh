@@ -19,9 +19,10 @@
 // tensor pipe, so expanding each operand once beats re-expanding a weight
 // tile for every tile of tokens inside the GEMM (an in-GEMM expansion into
 // tensor memory kept the integer pipe 80% busy and the tensor pipe 30%).
-// Tile: 128 rows k (TMEM lanes) x BN columns (m for dX, n for dW), 128
-// contraction elements (8 MMAs) per stage; the epilogue's 32 lanes store 32
-// consecutive k of one output row.  Warps: two TMA producers (alternate
+// Tile: 128 rows k (TMEM lanes) x BN columns (m for dX, n for dW), 64
+// contraction elements (4 MMAs) per stage in a ring of four (deeper rings of
+// smaller stages fed the MMAs better than two stages of 128); the epilogue's
+// 32 lanes store 32 consecutive k of one output row.  Warps: two TMA producers (alternate
 // stages), one MMA issuer that also allocates TMEM, four epilogue warps; the
 // fp32 accumulator is double-buffered in TMEM; every wait is bounded.
 #pragma once
@@ -34,7 +35,7 @@
 namespace bitnet {
 
 constexpr int kSteBM = 128;  // output rows (k) per tile
-constexpr int kSteBJ = 128;  // contraction elements per stage (8 MMAs of K = 16)
+constexpr int kSteBJ = 64;   // contraction elements per stage (4 MMAs of K = 16)
 constexpr int kSteBox = 64;  // bf16 per 128-byte swizzled box
 constexpr int kStePad = 64;  // contraction lengths of the expanded operands are padded to this
 constexpr int kSteEpiWarps = 4;
