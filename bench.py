@@ -220,6 +220,20 @@ def oracle_step_sample(lins, time_budget_s: float):
     return (lambda: run(frac)), bytes_for(frac), desc, frac
 
 
+def host_info() -> dict:
+    """CPU model and logical core count of the host the oracle runs on."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count()}
+
+
 def run_reference(args, lins, rank: int):
     if rank != 0:
         return
@@ -237,7 +251,8 @@ def run_reference(args, lins, rank: int):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
         "config": {"workload": args.workload, "linears": [[l.M, l.K, l.N] for l in lins], "parallelism": "replicas"},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc,
+                         "host": host_info()},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -365,16 +380,26 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
         barrier(group, dev)
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        # an event after every graph of G steps: per-step percentiles over the replays
+        marks = [torch.cuda.Event(enable_timing=True) for _ in range(full)]
         with torch.cuda.stream(stream):
             e0.record(stream)
-            for _ in range(full):
+            for r in range(full):
                 g_main.replay()
+                marks[r].record(stream)
             if g_rem is not None:
                 g_rem.replay()
             e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier(group, dev)
     el_ms = max_over_ranks(e0.elapsed_time(e1), group, dev)
+    per_step_us = [(a.elapsed_time(b) if a is not None else e0.elapsed_time(b)) * 1e3 / G
+                   for a, b in zip([None] + marks[:-1], marks)]
+    step_stats = None
+    if len(per_step_us) >= 2:
+        qs = np.percentile(per_step_us, [10, 50, 90])
+        step_stats = {"p10_us": float(qs[0]), "p50_us": float(qs[1]), "p90_us": float(qs[2]),
+                      "samples": len(per_step_us), "per": f"graph replay of {G} steps"}
     step_bytes = sum(linear_bytes(l)["quant"] + linear_bytes(l)["product"] for l in lins)
     value = ws * K * step_bytes / (el_ms / 1e3) / 1e9
 
@@ -496,13 +521,14 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
             n += 1
         el = time.perf_counter() - t0
         cpu = {"value": nbytes * n / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": f"{n} steps, each {desc}; {el:.1f} s"}
+               "sample": f"{n} steps, each {desc}; {el:.1f} s", "host": host_info()}
 
     if rank == 0:
         clk = clocks.summary()
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": K, "warmup": args.warmup,
-            "ms_per_step": el_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "ms_per_step": el_ms / K, "step_percentiles": step_stats, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None,
             "dtype": "int8", "data": "synthetic",
             "config": {"workload": args.workload, "linears": [[l.M, l.K, l.N] for l in lins],
                        "step": ("per linear: one bitnet_bitlinear_gemv kernel (RMSNorm/absmax int8 quantisation of "
