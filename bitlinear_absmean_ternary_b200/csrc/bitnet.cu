@@ -130,13 +130,13 @@ bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t r
 
 // ------------------------------------------------------------ launchers
 
-template <typename T, int MAXC>
+template <typename T, int MAXC, int NTHR = kQuantThreads>
 cudaError_t launch_quant_t(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
-                           int32_t* rs, cudaStream_t s) {
+                           int32_t* rs, cudaStream_t s, int threads = kQuantThreads) {
   static bool done[kMaxDevices] = {};
-  const cudaError_t e = set_smem(quant_act_kernel<T, MAXC>, 0, done);
+  const cudaError_t e = set_smem(quant_act_kernel<T, MAXC, NTHR>, 0, done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(quant_act_kernel<T, MAXC>, dim3(static_cast<unsigned>(M)), dim3(kQuantThreads), 0, s,
+  return launch_pdl(quant_act_kernel<T, MAXC, NTHR>, dim3(static_cast<unsigned>(M)), dim3(threads), 0, s,
                     static_cast<const T*>(x), K, static_cast<const T*>(gain), eps, xq, a, rs);
 }
 
@@ -144,6 +144,18 @@ template <typename T>
 cudaError_t launch_quant(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
                          int32_t* rs, cudaStream_t s) {
   const int per_thread = (K / 8 + kQuantThreads - 1) / kQuantThreads;
+  if (gain == nullptr) {
+    // No norm, so no fixed order: the fewest whole warps (at most 256 threads)
+    // that give every thread the same number of 8-element chunks.
+    const int mc = per_thread <= 1 ? 1 : per_thread <= 2 ? 2 : per_thread <= 4 ? 4 : per_thread <= 8 ? 8 : 16;
+    const int threads = ((K / 8 + mc - 1) / mc + 31) / 32 * 32;
+    if (mc == 1) return launch_quant_t<T, 1>(x, M, K, gain, eps, xq, a, rs, s, threads);
+    if (mc == 2) return launch_quant_t<T, 2>(x, M, K, gain, eps, xq, a, rs, s, threads);
+    if (mc == 4) return launch_quant_t<T, 4>(x, M, K, gain, eps, xq, a, rs, s, threads);
+    if (mc == 8) return launch_quant_t<T, 8>(x, M, K, gain, eps, xq, a, rs, s, threads);
+    if constexpr (sizeof(T) == 2) return launch_quant_t<T, 16>(x, M, K, gain, eps, xq, a, rs, s, threads);
+    return cudaErrorInvalidValue;
+  }
   if (per_thread <= 1) return launch_quant_t<T, 1>(x, M, K, gain, eps, xq, a, rs, s);
   if (per_thread <= 2) return launch_quant_t<T, 2>(x, M, K, gain, eps, xq, a, rs, s);
   if (per_thread <= 4) return launch_quant_t<T, 4>(x, M, K, gain, eps, xq, a, rs, s);

@@ -79,6 +79,13 @@ BN_DEV uint32_t pack4_s8(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
 
 BN_DEV void prefetch_l1(const void* p) { asm volatile("prefetch.global.L1 [%0];" ::"l"(p)); }
 
+// Unsigned 16-bit maximum of both halves.
+BN_DEV uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // Barrier over the first NT threads of the CTA (named barrier 1), or over
 // the whole CTA when NT == 0.
 template <int NT>
@@ -178,8 +185,28 @@ BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict_
 
   // h = RN32(RN32(v * r) * g) or v; amax = max |h| (order-free).
   float amax = 0.0f;
+  if constexpr (sizeof(T) == 2) {
+    if (gain == nullptr) {
+      // bf16 without a norm: |v| orders like the bit pattern with the sign
+      // cleared, so two values take one 16-bit integer max.
+      uint32_t m2 = 0;
 #pragma unroll
-  for (int i = 0; i < MAXC; ++i) {
+      for (int i = 0; i < MAXC; ++i) {
+        const int c = t + nt * i;
+        if (c < nchunks) {
+          const uint4 u = reinterpret_cast<const uint4&>(ch[i]);
+          m2 = max_u16x2(m2, u.x & 0x7FFF7FFFu);
+          m2 = max_u16x2(m2, u.y & 0x7FFF7FFFu);
+          m2 = max_u16x2(m2, u.z & 0x7FFF7FFFu);
+          m2 = max_u16x2(m2, u.w & 0x7FFF7FFFu);
+        }
+      }
+      const uint32_t mb = (m2 & 0xFFFFu) > (m2 >> 16) ? (m2 & 0xFFFFu) : (m2 >> 16);
+      amax = __uint_as_float(mb << 16);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < MAXC && !(sizeof(T) == 2 && gain == nullptr); ++i) {
     const int c = t + nt * i;
     if (c < nchunks) {
       Chunk8<T> g;
@@ -236,9 +263,12 @@ BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict_
   sum_out = tot;
 }
 
-// Standalone kernel: one CTA per token row.
-template <typename T, int MAXC>
-__global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(const T* __restrict__ x, int K,
+// Standalone kernel: one CTA per token row.  256 threads with RMSNorm (the
+// fixed summation order is defined on 256 lanes); without it the launcher
+// takes the fewest whole warps that give every thread the same number of
+// chunks (160 threads x 2 chunks for K = 2560, 224 x 4 for K = 6912).
+template <typename T, int MAXC, int NTHR = kQuantThreads>
+__global__ void __launch_bounds__(NTHR) quant_act_kernel(const T* __restrict__ x, int K,
                                                                   const T* __restrict__ gain, float rms_eps,
                                                                   int8_t* __restrict__ xq, float* __restrict__ a_out,
                                                                   int32_t* __restrict__ rowsum_out) {
