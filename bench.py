@@ -276,7 +276,10 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
     peaks, peak_src = load_peaks()
     stream = torch.cuda.Stream(dev)
 
-    # ---- inputs and offline weight packing (timed once, reported under "stages")
+    # ---- inputs and offline weight packing (timed once, reported under "stages"); one
+    # untimed pack first so that the library's first-call setup is not in the figure
+    bl.bitnet_pack_weights(torch.ones((64, 64), dtype=torch.float32, device=dev), EPS_W)
+    torch.cuda.synchronize(dev)
     packs, xs, gains, bufs = [], [], [], []
     pack_ms = []
     for lin in lins:
