@@ -38,8 +38,8 @@ constexpr int kSteBM = 128;  // output rows (k) per tile
 constexpr int kSteBJ = 64;   // contraction elements per stage (4 MMAs of K = 16)
 constexpr int kSteBox = 64;  // bf16 per 128-byte swizzled box
 constexpr int kStePad = 64;  // contraction lengths of the expanded operands are padded to this
-constexpr int kSteEpiWarps = 4;
-constexpr int kSteThreads = (3 + kSteEpiWarps) * 32;  // producer, MMA, 4 epilogue, producer
+constexpr int kSteEpiWarps = 8;  // two per TMEM lane quarter, half of a tile's columns each
+constexpr int kSteThreads = (3 + kSteEpiWarps) * 32;  // producer, MMA, epilogue warps, producer
 
 // BN output columns per tile, S ring stages.  TMEM holds two accumulators of
 // BN fp32 columns.
@@ -54,7 +54,7 @@ struct SteCfg {
   static constexpr int kSmemBytes = 1024 + kBarOffset + 256;
   static_assert(kStageBytes % 1024 == 0, "stage tiles must stay 1024-byte aligned");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "MMA N; two 32-column-multiple halves");
   static_assert(S % 2 == 0 || S == 3, "ring");
 };
 
@@ -192,8 +192,9 @@ __global__ void __launch_bounds__(kSteThreads, 1)
       mbar_wait(done, 0);
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2 .. 5)
+    // ------------------------------------------------------------ epilogue (warps 2 .. 2 + kSteEpiWarps - 1)
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;  // which half of the tile's columns
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
     const float scale = scale_ptr != nullptr ? __ldg(scale_ptr) : 1.0f;
     int tc = 0;
@@ -204,7 +205,7 @@ __global__ void __launch_bounds__(kSteThreads, 1)
       const int k = (t % r_tiles) * kSteBM + 32 * q + lane;
       const int c0 = (t / r_tiles) * BN;
 #pragma unroll 1
-      for (int cc = 0; cc < BN; cc += 32) {
+      for (int cc = half * (BN / 2); cc < (half + 1) * (BN / 2); cc += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(lane_base + b * BN + cc, v);
         tmem_ld_wait();
