@@ -823,7 +823,7 @@ bitnet_status bitnet_ste_backward_weight(const void* dY, const int8_t* x_q, cons
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   __nv_bfloat16* dyst = static_cast<__nv_bfloat16*>(workspace);  // [N][Mp]
   __nv_bfloat16* xt = dyst + N * Mp;                              // [K][Mp]
-  const dim3 g1(static_cast<unsigned>((N + 31) / 32), static_cast<unsigned>(Mp / 32));
+  const dim3 g1(static_cast<unsigned>((N + 63) / 64), static_cast<unsigned>(Mp / 64));
   if (launch_pdl(ste_scale_transpose_kernel, g1, dim3(256), 0, s, static_cast<const __nv_bfloat16*>(dY), a_scale,
                  static_cast<int>(M), static_cast<int>(N), static_cast<int>(Mp), dyst) != cudaSuccess)
     return BITNET_ERR_CUDA;

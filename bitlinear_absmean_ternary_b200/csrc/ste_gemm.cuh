@@ -262,46 +262,82 @@ __global__ void __launch_bounds__(256) ste_expand_wt_kernel(const uint8_t* __res
 }
 
 // Expansion of the activations for the weight gradient: XT[k][m] = x_q[m][k]
-// as bf16 (exact) for m < M, 0 for M <= m < Mp.
+// as bf16 (exact) for m < M, 0 for M <= m < Mp.  One 64 x 64 tile per CTA:
+// 16-byte reads of x_q rows (16 values of k), 16-byte writes of XT rows
+// (8 values of m) through a padded bf16 tile in shared memory.
 __global__ void __launch_bounds__(256) ste_expand_xt_kernel(const int8_t* __restrict__ xq, int M, int K, int Mp,
                                                             __nv_bfloat16* __restrict__ xt) {
-  __shared__ int8_t tile[64][65];  // [m][k]
+  __shared__ __align__(16) __nv_bfloat16 tile[64][72];  // [m][k]
   pdl_wait();
   const int m0 = blockIdx.x * 64, k0 = blockIdx.y * 64;
-  for (int i = threadIdx.x; i < 64 * 64; i += 256) {
-    const int m = i >> 6, k = i & 63;
-    tile[m][k] = (m0 + m < M && k0 + k < K) ? xq[static_cast<int64_t>(m0 + m) * K + k0 + k] : int8_t{0};
+  {
+    const int m = threadIdx.x >> 2, kc = (threadIdx.x & 3) * 16;  // 64 rows x 4 chunks of 16
+    int4 v = make_int4(0, 0, 0, 0);
+    if (m0 + m < M) v = __ldg(reinterpret_cast<const int4*>(xq + static_cast<int64_t>(m0 + m) * K + k0 + kc));
+    const uint32_t w[4] = {static_cast<uint32_t>(v.x), static_cast<uint32_t>(v.y), static_cast<uint32_t>(v.z),
+                           static_cast<uint32_t>(v.w)};
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      tile[m][kc + e] = __float2bfloat16_rn(static_cast<float>(static_cast<int8_t>(w[e >> 2] >> (8 * (e & 3)))));
   }
   __syncthreads();
   pdl_launch_dependents();
-  const int mm = threadIdx.x & 63, kr = threadIdx.x >> 6;
-  for (int k = kr; k < 64; k += 4)
-    if (k0 + k < K && m0 + mm < Mp)
-      xt[static_cast<int64_t>(k0 + k) * Mp + m0 + mm] = __float2bfloat16_rn(static_cast<float>(tile[mm][k]));
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {
+    const int idx = threadIdx.x + 256 * p;  // 64 rows of k x 8 chunks of 8 m
+    const int k = idx >> 3, mc = (idx & 7) * 8;
+    if (k0 + k < K && m0 + mc < Mp) {
+      uint32_t o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        o[e] = static_cast<uint32_t>(__bfloat16_as_ushort(tile[mc + 2 * e][k])) |
+               (static_cast<uint32_t>(__bfloat16_as_ushort(tile[mc + 2 * e + 1][k])) << 16);
+      *reinterpret_cast<uint4*>(xt + static_cast<int64_t>(k0 + k) * Mp + m0 + mc) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
 }
 
 // Pre-pass of the weight gradient: dYsT[n][m] = bf16_RNE(RN32(dY[m][n] * a[m]))
-// for m < M, 0 for M <= m < Mp (Mp a multiple of 64).  32 x 32 tiles through
-// shared memory so that both the reads of dY rows and the writes of dYsT rows
-// are coalesced.
+// for m < M, 0 for M <= m < Mp (Mp a multiple of 64).  One 64 x 64 tile per
+// CTA: 16-byte reads of dY rows (8 values of n), 16-byte writes of dYsT rows
+// (8 values of m) through a padded bf16 tile in shared memory.
 __global__ void __launch_bounds__(256) ste_scale_transpose_kernel(const __nv_bfloat16* __restrict__ dY,
                                                                   const float* __restrict__ a, int M, int N, int Mp,
                                                                   __nv_bfloat16* __restrict__ out) {
-  __shared__ float tile[32][33];
+  __shared__ __align__(16) __nv_bfloat16 tile[64][72];  // [m][n]
   pdl_wait();
-  const int n0 = blockIdx.x * 32, m0 = blockIdx.y * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8 threads
-  for (int i = ty; i < 32; i += 8) {
-    const int m = m0 + i, n = n0 + tx;
-    float v = 0.0f;
-    if (m < M && n < N) v = __fmul_rn(__bfloat162float(dY[static_cast<int64_t>(m) * N + n]), __ldg(a + m));
-    tile[i][tx] = v;
+  const int n0 = blockIdx.x * 64, m0 = blockIdx.y * 64;
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {
+    const int idx = threadIdx.x + 256 * p;  // 64 rows of m x 8 chunks of 8 n
+    const int m = idx >> 3, nc = (idx & 7) * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    float am = 0.0f;
+    if (m0 + m < M && n0 + nc < N) {
+      v = __ldg(reinterpret_cast<const uint4*>(dY + static_cast<int64_t>(m0 + m) * N + n0 + nc));
+      am = __ldg(a + m0 + m);
+    }
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t bits = (e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16);
+      tile[m][nc + e] = __float2bfloat16_rn(__fmul_rn(__uint_as_float(bits), am));
+    }
   }
   __syncthreads();
   pdl_launch_dependents();
-  for (int i = ty; i < 32; i += 8) {
-    const int n = n0 + i, m = m0 + tx;
-    if (n < N && m < Mp) out[static_cast<int64_t>(n) * Mp + m] = __float2bfloat16_rn(tile[tx][i]);
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {
+    const int idx = threadIdx.x + 256 * p;  // 64 rows of n x 8 chunks of 8 m
+    const int n = idx >> 3, mc = (idx & 7) * 8;
+    if (n0 + n < N && m0 + mc < Mp) {
+      uint32_t o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        o[e] = static_cast<uint32_t>(__bfloat16_as_ushort(tile[mc + 2 * e][n])) |
+               (static_cast<uint32_t>(__bfloat16_as_ushort(tile[mc + 2 * e + 1][n])) << 16);
+      *reinterpret_cast<uint4*>(out + static_cast<int64_t>(n0 + n) * Mp + m0 + mc) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
   }
 }
 
