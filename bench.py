@@ -66,10 +66,15 @@ def load_peaks() -> tuple:
 
 
 def kernel_source_hash(names) -> str:
+    """Hash of the kernel sources with comments and whitespace removed, so that
+    an edit of a comment does not orphan an ncu summary of the same code."""
     h = hashlib.sha256()
     for n in names:
-        with open(os.path.join(ROOT, "bitlinear_absmean_ternary_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "bitlinear_absmean_ternary_b200", "csrc", n), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(re.sub(r"\s+", "", text).encode())
     return h.hexdigest()[:16]
 
 

@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
         L.bitnet_bitlinear_gemv.restype = I
         L.bitnet_bitlinear_ffn_gemv.argtypes = [P, I, I64, I64, I64, P, F, P, P, P, P, P, F, P, P, P, P, I, P, P]
         L.bitnet_bitlinear_ffn_gemv.restype = I
+        L.bitnet_pack_weights_noalloc.argtypes = [P, I64, I64, F, P, P, P]
+        L.bitnet_pack_weights_noalloc.restype = I
         L.bitnet_b3_row_bytes.argtypes = [I64]
         L.bitnet_b3_row_bytes.restype = ctypes.c_size_t
         L.bitnet_pack_weights_b3.argtypes = [P, I64, I64, F, P, P, P, ctypes.c_size_t, P]
@@ -89,7 +91,7 @@ def declared_functions() -> list:
     with open(HEADER_PATH) as f:
         text = f.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(bitnet_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(bitnet_[a-z0-9_]+)\s*\(", text)))
 
 
 def status_string(status: int) -> str:
@@ -97,6 +99,11 @@ def status_string(status: int) -> str:
         return lib().bitnet_status_string(int(status)).decode()
     except Exception:  # the library itself is unavailable
         return "unknown"
+
+
+def bitnet_status_string(status: int) -> str:
+    """Text of a bitnet_status code."""
+    return status_string(status)
 
 
 def _check(fn: str, status: int) -> None:
@@ -163,6 +170,23 @@ def bitnet_pack_weights(W, eps: float = 1e-5, W_packed=None, gamma=None, workspa
     st = lib().bitnet_pack_weights(_ptr(W), N, K, eps, _ptr(W_packed), _ptr(gamma), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(W.device))
     _check("bitnet_pack_weights", st)
+    return W_packed, gamma
+
+
+def bitnet_pack_weights_noalloc(W, eps: float = 1e-5, W_packed=None, gamma=None):
+    """As bitnet_pack_weights, with the library's own fixed scratch instead of a
+    caller workspace (at most BITNET_PACK_NOALLOC_MAX_ROWS rows; concurrent calls
+    must not overlap).  Returns (W_packed, gamma).  Synchronises."""
+    torch = _torch()
+    _need_cuda(W)
+    N, K = W.shape
+    if W_packed is None:
+        W_packed = torch.empty((N, K // 4), dtype=torch.uint8, device=W.device)
+    if gamma is None:
+        gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    _need_cuda(W_packed, gamma)
+    st = lib().bitnet_pack_weights_noalloc(_ptr(W), N, K, eps, _ptr(W_packed), _ptr(gamma), _stream(W.device))
+    _check("bitnet_pack_weights_noalloc", st)
     return W_packed, gamma
 
 

@@ -27,7 +27,7 @@
 //
 // The first weight items are requested before waiting on the previous
 // kernel (programmatic dependent launch), because the weights never depend
-// on it; about 110 KB of shared memory per CTA lets the next kernel's CTA
+// on it; about 90 KB of shared memory per CTA lets the next kernel's CTA
 // sit on the same SM and do the same.
 #pragma once
 

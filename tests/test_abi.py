@@ -24,6 +24,14 @@ def test_every_declared_symbol_is_exported(L):
         assert hasattr(L, n), n
 
 
+def test_every_declared_entry_point_has_a_same_named_binding(L):
+    names = bl.declared_functions()
+    assert {"bitnet_b3_row_bytes", "bitnet_pack_weights_b3", "bitnet_bitlinear_gemv_b3", "bitnet_bitlinear_ffn_gemv",
+            "bitnet_ste_backward_input", "bitnet_ste_backward_weight"} <= set(names)
+    for n in names:
+        assert callable(getattr(bl, n, None)), n
+
+
 def test_status_strings(L):
     for code in range(6):
         s = bl.status_string(code)
