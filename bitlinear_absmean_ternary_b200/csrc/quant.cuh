@@ -1,6 +1,6 @@
 // Per-token absmax int8 activation quantisation fused with the RMSNorm that
 // precedes it (comrad404.com review, "Метод: как устроен BitNet b1.58":
-// 8-bit activations; RMSNorm; "normalise the input, then quantise").
+// 8-bit activations; RMSNorm; the input is normalised, then quantised).
 //
 // 256 threads per token row; thread t owns the 8-element chunks c = t,
 // t+256, ... and keeps them in registers, so x is read from HBM once.

@@ -116,8 +116,8 @@ bitnet_status bitnet_pack_weights_noalloc(const float* W, int64_t N, int64_t K, 
 /*
  * Per-token absmax int8 quantisation of activations, optionally fused with
  * the RMSNorm that precedes it (comrad404.com review, section "Метод":
- * 8-bit activations, RMSNorm in the LLaMA-like stack, "normalise, then
- * quantise").  One pass over x.  For each token row v (values widened to
+ * 8-bit activations, RMSNorm in the LLaMA-like stack, the input normalised
+ * before it is quantised).  One pass over x.  For each token row v (values widened to
  * fp32 exactly):
  *   with rms_gain:  ss = sum of RN32(v_k^2) in a fixed order (256 lanes, lane
  *                   l owning the 8-element chunks c = l, l+256, ... summed in

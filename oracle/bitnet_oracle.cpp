@@ -134,8 +134,8 @@ int oracle_pack_weights(const float* W, int64_t N, int64_t K, float eps, uint8_t
   return 0;
 }
 
-// RMSNorm of one token [Review, "Метод": RMSNorm in the LLaMA-like stack and
-// "normalise the input" as the first BitLinear step].
+// RMSNorm of one token [Review, "Метод": RMSNorm in the LLaMA-like stack, and
+// normalising the input is the first BitLinear step].
 void oracle_rmsnorm_row(const float* v, const float* g, int64_t K, float eps, float* h) {
   float lane[256];
   for (int l = 0; l < 256; ++l) lane[l] = 0.0f;
