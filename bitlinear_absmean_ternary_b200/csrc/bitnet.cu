@@ -18,6 +18,7 @@
 #include "pack.cuh"
 #include "ptx.cuh"
 #include "quant.cuh"
+#include "quant_rows.cuh"
 #include "ste_gemm.cuh"
 
 namespace {
@@ -140,9 +141,43 @@ cudaError_t launch_quant_t(const void* x, int64_t M, int K, const void* gain, fl
                     static_cast<const T*>(x), K, static_cast<const T*>(gain), eps, xq, a, rs);
 }
 
+template <int MAXC, bool NORM>
+cudaError_t launch_quant_rows_t(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
+                                int32_t* rs, cudaStream_t s) {
+  static bool done[kMaxDevices] = {};
+  const cudaError_t e = set_smem(quant_rows_kernel<MAXC, NORM>, 0, done);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = (M + kQuantRowsWarps - 1) / kQuantRowsWarps;
+  return launch_pdl(quant_rows_kernel<MAXC, NORM>, dim3(static_cast<unsigned>(grid)), dim3(kQuantRowsThreads), 0, s,
+                    static_cast<const __nv_bfloat16*>(x), M, K, static_cast<const __nv_bfloat16*>(gain), eps, xq, a,
+                    rs);
+}
+
+template <bool NORM>
+cudaError_t launch_quant_rows(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
+                              int32_t* rs, cudaStream_t s) {
+  const int per_lane = (K / 8 + 31) / 32;
+#define BN_QROWS(C) \
+  if (per_lane <= C) return launch_quant_rows_t<C, NORM>(x, M, K, gain, eps, xq, a, rs, s);
+  BN_QROWS(2) BN_QROWS(4) BN_QROWS(6) BN_QROWS(8) BN_QROWS(10) BN_QROWS(12) BN_QROWS(16) BN_QROWS(20)
+  BN_QROWS(24)
+#undef BN_QROWS
+  return cudaErrorInvalidValue;
+}
+
+// Token count from which the warp-per-row kernel takes over (bf16 input,
+// K <= 6144): from there on it keeps more rows in flight per SM; below, a CTA
+// per row spreads a short batch over more SMs.
+constexpr int64_t kQuantRowsMinM = 512;
+
 template <typename T>
 cudaError_t launch_quant(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
                          int32_t* rs, cudaStream_t s) {
+  if constexpr (sizeof(T) == 2) {
+    if (M >= kQuantRowsMinM && K <= 32 * 8 * kQuantRowsMaxChunks)
+      return gain != nullptr ? launch_quant_rows<true>(x, M, K, gain, eps, xq, a, rs, s)
+                             : launch_quant_rows<false>(x, M, K, gain, eps, xq, a, rs, s);
+  }
   const int per_thread = (K / 8 + kQuantThreads - 1) / kQuantThreads;
   if (gain == nullptr) {
     // No norm, so no fixed order: the fewest whole warps (at most 256 threads)

@@ -125,6 +125,18 @@ QUANT_CASES = [
     (5, 1344, "student_t4", 0.0, 1.0, "f32", True),
     (2, 32768, "normal", 0.0, 1.0, "bf16", True),
     (2, 16384, "normal", 0.0, 1.0, "f32", False),
+    # from 512 bf16 rows with K <= 6144 a warp quantises each row (quant_rows_kernel)
+    (512, 2560, "normal", 0.01, 20.0, "bf16", True),
+    (1024, 2624, "student_t4", 0.0, 1.0, "bf16", True),   # 328 chunks: lanes own 10 or 11
+    (600, 6144, "normal", 0.01, 20.0, "bf16", True),     # 24 chunks per lane, the most a warp holds
+    (513, 6080, "normal", 0.0, 1.0, "bf16", False),      # 760 chunks: lanes own 23 or 24
+    (600, 6912, "normal", 0.01, 20.0, "bf16", True),     # K above 6144: a CTA per row again
+    (777, 64, "normal", 0.0, 1.0, "bf16", True),         # 8 chunks: 24 lanes own none
+    (640, 1344, "student_t4", 0.0, 1.0, "bf16", False),
+    (2048, 5376, "normal", 0.005, 30.0, "bf16", True),
+    (4096, 6912, "student_t4", 0.0, 1.0, "bf16", False),  # the prefill down projection's input
+    (511, 2560, "normal", 0.0, 1.0, "bf16", True),       # one row below the warp kernel's threshold
+    (1024, 1344, "normal", 0.0, 1.0, "f32", True),       # fp32 input: a CTA per row at any M
 ]
 
 
@@ -161,6 +173,35 @@ def test_quant_edge_tokens(dev, orc):
     xq2, a2, rs2 = bl.bitnet_quant_act(_t(x, dev))
     assert rs2 is None
     np.testing.assert_array_equal(xq2.cpu().numpy(), orc.quant_act(x)[0])
+
+
+def test_quant_edge_tokens_many_rows(dev, orc):
+    """The same edge rows among 640 bf16 tokens, where one warp quantises each
+    row: zero, one-hot, exact ties after scaling, huge, tiny and a row whose
+    maximum sits in its last chunk (held by lane 31 for K = 2560 and 6144)."""
+    import torch
+    for K in (128, 2560, 6144):
+        x = synth.activations(640, K, 5, 2, "normal", 0.0, 1.0, "bf16")
+        x[0] = 0.0
+        x[1] = 0.0
+        x[1, K - 1] = -3.0
+        x[2, :10] = [127, 0.5, 1.5, 2.5, -2.5, -0.5, 126.5, 3.5, -3.5, 0.25]
+        x[2, 10:] = 0.0
+        x[3] *= np.float32(2.0 ** 40)
+        x[4] *= np.float32(2.0 ** -60)
+        x[5, K - 8:] = 100.0
+        x = orc.bf16_to_f32(orc.f32_to_bf16(x))
+        for norm in (False, True):
+            g = synth.gain(K, 5, 3, "bf16") if norm else None
+            xq, a, rs = bl.bitnet_quant_act(_x_dev(x, "bf16", dev), None if g is None else _x_dev(g, "bf16", dev),
+                                            EPS_RMS, want_rowsum=True)
+            xq_r, a_r, rs_r = orc.quant_act(x, g, EPS_RMS)
+            np.testing.assert_array_equal(xq.cpu().numpy(), xq_r)
+            np.testing.assert_array_equal(a.cpu().numpy(), a_r)
+            np.testing.assert_array_equal(rs.cpu().numpy(), rs_r)
+        # the first 511 rows alone take the CTA-per-row kernel: same codes and scales
+        xq5, a5, _ = bl.bitnet_quant_act(_x_dev(x[:511], "bf16", dev), _x_dev(g, "bf16", dev), EPS_RMS)
+        assert torch.equal(xq5, xq[:511]) and torch.equal(a5, a[:511])
 
 
 # --------------------------------------------------------------------------- linear
