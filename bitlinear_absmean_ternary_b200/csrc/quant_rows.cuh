@@ -3,13 +3,15 @@
 // review, "Метод: как устроен BitNet b1.58": 8-bit activations; the input is
 // normalised, then quantised).
 //
-// The CTA-per-row kernel of quant.cuh spends most of a row's life in its
-// three CTA barriers and keeps only a few rows' loads in flight per SM.  Here
-// a warp owns a row: lane l holds the 8-element chunks c = l, l+32, ... in
-// registers (MAXC of them, read once with 16-byte loads: the warp reads 512
-// contiguous bytes per load), and every reduction is a handful of shuffles,
-// so an SM keeps sixteen to thirty-odd rows in flight without any CTA
-// barrier.  bf16 input only, K <= 32 * 8 * MAXC.
+// The CTA-per-row kernel of quant.cuh passes three CTA barriers per row (one
+// per reduction).  Here a warp owns a row: lane l holds the 8-element chunks
+// c = l, l+32, ... in registers (MAXC of them, read once with 16-byte loads:
+// the warp reads 512 contiguous bytes per load), and every reduction is a
+// handful of shuffles, so rows proceed independently of one another; an SM
+// holds 16 of them at K = 6144 and 28 at K = 2560 (by register use), more
+// for shorter rows.  Back to back over 4096 rows of K = 2560 it moved
+// 4.45 TB/s against 3.62 TB/s for the CTA-per-row kernel.  bf16 input only,
+// K <= 32 * 8 * MAXC.
 //
 // The arithmetic, and with RMSNorm the order of the sum of squares, are those
 // of quant_row_cta, so the two kernels give the same bits.  That order is
