@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -38,24 +39,26 @@ int current_device() {
 }
 
 int sm_count() {
-  static int cache[kMaxDevices] = {};
+  static std::atomic<int> cache[kMaxDevices] = {};
   const int d = current_device();
   if (d < 0 || d >= kMaxDevices) return 148;
-  if (cache[d] == 0) {
-    int n = 0;
+  int n = cache[d].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess || n <= 0) n = 148;
-    cache[d] = n;
+    cache[d].store(n, std::memory_order_relaxed);
   }
-  return cache[d];
+  return n;
 }
 
 // Opt a kernel into more than 48 KB of dynamic shared memory and ask for the
-// largest shared-memory carveout (once per device).  With every kernel of the
+// largest shared-memory carveout (once per device; the flags are atomic, so
+// host threads making their first calls at once at worst repeat these
+// idempotent attribute calls).  With every kernel of the
 // library on the same carveout, a kernel launched with programmatic
 // dependent launch can place its CTAs next to the previous kernel's CTAs
 // without the SM first draining to change its L1/shared split.
 template <typename F>
-cudaError_t set_smem(F* fn, int bytes, bool (&done)[kMaxDevices]) {
+cudaError_t set_smem(F* fn, int bytes, std::atomic<bool> (&done)[kMaxDevices]) {
   const int d = current_device();
   if (d >= 0 && d < kMaxDevices && done[d]) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
@@ -134,7 +137,7 @@ bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t r
 template <typename T, int MAXC, int NTHR = kQuantThreads>
 cudaError_t launch_quant_t(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
                            int32_t* rs, cudaStream_t s, int threads = kQuantThreads) {
-  static bool done[kMaxDevices] = {};
+  static std::atomic<bool> done[kMaxDevices] = {};
   const cudaError_t e = set_smem(quant_act_kernel<T, MAXC, NTHR>, 0, done);
   if (e != cudaSuccess) return e;
   return launch_pdl(quant_act_kernel<T, MAXC, NTHR>, dim3(static_cast<unsigned>(M)), dim3(threads), 0, s,
@@ -144,7 +147,7 @@ cudaError_t launch_quant_t(const void* x, int64_t M, int K, const void* gain, fl
 template <int MAXC, bool NORM>
 cudaError_t launch_quant_rows_t(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
                                 int32_t* rs, cudaStream_t s) {
-  static bool done[kMaxDevices] = {};
+  static std::atomic<bool> done[kMaxDevices] = {};
   const cudaError_t e = set_smem(quant_rows_kernel<MAXC, NORM>, 0, done);
   if (e != cudaSuccess) return e;
   const int64_t grid = (M + kQuantRowsWarps - 1) / kQuantRowsWarps;
@@ -202,7 +205,7 @@ cudaError_t launch_quant(const void* x, int64_t M, int K, const void* gain, floa
 template <int MT, bool U8, bool XS>
 cudaError_t launch_gemv_x(const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
                           const int32_t* rs, void* y, int yd, cudaStream_t s) {
-  static bool done[kMaxDevices] = {};
+  static std::atomic<bool> done[kMaxDevices] = {};
   const cudaError_t e = set_smem(gemv_kernel<MT, U8, XS>, gemv_smem_bytes(MT, kGemvXMaxBytes / MT, XS), done);
   if (e != cudaSuccess) return e;
   const int64_t groups = (N + kGemvRows - 1) / kGemvRows;
@@ -260,10 +263,10 @@ cudaLaunchConfig_t gemm_config(int clusters, cudaStream_t s, cudaLaunchAttribute
 // one GPC, so this is not simply SMs / KS).  Cached per device.
 template <int BN, int S, bool U8, int KS>
 int gemm_cluster_capacity() {
-  static int cache[kMaxDevices] = {};
+  static std::atomic<int> cache[kMaxDevices] = {};
   const int d = current_device();
   if (d >= 0 && d < kMaxDevices && cache[d] > 0) return cache[d];
-  static bool done[kMaxDevices] = {};
+  static std::atomic<bool> done[kMaxDevices] = {};
   int n = 0;
   if (set_smem(gemm_kernel<BN, S, U8, KS>, GemmCfg<BN, S, KS>::kSmemBytes, done) == cudaSuccess) {
     if (KS == 1) {
@@ -284,7 +287,7 @@ template <int BN, int S, bool U8, int KS>
 cudaError_t launch_gemm_ks(const CUtensorMap& mx, const CUtensorMap& mw, const float* gamma, const float* a,
                            const int32_t* rs, int M, int N, int K, void* y, int yd, cudaStream_t s) {
   using C = GemmCfg<BN, S, KS>;
-  static bool done[kMaxDevices] = {};
+  static std::atomic<bool> done[kMaxDevices] = {};
   const cudaError_t e = set_smem(gemm_kernel<BN, S, U8, KS>, C::kSmemBytes, done);
   if (e != cudaSuccess) return e;
   const int64_t tiles = static_cast<int64_t>((N + kGemmBM - 1) / kGemmBM) * ((M + BN - 1) / BN);
@@ -368,7 +371,7 @@ cudaError_t launch_gemm_bn(const uint8_t* Wp, const float* gamma, int N, int K, 
 template <int MT, typename T, int MAXC>
 cudaError_t launch_fused_t(const void* x, const void* gain, float eps, const uint8_t* Wp, const float* gamma, int N,
                            int K, void* y, int yd, cudaStream_t s) {
-  static bool done[kMaxDevices] = {};
+  static std::atomic<bool> done[kMaxDevices] = {};
   auto kern = gemv_kernel<MT, true, true, true, T, MAXC>;
   const cudaError_t e = set_smem(kern, gemv_smem_bytes(MT, kGemvXMaxBytes / MT, true), done);
   if (e != cudaSuccess) return e;
@@ -414,7 +417,7 @@ cudaError_t launch_fused(int M, const void* x, const void* gain, float eps, cons
 // start while the previous kernel on the stream finishes.
 template <int MT, int MAXC>
 cudaError_t launch_ffn_t(const FfnArgs& a, int grid, size_t smem, cudaStream_t s) {
-  static bool done[kMaxDevices] = {};
+  static std::atomic<bool> done[kMaxDevices] = {};
   auto kern = ffn_kernel<MT, MAXC>;
   const cudaError_t e = set_smem(kern, kFfnSmemMax, done);
   if (e != cudaSuccess) return e;
@@ -469,7 +472,7 @@ constexpr int kGemvB3XMaxBytes = 24000;  // M * Kp: the quantised, zero-padded t
 template <int MT, typename T, int MAXC>
 cudaError_t launch_b3_t(const void* x, const void* gain, float eps, const uint8_t* Wp, const float* gamma, int N,
                         int K, void* y, int yd, cudaStream_t s) {
-  static bool done[kMaxDevices] = {};
+  static std::atomic<bool> done[kMaxDevices] = {};
   auto kern = gemv_b3_kernel<MT, T, MAXC>;
   const cudaError_t e = set_smem(kern, gemv_b3_smem_bytes(MT, kGemvB3XMaxBytes / MT), done);
   if (e != cudaSuccess) return e;
@@ -514,7 +517,7 @@ constexpr int kSteStages = 4;
 cudaError_t launch_ste(const CUtensorMap& ma, const CUtensorMap& mb, const float* scale, int R, int C, int J,
                        void* out, int od, cudaStream_t s) {
   using Cfg = SteCfg<kSteBN, kSteStages>;
-  static bool done[kMaxDevices] = {};
+  static std::atomic<bool> done[kMaxDevices] = {};
   auto kern = ste_gemm_kernel<kSteBN, kSteStages>;
   const cudaError_t e = set_smem(kern, Cfg::kSmemBytes, done);
   if (e != cudaSuccess) return e;
