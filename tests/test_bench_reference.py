@@ -31,3 +31,23 @@ def test_bench_rejects_too_few_warmup_steps():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--warmup", "2"],
                          capture_output=True, text=True, timeout=300, cwd=ROOT)
     assert out.returncode != 0
+
+
+def test_reference_arm_under_torchrun_prints_once_from_rank_0():
+    """Launched like the multi-GPU runs (torchrun, two ranks on 127.0.0.1): rank 0
+    alone times the oracle and prints the line, the other rank exits 0 without
+    work."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    out = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+                          "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+                          "--impl", "reference", "--gpus", "2", "--steps", "2", "--warmup", "3",
+                          "--workload", "bitlinear_m4_k256_n256"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, out.stdout[-2000:]
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
