@@ -269,6 +269,9 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
     import torch
     import bitlinear_absmean_ternary_b200 as bl
 
+    if not torch.cuda.is_available():
+        # no CPU fallback: the measured path is the CUDA library or nothing
+        sys.exit("bench.py: no CUDA device; this arm times the CUDA library (the oracle is --impl reference)")
     group = False
     if ws > 1:
         import torch.distributed as dist

@@ -51,3 +51,16 @@ def test_reference_arm_under_torchrun_prints_once_from_rank_0():
     assert len(lines) == 1, out.stdout[-2000:]
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+
+
+def test_gpu_arm_refuses_to_run_without_a_device():
+    """No CPU fallback: without CUDA the default arm exits non-zero with a plain message."""
+    import torch
+    if torch.cuda.is_available():
+        import pytest
+        pytest.skip("a CUDA device is present")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--steps", "1", "--warmup", "3", "--no-cpu"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode != 0
+    assert "no CUDA device" in out.stderr
+    assert not out.stdout.strip()
