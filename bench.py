@@ -6,19 +6,29 @@
 One step = one pass of the whole hot path over one batch: for every linear
 of the workload, the RMSNorm/absmax int8 quantisation of its input and the
 W1.58A8 product with dequant epilogue.  Decode shapes (M <= 8) run it as one
-kernel per linear (bitnet_bitlinear_gemv); the two-kernel path
-(bitnet_quant_act + bitnet_linear_gemv) is timed alongside under
-"unfused_step".  Larger batches use bitnet_quant_act + the tcgen05 GEMM.  Weight packing (absmean ternarisation) is the offline
-step: it runs once before timing and is reported separately under "stages".
+kernel per linear (bitnet_bitlinear_gemv, quantisation fused into the GEMV);
+larger batches run bitnet_quant_act + the tcgen05 GEMM.  Weight packing
+(absmean ternarisation) is the offline step: it runs once before timing and
+is reported separately under "stages".
 
-Timed region: W untimed warm-up steps, then exactly K steps replayed from
-CUDA graphs, bracketed by a barrier and a device synchronisation, timed with
-CUDA events on the launching stream; the max over ranks is taken.  Each step
-reads a different copy of the packed weights (32 copies per linear, more
-than twice the 126 MB L2 in total), the way successive layers of a model do,
-so the weights come from HBM.  value = algorithmic bytes of all ranks' steps
-/ max elapsed time.  With N > 1 every rank runs an independent replica (the
-path has no exchange step), so scaling is weak.
+The headline workload is the largest configuration that fits one GPU: the
+27B-class FFN at decode (M = 1, up 5376 -> 21504 and down 21504 -> 5376),
+in GB/s.  Every other configuration of the benchmark set is measured in the
+same run and reported under "configs", each with its own roofline and CPU
+oracle baseline: the small correctness case, the 2.5B decode GEMV, the
+batched decode through a 2.5B block (M = 64), the 2.5B prefill (M = 4096)
+and the 27B FFN at M = 16 and M = 2048.
+
+Timed region (headline): W untimed warm-up steps, then exactly K steps
+replayed from CUDA graphs, bracketed by a barrier and a device
+synchronisation, timed with CUDA events on the launching stream; the max over
+ranks is taken.  Every graph the timed region replays has been replayed
+before it starts.  Each step reads a different copy of the packed weights
+(enough copies that one rotation is over three times the 126 MB L2), the way
+successive layers of a model do, so the weights come from HBM.  value =
+algorithmic bytes of all ranks' steps / max elapsed time.  With N > 1 every
+rank runs an independent replica (the path has no exchange step), so scaling
+is weak.
 
 Rank 0 prints one JSON line.  `--impl reference` times the CPU oracle (the
 plain single-threaded C++ definition) on a bounded sample of the same
@@ -46,12 +56,18 @@ if ROOT not in sys.path:
 from bitlinear_absmean_ternary_b200 import synth  # noqa: E402
 
 METRIC = "BitLinear W1.58A8: decode GB/s & prefill TOPS, % of B200 roofline"
-DEFAULT_WORKLOAD = "decode_m1_2p5b_ffn"
+DEFAULT_WORKLOAD = "ffn27b_m1"
+# the benchmark configurations, smallest first (each reported under "configs")
+CONFIG_WORKLOADS = ["bitlinear_m4_k256_n256", "decode_m1_2p5b_ffn", "decode_m64_2p5b_block",
+                    "prefill_m4096_2p5b_ffn", "ffn27b_m1", "ffn27b_m16", "ffn27b_m2048"]
 EPS_W = 1e-5
 EPS_RMS = 1e-5
-COPIES = 32
+L2_BYTES = 126e6
+MAX_COPIES = 32
 GRAPH_STEPS = 128
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemv_decode_m1_2p5b_ffn.md")
+FLUSH_BYTES = 256 << 20
+NOMINAL_INT8_TOPS = 4500.0
+PROFILES = os.path.join(ROOT, "profiles")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -78,13 +94,13 @@ def kernel_source_hash(names) -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(path: str, src_hash: str):
+def profiled_traffic(path: str, src_hash: str, key: str = "traffic_bytes_per_launch"):
     """DRAM bytes per launch from a committed ncu summary, or None when the
     summary is missing or was taken on a different kernel source."""
     if not os.path.exists(path):
         return None
     text = open(path).read()
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m = re.search(re.escape(key) + r":\s*([0-9.eE+]+)", text)
     h = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
     if not m or not h or h.group(1) != src_hash:
         return None
@@ -93,12 +109,60 @@ def profiled_traffic(path: str, src_hash: str):
 
 def linear_bytes(lin) -> dict:
     """Algorithmic bytes of one linear: quant (x in, x_q/a/rowsum out) and
-    product (packed W, x_q, a, rowsum, gamma in; y out)."""
+    product (packed W, x_q, a, rowsum, gamma in; y out); `fused` is the
+    fused decode kernel's (x in, packed W, gamma, y out)."""
     xin = lin.M * lin.K * (2 if lin.x_dtype == "bf16" else 4) + (lin.K * 2 if lin.norm else 0)
     quant = xin + lin.M * lin.K + 8 * lin.M
     yb = lin.M * lin.N * (2 if lin.y_dtype == "bf16" else 4)
-    prod = lin.N * lin.K // 4 + lin.M * lin.K + 8 * lin.M + 4 + yb
-    return {"quant": quant, "product": prod, "x_in": xin, "y_out": yb}
+    w = lin.N * lin.K // 4
+    prod = w + lin.M * lin.K + 8 * lin.M + 4 + yb
+    return {"quant": quant, "product": prod, "fused": xin + w + 4 + yb, "x_in": xin, "y_out": yb, "w": w}
+
+
+def step_bytes(lins) -> int:
+    """Algorithmic bytes of one step (quantisation + product of every linear);
+    the same count for the fused and the two-kernel path."""
+    return sum(linear_bytes(l)["quant"] + linear_bytes(l)["product"] for l in lins)
+
+
+def step_ops(lins) -> int:
+    return sum(l.ops for l in lins)
+
+
+def int8_peak(peaks) -> float:
+    """Dense int8 tensor peak: the measured dense bf16 burst x 2 (the nominal
+    int8 / bf16 ratio, 4.5 / 2.25 PFLOP/s)."""
+    return float(peaks["bf16_tflops"]) * 2.0
+
+
+def roofline_bound(nbytes: float, ops: float, peaks) -> str:
+    """'tensor' when the int8 contraction takes longer at peak than moving the
+    algorithmic bytes at the measured HBM rate, else 'hbm'."""
+    t_hbm = nbytes / (float(peaks["hbm_gbs"]) * 1e9)
+    t_tc = ops / (int8_peak(peaks) * 1e12)
+    return "tensor" if t_tc > t_hbm else "hbm"
+
+
+def roofline(kernel: str, nbytes: float, ops: float, seconds: float, peaks, peak_src: str, how: str,
+             traffic=None, launches: int = 1) -> dict:
+    """Roofline object of a kernel: achieved rate of its algorithmic bytes or
+    ops (per launch, summed over `launches` launches taking `seconds`)."""
+    bound = roofline_bound(nbytes, ops, peaks)
+    src = "measured (MEASURED_PEAKS.json)" if peak_src == "measured" else "fallback"
+    if bound == "hbm":
+        peak = float(peaks["hbm_gbs"])
+        ach = nbytes / seconds / 1e9
+        out = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+               "peak_source": f"{src} hbm_gbs"}
+    else:
+        peak = int8_peak(peaks)
+        ach = ops / seconds / 1e12
+        out = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TOP/s", "frac": ach / peak,
+               "frac_of_nominal_int8": ach / NOMINAL_INT8_TOPS,
+               "peak_source": f"{src} bf16_tflops x 2 (dense int8 / dense bf16 nominal ratio)"}
+    out.update({"kernel": kernel, "traffic": traffic, "launch_us": seconds / launches * 1e6,
+                "bytes_per_launch": nbytes / launches, "ops_per_launch": ops / launches, "how": how})
+    return out
 
 
 class ClockSampler:
@@ -124,16 +188,19 @@ class ClockSampler:
         except Exception:
             self._nv = None
 
+    def _sample(self):
+        try:
+            self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+            bits = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            for b, name in self.REASONS.items():
+                if bits & b:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
     def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
-                bits = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
-                for b, name in self.REASONS.items():
-                    if bits & b:
-                        self.reasons.add(name)
-            except Exception:
-                pass
+            self._sample()
             time.sleep(self._period)
 
     def __enter__(self):
@@ -146,6 +213,7 @@ class ClockSampler:
         if self.ok:
             self._stop.set()
             self._t.join()
+            self._sample()  # one sample at the end of the region as well
 
     def summary(self) -> dict:
         if not self.ok or not self.samples:
@@ -181,50 +249,6 @@ def barrier(group_active: bool, device=None):
             dist.barrier()
 
 
-# ----------------------------------------------------------------------------- CPU oracle
-
-def oracle_step_sample(lins, time_budget_s: float):
-    """Prepare oracle inputs and a callable running one bounded sample step.
-
-    A sample step quantises every linear's input and forms the product for the
-    first `rows` output features of each linear (all tokens), where `rows` is
-    chosen so the step takes about time_budget_s.  Returns (step_fn,
-    bytes_per_step, description)."""
-    import oracle
-    prep = []
-    for lin in lins:
-        W = lin.make_w(0)
-        packed, gamma = oracle.pack_weights(W, EPS_W)
-        x = lin.make_x(0)
-        g = lin.make_gain(0)
-        prep.append((lin, packed, gamma, x, g))
-
-    def run(rows_frac: float):
-        for lin, packed, gamma, x, g in prep:
-            rows = max(1, int(round(lin.N * rows_frac)))
-            xq, a, rs = oracle.quant_act(x, g, EPS_RMS)
-            oracle.bitlinear(packed[:rows], gamma, lin.K, xq, a)
-
-    # calibrate on a small fraction
-    frac = 1.0 / 64
-    t0 = time.perf_counter()
-    run(frac)
-    dt = max(time.perf_counter() - t0, 1e-6)
-    frac = min(1.0, frac * time_budget_s / dt)
-
-    def bytes_for(f):
-        tot = 0
-        for lin, *_ in prep:
-            rows = max(1, int(round(lin.N * f)))
-            b = linear_bytes(lin)
-            tot += b["quant"] + rows * lin.K // 4 + lin.M * lin.K + 8 * lin.M + 4 + b["y_out"] * rows // lin.N
-        return tot
-
-    desc = (f"oracle on {frac * 100:.2f}% of the output features of every linear (all tokens; the full "
-            f"quantisation of every input) per step")
-    return (lambda: run(frac)), bytes_for(frac), desc, frac
-
-
 def host_info() -> dict:
     """CPU model and logical core count of the host the oracle runs on."""
     model = "unknown"
@@ -239,31 +263,318 @@ def host_info() -> dict:
     return {"cpu_model": model, "nproc": os.cpu_count()}
 
 
+def config_unit(lins, peaks) -> str:
+    """A configuration's rate unit: TOPS when its product is tensor-bound, else GB/s."""
+    b = sum(linear_bytes(l)["product"] for l in lins)
+    return "TOPS" if roofline_bound(b, step_ops(lins), peaks) == "tensor" else "GB/s"
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+_WCACHE = {}
+
+
+def weights_for(lin):
+    """Latent fp32 weights of a linear, generated once per weight spec."""
+    key = (lin.N, lin.K, lin.w_sigma, lin.w_id)
+    if key not in _WCACHE:
+        _WCACHE[key] = lin.make_w(0)
+    return _WCACHE[key]
+
+
+_OCACHE = {}
+
+
+def oracle_packed(lin):
+    import oracle
+    key = (lin.N, lin.K, lin.w_sigma, lin.w_id)
+    if key not in _OCACHE:
+        _OCACHE[key] = oracle.pack_weights(weights_for(lin), EPS_W)
+    return _OCACHE[key]
+
+
+def oracle_sample(lins, budget_s: float, unit: str):
+    """A bounded sample of one step of the workload on the CPU oracle.
+
+    Every linear quantises `tok` token rows of its input (all of them, or a
+    64-token slice for M >= 256, extrapolated per token) and forms the
+    product for the first `rows` output features, `rows` chosen so that the
+    call takes about budget_s.  Returns (call, work done per call in `unit`
+    (bytes for GB/s, ops for TOPS), description)."""
+    import oracle
+    prep = []
+    for lin in lins:
+        packed, gamma = oracle_packed(lin)
+        tok = lin.M if lin.M < 256 else 64
+        x = lin.make_x(0)[:tok]
+        g = lin.make_gain(0)
+        prep.append((lin, packed, gamma, np.ascontiguousarray(x), g, tok))
+
+    def run(frac: float):
+        for lin, packed, gamma, x, g, tok in prep:
+            rows = max(1, int(round(lin.N * frac)))
+            xq, a, _ = oracle.quant_act(x, g, EPS_RMS)
+            oracle.bitlinear(packed[:rows], gamma, lin.K, xq, a)
+
+    frac = 1.0 / 256
+    t0 = time.perf_counter()
+    run(frac)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    frac = min(1.0, frac * budget_s / dt)
+
+    def work(f):
+        tot = 0.0
+        for lin, _p, _g, _x, _gn, tok in prep:
+            rows = max(1, int(round(lin.N * f)))
+            if unit == "TOPS":
+                tot += 2.0 * tok * rows * lin.K
+            else:
+                b = linear_bytes(lin)
+                tot += (b["quant"] * tok / lin.M + rows * lin.K // 4 + tok * lin.K + 8 * tok + 4
+                        + b["y_out"] * tok / lin.M * rows / lin.N)
+        return tot
+
+    sliced = [p for p in prep if p[-1] != p[0].M]
+    slice_note = f"; a {sliced[0][-1]}-token slice of every input, extrapolated per token" if sliced else ""
+    desc = (f"oracle on {frac * 100:.2f}% of the output features of every linear (the full quantisation of the "
+            f"tokens it takes){slice_note}")
+    return (lambda: run(frac)), work(frac), desc
+
+
+def cpu_baseline(lins, unit: str, seconds: float) -> dict:
+    """The oracle as it stands, single-threaded, on a bounded sample (about `seconds` of CPU)."""
+    step, work, desc = oracle_sample(lins, min(2.0, seconds / 3), unit)
+    step()
+    n, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        step()
+        n += 1
+    el = time.perf_counter() - t0
+    scale = 1e9 if unit == "GB/s" else 1e12
+    return {"value": work * n / el / scale, "unit": unit, "cores": 1, "kind": "oracle",
+            "sample": f"{n} calls in {el:.1f} s, each {desc}", "host": host_info()}
+
+
 def run_reference(args, lins, rank: int):
     if rank != 0:
         return
+    import oracle
+    oracle.build()
     budget = 100.0 / max(1, args.steps + args.warmup)  # whole run about 100 s of CPU work
-    step, nbytes, desc, frac = oracle_step_sample(lins, budget)
+    unit = "GB/s"
+    step, work, desc = oracle_sample(lins, budget, unit)
     for _ in range(args.warmup):
         step()
     t0 = time.perf_counter()
     for _ in range(args.steps):
         step()
     el = time.perf_counter() - t0
-    value = nbytes * args.steps / el / 1e9
+    value = work * args.steps / el / 1e9
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
         "config": {"workload": args.workload, "linears": [[l.M, l.K, l.N] for l in lins], "parallelism": "replicas"},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": desc,
+        "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle", "sample": desc,
                          "host": host_info()},
-        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
 # ----------------------------------------------------------------------------- GPU arm
+
+class Workload:
+    """Device state of one workload: packed weights (rotated copies), inputs,
+    output buffers, and the launches of one step."""
+
+    def __init__(self, torch, bl, dev, lins, packs, rotate: bool):
+        self.torch, self.bl, self.dev, self.lins = torch, bl, dev, lins
+        wbytes = sum(l.N * l.K // 4 for l in lins)
+        self.copies = max(2, min(MAX_COPIES, math.ceil(3 * L2_BYTES / wbytes))) if rotate else 1
+        self.packs = [packs.get(torch, bl, dev, l, self.copies) for l in lins]
+        self.xs, self.gains, self.bufs = [], [], []
+        for lin in lins:
+            self.xs.append(self._act(lin.make_x(0), lin.x_dtype))
+            g = lin.make_gain(0)
+            self.gains.append(None if g is None else self._act(g, lin.x_dtype))
+            ydt = torch.bfloat16 if lin.y_dtype == "bf16" else torch.float32
+            self.bufs.append({
+                "xq": torch.empty((lin.M, lin.K), dtype=torch.int8, device=dev),
+                "a": torch.empty(lin.M, dtype=torch.float32, device=dev),
+                "rs": torch.empty(lin.M, dtype=torch.int32, device=dev),
+                "y": torch.empty((lin.M, lin.N), dtype=ydt, device=dev)})
+        self.fused = all(l.M <= 8 and l.M * l.K <= 21504 for l in lins)
+        self.kernels_per_step = (1 if self.fused else 2) * len(lins)
+        self.product_kernel = ("gemv_kernel (fused quantisation + GEMV, bitnet_bitlinear_gemv)" if self.fused else
+                               "gemv_kernel (bitnet_linear_gemv)" if all(l.M <= 8 for l in lins) else
+                               "gemm_kernel (tcgen05, bitnet_linear_gemm)")
+
+    def _act(self, a, dtype):
+        torch = self.torch
+        if dtype == "bf16":
+            return torch.from_numpy(synth.f32_to_bf16_bits(a).view(np.int16).copy()).to(self.dev).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(self.dev)
+
+    def quant(self, i, _c):
+        b = self.bufs[i]
+        self.bl.bitnet_quant_act(self.xs[i], self.gains[i], EPS_RMS, b["xq"], b["a"], b["rs"])
+
+    def product(self, i, c):
+        lin, b = self.lins[i], self.bufs[i]
+        fn = self.bl.bitnet_linear_gemv if lin.M <= 8 else self.bl.bitnet_linear_gemm
+        fn(self.packs[i][0][c % self.copies], self.packs[i][1], b["xq"], b["a"], b["rs"], y=b["y"])
+
+    def fused_linear(self, i, c):
+        self.bl.bitnet_bitlinear_gemv(self.xs[i], self.packs[i][0][c % self.copies], self.packs[i][1],
+                                      self.gains[i], EPS_RMS, y=self.bufs[i]["y"])
+
+    def linear(self, i, c):
+        if self.fused:
+            self.fused_linear(i, c)
+        else:
+            self.quant(i, c)
+            self.product(i, c)
+
+    def step(self, c):
+        for i in range(len(self.lins)):
+            self.linear(i, c)
+
+    def step_unfused(self, c):
+        for i in range(len(self.lins)):
+            self.quant(i, c)
+            self.product(i, c)
+
+
+class PackCache:
+    """Packed weights (and their rotated copies) per weight spec, shared by the
+    workloads that use the same matrices; the pack time is recorded."""
+
+    def __init__(self):
+        self.d = {}
+        self.pack_ms = {}
+
+    def get(self, torch, bl, dev, lin, copies):
+        key = (lin.N, lin.K, lin.w_sigma, lin.w_id)
+        if key not in self.d:
+            W = torch.from_numpy(weights_for(lin)).to(dev)
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            P, G = bl.bitnet_pack_weights(W, EPS_W)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            self.pack_ms[f"{lin.N}x{lin.K}"] = e0.elapsed_time(e1)
+            del W
+            self.d[key] = ([P], G)
+        lst, G = self.d[key]
+        while len(lst) < copies:
+            lst.append(lst[0].clone())
+        return lst, G
+
+
+def capture(torch, stream, fn_per_step, nsteps: int, start: int = 0):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for s in range(nsteps):
+            fn_per_step(start + s)
+    return g
+
+
+def replay_ms(torch, dev, stream, graph, replays: int, group=False) -> float:
+    """CUDA-event time of `replays` back-to-back replays (the graph was replayed before)."""
+    barrier(group, dev)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):  # replay() launches on the current stream
+        e0.record(stream)
+        for _ in range(replays):
+            graph.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(group, dev)
+    return max_over_ranks(e0.elapsed_time(e1), group, dev)
+
+
+def per_launch_ms(torch, dev, stream, wl, fn, i, steps: int = GRAPH_STEPS, replays: int = 10, group=False) -> float:
+    """Average time of one launch kind of linear i, back to back in a CUDA graph
+    over the rotating weight copies (after one untimed replay)."""
+    g = capture(torch, stream, lambda c: fn(i, c), steps)
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize(dev)
+    return replay_ms(torch, dev, stream, g, replays, group) / (steps * replays)
+
+
+def measure_rotating(torch, bl, dev, stream, wl, peaks, peak_src, group, steps=GRAPH_STEPS, replays=20) -> dict:
+    """A decode-sized configuration: steps back to back in CUDA graphs over the
+    rotating weight copies, and each kernel kind alone the same way."""
+    g = capture(torch, stream, wl.step, steps)
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize(dev)
+    ms = replay_ms(torch, dev, stream, g, replays, group) / (steps * replays)
+    lins = wl.lins
+    per = []
+    for i, lin in enumerate(lins):
+        prod = wl.fused_linear if wl.fused else wl.product
+        pms = per_launch_ms(torch, dev, stream, wl, prod, i, group=group)
+        qms = None if wl.fused else per_launch_ms(torch, dev, stream, wl, wl.quant, i, group=group)
+        per.append({"linear": lin.name, "M": lin.M, "K": lin.K, "N": lin.N, "product_us": pms * 1e3,
+                    "quant_us": None if qms is None else qms * 1e3})
+    kbytes = sum(linear_bytes(l)["fused" if wl.fused else "product"] for l in lins)
+    ksec = sum(p["product_us"] for p in per) * 1e-6
+    rl = roofline(wl.product_kernel, kbytes, step_ops(lins), ksec, peaks, peak_src,
+                  "each linear's product kernel alone, back to back in CUDA graphs over the rotating weight copies, "
+                  "CUDA events on the launching stream; bytes and time summed over the linears", launches=len(lins))
+    return {"ms_per_step": ms, "per_linear": per, "roofline": rl, "weight_copies": wl.copies,
+            "device_status": bl.bitnet_get_device_status(),
+            "timing": f"CUDA graphs of {steps} steps over {wl.copies} rotating weight copies, {replays} replays "
+                      "after one untimed replay, CUDA events"}
+
+
+def measure_flushed(torch, bl, dev, stream, wl, peaks, peak_src, group, reps=10) -> dict:
+    """A prefill-sized configuration: each step with the L2 flushed (256 MB
+    write) before it; CUDA events around every kernel; medians of reps steps
+    after 3 untimed ones."""
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    lins = wl.lins
+    qt = [[] for _ in lins]
+    pt = [[] for _ in lins]
+    st = []
+    with torch.cuda.stream(stream):
+        for it in range(reps + 3):
+            flush.zero_()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * len(lins) + 1)]
+            ev[0].record(stream)
+            for i in range(len(lins)):
+                wl.quant(i, 0)
+                ev[2 * i + 1].record(stream)
+                wl.product(i, 0)
+                ev[2 * i + 2].record(stream)
+            torch.cuda.synchronize(dev)
+            if it >= 3:
+                for i in range(len(lins)):
+                    qt[i].append(ev[2 * i].elapsed_time(ev[2 * i + 1]))
+                    pt[i].append(ev[2 * i + 1].elapsed_time(ev[2 * i + 2]))
+                st.append(ev[0].elapsed_time(ev[-1]))
+    med = lambda v: max_over_ranks(statistics.median(v), group, dev)
+    per = []
+    for i, lin in enumerate(lins):
+        qb = linear_bytes(lin)["quant"]
+        qms, pms = med(qt[i]), med(pt[i])
+        per.append({"linear": lin.name, "M": lin.M, "K": lin.K, "N": lin.N, "product_us": pms * 1e3,
+                    "product_tops": lin.ops / (pms / 1e3) / 1e12, "quant_us": qms * 1e3,
+                    "quant_gbs": qb / (qms / 1e3) / 1e9, "quant_frac": qb / (qms / 1e3) / 1e9 / float(peaks["hbm_gbs"])})
+    kbytes = sum(linear_bytes(l)["product"] for l in lins)
+    ksec = sum(p["product_us"] for p in per) * 1e-6
+    rl = roofline(wl.product_kernel, kbytes, step_ops(lins), ksec, peaks, peak_src,
+                  "single launches with the L2 flushed before each step, CUDA events; median of "
+                  f"{reps}; ops and time summed over the linears", launches=len(lins))
+    return {"ms_per_step": med(st), "per_linear": per, "roofline": rl, "device_status": bl.bitnet_get_device_status(),
+            "timing": f"one step at a time with a {FLUSH_BYTES >> 20} MB L2 flush before it; median of {reps} "
+                      "steps after 3 untimed ones"}
+
 
 def run_ours(args, lins, ws: int, rank: int, local: int):
     import torch
@@ -283,115 +594,31 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
     bl.lib()
     peaks, peak_src = load_peaks()
     stream = torch.cuda.Stream(dev)
-
-    # ---- inputs and offline weight packing (timed once, reported under "stages"); one
-    # untimed pack first so that the library's first-call setup is not in the figure
+    packs = PackCache()
+    # one untimed pack first so that the library's first-call setup is not in the pack figures
     bl.bitnet_pack_weights(torch.ones((64, 64), dtype=torch.float32, device=dev), EPS_W)
     torch.cuda.synchronize(dev)
-    packs, xs, gains, bufs = [], [], [], []
-    pack_ms = []
-    for lin in lins:
-        W = torch.from_numpy(lin.make_w(0)).to(dev)
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            P, G = bl.bitnet_pack_weights(W, EPS_W)
-            e1.record(stream)
-        torch.cuda.synchronize(dev)
-        pack_ms.append(e0.elapsed_time(e1))
-        copies = [P] + [P.clone() for _ in range(COPIES - 1)]
-        packs.append((copies, G))
-        del W
-        x = lin.make_x(0)
-        if lin.x_dtype == "bf16":
-            xt = torch.from_numpy(synth.f32_to_bf16_bits(x).view(np.int16).copy()).to(dev).view(torch.bfloat16)
-        else:
-            xt = torch.from_numpy(x).to(dev)
-        xs.append(xt)
-        g = lin.make_gain(0)
-        if g is None:
-            gains.append(None)
-        elif lin.x_dtype == "bf16":
-            gains.append(torch.from_numpy(synth.f32_to_bf16_bits(g).view(np.int16).copy()).to(dev).view(torch.bfloat16))
-        else:
-            gains.append(torch.from_numpy(g).to(dev))
-        ydt = torch.bfloat16 if lin.y_dtype == "bf16" else torch.float32
-        bufs.append({
-            "xq": torch.empty((lin.M, lin.K), dtype=torch.int8, device=dev),
-            "a": torch.empty(lin.M, dtype=torch.float32, device=dev),
-            "rs": torch.empty(lin.M, dtype=torch.int32, device=dev),
-            "y": torch.empty((lin.M, lin.N), dtype=ydt, device=dev),
-        })
-    torch.cuda.synchronize(dev)
 
-    def quant(i, _c):
-        b = bufs[i]
-        bl.bitnet_quant_act(xs[i], gains[i], EPS_RMS, b["xq"], b["a"], b["rs"])
-
-    def product(i, c):
-        lin, b = lins[i], bufs[i]
-        fn = bl.bitnet_linear_gemv if lin.M <= 8 else bl.bitnet_linear_gemm
-        fn(packs[i][0][c % COPIES], packs[i][1], b["xq"], b["a"], b["rs"], y=b["y"])
-
-    def fused(i, c):
-        # quantisation + product in one kernel (decode shapes)
-        b = bufs[i]
-        bl.bitnet_bitlinear_gemv(xs[i], packs[i][0][c % COPIES], packs[i][1], gains[i], EPS_RMS, y=b["y"])
-
-    def step_unfused(c):
-        for i in range(len(lins)):
-            quant(i, c)
-            product(i, c)
-
-    def step_fused(c):
-        for i in range(len(lins)):
-            fused(i, c)
-
-    use_fused = all(l.M <= 8 and l.M * l.K <= 21504 for l in lins)
-    step = step_fused if use_fused else step_unfused
-
-    def capture(fn_per_step, nsteps: int, start: int = 0):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for s in range(nsteps):
-                fn_per_step(start + s)
-        return g
-
-    def time_graph(graph, replays: int) -> float:
-        barrier(group, dev)
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):  # replay() launches on the current stream
-            e0.record(stream)
-            for _ in range(replays):
-                graph.replay()
-            e1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier(group, dev)
-        return e0.elapsed_time(e1)
-
-    G = GRAPH_STEPS
+    # ------------------------------------------------------------------ headline: exactly K steps
+    wl = Workload(torch, bl, dev, lins, packs, rotate=True)
     K = args.steps
+    G = min(GRAPH_STEPS, K)
     full, rem = divmod(K, G)
-    g_main = capture(step, G)
-    g_rem = capture(step, rem) if rem else None
-    # warm-up: W untimed steps
-    wfull, wrem = divmod(args.warmup, G)
-    g_warm = capture(step, wrem) if wrem else None
+    g_main = capture(torch, stream, wl.step, G)
+    g_rem = capture(torch, stream, wl.step, rem, start=full * G) if rem else None
+    # warm-up: at least W steps, and every graph of the timed region replayed once
+    warm_replays = max(1, math.ceil(max(0, args.warmup - rem) / G)) if full else 0
     with torch.cuda.stream(stream):
-        for _ in range(wfull):
+        for _ in range(warm_replays):
             g_main.replay()
-        if g_warm is not None:
-            g_warm.replay()
+        if g_rem is not None:
+            g_rem.replay()
     torch.cuda.synchronize(dev)
-    # the timed region: exactly K steps
-    kernels_per_step = (1 if use_fused else 2) * len(lins)
+    warm_steps = warm_replays * G + rem
     with ClockSampler(dev.index) as clocks:
         barrier(group, dev)
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        # an event after every graph of G steps: per-step percentiles over the replays
         marks = [torch.cuda.Event(enable_timing=True) for _ in range(full)]
         with torch.cuda.stream(stream):
             e0.record(stream)
@@ -404,163 +631,131 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
         torch.cuda.synchronize(dev)
         barrier(group, dev)
     el_ms = max_over_ranks(e0.elapsed_time(e1), group, dev)
-    per_step_us = [(a.elapsed_time(b) if a is not None else e0.elapsed_time(b)) * 1e3 / G
-                   for a, b in zip([None] + marks[:-1], marks)]
+    head_status = bl.bitnet_get_device_status()
+    per_rep = [(a.elapsed_time(b) if a is not None else e0.elapsed_time(b)) * 1e3 / G
+               for a, b in zip([None] + marks[:-1], marks)]
     step_stats = None
-    if len(per_step_us) >= 2:
-        qs = np.percentile(per_step_us, [10, 50, 90])
+    if len(per_rep) >= 2:
+        qs = np.percentile(per_rep, [10, 50, 90])
         step_stats = {"p10_us": float(qs[0]), "p50_us": float(qs[1]), "p90_us": float(qs[2]),
-                      "samples": len(per_step_us), "per": f"graph replay of {G} steps"}
-    step_bytes = sum(linear_bytes(l)["quant"] + linear_bytes(l)["product"] for l in lins)
-    value = ws * K * step_bytes / (el_ms / 1e3) / 1e9
+                      "samples": len(per_rep), "per": f"graph replay of {G} steps"}
+    sbytes = step_bytes(lins)
+    value = ws * K * sbytes / (el_ms / 1e3) / 1e9
+    del g_main, g_rem
 
-    # ---- per-kernel-kind graphs for the stage breakdown and the roofline (same
-    # kernels, same launch configuration, same weight rotation, back to back)
-    def per_stage(fn, label):
-        g = capture(lambda c: [fn(i, c) for i in range(len(lins))], G)
-        with torch.cuda.stream(stream):
-            g.replay()
-        torch.cuda.synchronize(dev)
-        reps = max(1, min(50, (K // G) // 4))
-        ms = max_over_ranks(time_graph(g, reps), group, dev)
-        return ms / (reps * G * len(lins))  # per launch
-
-    prod_ms = per_stage(product, "product")
-    quant_ms = per_stage(quant, "quant")
-    fused_ms = per_stage(fused, "fused") if use_fused else None
-    prod_bytes = statistics.mean(linear_bytes(l)["product"] for l in lins)
-    quant_bytes = statistics.mean(linear_bytes(l)["quant"] for l in lins)
-    hbm_peak = float(peaks["hbm_gbs"])
-    if use_fused:
-        # the dominant (only) kernel of the step: fused quantisation + GEMV;
-        # its algorithmic bytes: x in, packed W, scales, y out
-        kern, kern_ms = "gemv_kernel (fused quant + GEMV, bitnet_bitlinear_gemv)", fused_ms
-        kern_bytes = statistics.mean(linear_bytes(l)["x_in"] + l.N * l.K // 4 + 4 + linear_bytes(l)["y_out"]
-                                     for l in lins)
-        src = kernel_source_hash(["gemv.cuh", "quant.cuh", "ptx.cuh"])
-    elif lins[0].M <= 8:
-        kern, kern_ms, kern_bytes = "gemv_kernel", prod_ms, prod_bytes
-        src = kernel_source_hash(["gemv.cuh", "ptx.cuh"])
-    else:
-        kern, kern_ms, kern_bytes = "gemm_kernel", prod_ms, prod_bytes
-        src = kernel_source_hash(["gemm.cuh", "ptx.cuh"])
-    traffic = profiled_traffic(PROFILE_SUMMARY, src)
-    achieved = kern_bytes / (kern_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-                "traffic": traffic, "kernel": kern,
-                "peak_source": f"{peak_src} hbm_gbs (MEASURED_PEAKS.json)" if peak_src == "measured" else
-                "fallback 6650 GB/s", "launch_us": kern_ms * 1e3, "bytes_per_launch": kern_bytes,
-                "how": "back-to-back launches of this kernel alone in CUDA graphs over the rotating weight copies, "
-                       "CUDA events on the launching stream; average time per launch"}
-
-    # ---- the other path over the same K steps (four-call path when the fused one is timed above)
+    # ------------------------------------------------------------------ the headline's kernels and roofline
+    head = measure_rotating(torch, bl, dev, stream, wl, peaks, peak_src, group)
+    rl = head["roofline"]
+    if wl.fused and lins[0].K == 5376 and lins[0].N == 21504:
+        rl["traffic"] = profiled_traffic(os.path.join(PROFILES, "gemv_decode_m1_27b_ffn.md"),
+                                         kernel_source_hash(["gemv.cuh", "quant.cuh", "ptx.cuh"]))
     unfused = None
-    if use_fused:
-        gu = capture(step_unfused, G)
+    if wl.fused:
+        gu = capture(torch, stream, wl.step_unfused, GRAPH_STEPS)
         with torch.cuda.stream(stream):
             gu.replay()
         torch.cuda.synchronize(dev)
-        reps = max(1, K // G)
-        ms = max_over_ranks(time_graph(gu, reps), group, dev)
-        unfused = {"value": ws * reps * G * step_bytes / (ms / 1e3) / 1e9, "unit": "GB/s",
-                   "ms_per_step": ms / (reps * G), "steps": reps * G, "kernels_per_step": 2 * len(lins),
+        ms = replay_ms(torch, dev, stream, gu, 10, group) / (10 * GRAPH_STEPS)
+        del gu
+        unfused = {"value": ws * sbytes / (ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
+                   "kernels_per_step": 2 * len(lins),
                    "what": "bitnet_quant_act + bitnet_linear_gemv per linear (two kernels)"}
 
-    # ---- end to end through the public API with host buffers
+    # ------------------------------------------------------------------ end to end through the public API
     h2d = sum(linear_bytes(l)["x_in"] for l in lins)
     d2h = sum(linear_bytes(l)["y_out"] for l in lins)
-    xs_host = [x.cpu().pin_memory() for x in xs]
-    ys_host = [torch.empty_like(b["y"], device="cpu").pin_memory() for b in bufs]
-    k_e2e = min(K, 4000)
+    xs_host = [x.cpu().pin_memory() for x in wl.xs]
+    ys_host = [torch.empty_like(b["y"], device="cpu").pin_memory() for b in wl.bufs]
+    k_e2e = min(max(K, 200), 2000)
 
-    def e2e_step(c):
-        for i, lin in enumerate(lins):
-            xs[i].copy_(xs_host[i], non_blocking=True)
-            if use_fused:
-                fused(i, c)
-            else:
-                quant(i, c)
-                product(i, c)
-            ys_host[i].copy_(bufs[i]["y"], non_blocking=True)
+    def e2e_loop(n, copies=True, calls=True):
+        with torch.cuda.stream(stream):
+            torch.cuda.synchronize(dev)
+            barrier(group, dev)
+            t0 = time.perf_counter()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for c in range(n):
+                for i in range(len(lins)):
+                    if copies:
+                        wl.xs[i].copy_(xs_host[i], non_blocking=True)
+                    if calls:
+                        wl.linear(i, c)
+                    if copies:
+                        ys_host[i].copy_(wl.bufs[i]["y"], non_blocking=True)
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            host_ms = (time.perf_counter() - t0) * 1e3
+            barrier(group, dev)
+        return max_over_ranks(a.elapsed_time(b), group, dev), host_ms
 
-    with torch.cuda.stream(stream):
-        for c in range(min(200, k_e2e)):
-            e2e_step(c)
-        torch.cuda.synchronize(dev)
-        barrier(group, dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for c in range(k_e2e):
-            e2e_step(c)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier(group, dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), group, dev)
-    e2e = {"value": ws * k_e2e * step_bytes / (e2e_ms / 1e3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "steps": k_e2e,
+    e2e_loop(min(200, k_e2e))
+    e2e_ms, _ = e2e_loop(k_e2e)
+    copies_ms, _ = e2e_loop(min(500, k_e2e), calls=False)
+    calls_ms, calls_host_ms = e2e_loop(min(500, k_e2e), copies=False)
+    nb = min(500, k_e2e)
+    e2e = {"value": ws * k_e2e * sbytes / (e2e_ms / 1e3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "steps": k_e2e, "us_per_step": e2e_ms * 1e3 / k_e2e,
+           "breakdown_us_per_step": {"copies_only": copies_ms * 1e3 / nb, "api_calls_only": calls_ms * 1e3 / nb,
+                                     "api_calls_host_wall": calls_host_ms * 1e3 / nb,
+                                     "kernels_back_to_back": head["ms_per_step"] * 1e3},
            "how": "eager Python calls of the public API per step: pinned H2D copy of every input, the BitLinear "
-                  "call(s), D2H copy of every output"}
+                  "call(s), D2H copy of every output; the breakdown repeats the loop with the copies alone and the "
+                  "calls alone"}
+    del xs_host, ys_host
 
-    # ---- prefill tensor-core GEMM (M = 4096), a secondary line of the same metric
-    prefill = None
-    if not args.no_prefill and lins[0].M <= 8:
-        prefill = bench_prefill(torch, bl, dev, stream, peaks, peak_src, group)
+    # ------------------------------------------------------------------ every configuration
+    configs = {}
+    if not args.no_configs:
+        for name in CONFIG_WORKLOADS:
+            if name == args.workload:
+                continue
+            configs[name] = bench_config(torch, bl, dev, stream, name, packs, peaks, peak_src, group,
+                                         rank == 0 and ws == 1 and not args.no_cpu, args.config_cpu_seconds)
 
-    # ---- STE backward GEMMs at the prefill shapes, a secondary line
+    # ------------------------------------------------------------------ secondary kernels
+    ffn_block = None
+    if not args.no_ffn:
+        ffn_block = {n: bench_ffn_block(torch, bl, dev, stream, peaks, peak_src, group, n)
+                     for n in ("ffn_block_m1_27b", "ffn_block_m1_2p5b")}
+    decode_b3 = None
+    if not args.no_b3 and wl.fused and all(l.M * ((l.K + 79) // 80 * 80) <= 24000 for l in lins):
+        decode_b3 = bench_b3(torch, bl, dev, stream, wl, peaks, group, el_ms / K)
     ste = None
-    if not args.no_ste and lins[0].M <= 8:
+    if not args.no_ste:
         ste = bench_ste(torch, bl, dev, stream, peaks, peak_src, group)
 
-    # ---- the decode step on base-3 packed weights, a secondary line
-    decode_b3 = None
-    if not args.no_b3 and use_fused and all(l.M * ((l.K + 79) // 80 * 80) <= 24000 for l in lins):
-        decode_b3 = bench_b3(torch, bl, dev, stream, lins, xs, gains, peaks, peak_src, group, el_ms / K)
-
-    # ---- the one-launch decode FFN block (up, gate, squared-ReLU gating, down), a secondary line
-    ffn_block = None
-    if not args.no_ffn and lins[0].M <= 8:
-        ffn_block = bench_ffn_block(torch, bl, dev, stream, peaks, peak_src, group)
-
-    # ---- CPU oracle baseline (rank 0, N = 1)
+    # ------------------------------------------------------------------ CPU oracle baseline (rank 0, N = 1)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu:
-        stepfn, nbytes, desc, _ = oracle_step_sample(lins, 1.0)
-        stepfn()
-        n, t0 = 0, time.perf_counter()
-        while time.perf_counter() - t0 < args.cpu_seconds:
-            stepfn()
-            n += 1
-        el = time.perf_counter() - t0
-        cpu = {"value": nbytes * n / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": f"{n} steps, each {desc}; {el:.1f} s", "host": host_info()}
+        cpu = cpu_baseline(lins, "GB/s", args.cpu_seconds)
 
     if rank == 0:
-        clk = clocks.summary()
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": ws, "steps": K, "warmup": args.warmup,
-            "ms_per_step": el_ms / K, "step_percentiles": step_stats, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": "int8", "data": "synthetic",
+            "warmup_steps_run": warm_steps, "ms_per_step": el_ms / K, "step_percentiles": step_stats,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": {"workload": args.workload, "linears": [[l.M, l.K, l.N] for l in lins],
                        "step": ("per linear: one bitnet_bitlinear_gemv kernel (RMSNorm/absmax int8 quantisation of "
-                                "the input fused with the ternary GEMV and dequant)") if use_fused else
+                                "the input fused with the ternary GEMV and dequant)") if wl.fused else
                                "per linear: bitnet_quant_act + ternary product with dequant",
-                       "l2": f"{COPIES} rotating packed-weight copies per linear "
-                             f"({COPIES * sum(l.N * l.K // 4 for l in lins) / 1e6:.0f} MB > 126 MB L2)",
-                       "timing": f"CUDA graphs of {G} steps, programmatic dependent launch between kernels",
+                       "l2": f"{wl.copies} rotating packed-weight copies per linear "
+                             f"({wl.copies * sum(l.N * l.K // 4 for l in lins) / 1e6:.0f} MB > 126 MB L2)",
+                       "timing": f"CUDA graphs of {G} steps, programmatic dependent launch between kernels; every "
+                                 "graph of the timed region replayed during the warm-up",
                        "parallelism": "replicas" if ws > 1 else "single"},
-            "roofline": roofline,
+            "roofline": rl,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": K * kernels_per_step,
-            "clocks": clk,
+            "gpu_launches": K * wl.kernels_per_step,
+            "clocks": clocks.summary(),
+            "device_status": head_status,
+            "kernels": {"ms_per_step_back_to_back": head["ms_per_step"], "per_linear": head["per_linear"]},
             "unfused_step": unfused,
-            "stages": {"quant_us_per_launch": quant_ms * 1e3, "quant_gbs": quant_bytes / (quant_ms / 1e3) / 1e9,
-                       "product_us_per_launch": prod_ms * 1e3,
-                       "fused_us_per_launch": None if fused_ms is None else fused_ms * 1e3,
-                       "pack_ms": pack_ms, "pack_gbs": [l.N * l.K * 4.25 / (ms / 1e3) / 1e9
-                                                        for l, ms in zip(lins, pack_ms)]},
-            "prefill": prefill,
+            "stages": {"pack_ms": packs.pack_ms,
+                       "pack_gbs": {k: int(k.split("x")[0]) * int(k.split("x")[1]) * 4.25 / (v / 1e3) / 1e9
+                                    for k, v in packs.pack_ms.items()}},
+            "configs": configs,
             "ffn_block": ffn_block,
             "decode_b3": decode_b3,
             "ste_backward": ste,
@@ -568,64 +763,74 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
         print(json.dumps(line), flush=True)
     if group:
         import torch.distributed as dist
-        del g_main, g_rem
         dist.destroy_process_group()
 
 
-def bench_b3(torch, bl, dev, stream, lins, xs, gains, peaks, peak_src, group, two_bit_step_ms):
+def bench_config(torch, bl, dev, stream, name, packs, peaks, peak_src, group, with_cpu, cpu_seconds) -> dict:
+    """One configuration of the benchmark set: its step time, value in its unit,
+    the roofline of its product kernel and the CPU oracle beside it."""
+    lins = synth.WORKLOADS[name]
+    unit = config_unit(lins, peaks)
+    big = any(l.M >= 256 for l in lins)
+    wl = Workload(torch, bl, dev, lins, packs, rotate=not big)
+    m = (measure_flushed if big else measure_rotating)(torch, bl, dev, stream, wl, peaks, peak_src, group)
+    sec = m["ms_per_step"] / 1e3
+    value = step_ops(lins) / sec / 1e12 if unit == "TOPS" else step_bytes(lins) / sec / 1e9
+    out = {"workload": name, "linears": [[l.M, l.K, l.N] for l in lins], "value": value, "unit": unit,
+           "us_per_step": m["ms_per_step"] * 1e3, "kernels_per_step": wl.kernels_per_step,
+           "path": "fused decode GEMV" if wl.fused else ("quant + GEMV" if all(l.M <= 8 for l in lins)
+                                                         else "quant + tcgen05 GEMM"), **m}
+    del wl
+    torch.cuda.empty_cache()
+    if with_cpu:
+        out["cpu_baseline"] = cpu_baseline(lins, unit, cpu_seconds)
+    return out
+
+
+def bench_b3(torch, bl, dev, stream, wl, peaks, group, two_bit_step_ms):
     """The decode step with base-3 packed weights (bitnet_bitlinear_gemv_b3, five codes per byte): same
-    linears, inputs, weight rotation and graphs as the 2-bit step; GB/s on the base-3 byte count."""
+    linears, inputs and weight rotation as the 2-bit step; GB/s on the base-3 byte count."""
+    lins = wl.lins
     packs = []
     for lin in lins:
-        W = torch.from_numpy(lin.make_w(0)).to(dev)
+        W = torch.from_numpy(weights_for(lin)).to(dev)
         P, G = bl.bitnet_pack_weights_b3(W, EPS_W)
         del W
-        packs.append(([P] + [P.clone() for _ in range(COPIES - 1)], G))
-    ys = [torch.empty((l.M, l.N), dtype=torch.bfloat16 if l.y_dtype == "bf16" else torch.float32, device=dev)
-          for l in lins]
+        packs.append(([P] + [P.clone() for _ in range(wl.copies - 1)], G))
+    ys = [torch.empty_like(b["y"]) for b in wl.bufs]
 
     def step(c):
         for i in range(len(lins)):
-            bl.bitnet_bitlinear_gemv_b3(xs[i], packs[i][0][c % COPIES], packs[i][1], gains[i], EPS_RMS, y=ys[i])
+            bl.bitnet_bitlinear_gemv_b3(wl.xs[i], packs[i][0][c % wl.copies], packs[i][1], wl.gains[i], EPS_RMS,
+                                        y=ys[i])
 
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        for c in range(GRAPH_STEPS):
-            step(c)
+    g = capture(torch, stream, step, GRAPH_STEPS)
     with torch.cuda.stream(stream):
-        for _ in range(3):
+        for _ in range(2):
             g.replay()
     torch.cuda.synchronize(dev)
-    reps = 40
-    barrier(group, dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(group, dev)
-    ms = max_over_ranks(e0.elapsed_time(e1), group, dev) / (reps * GRAPH_STEPS)
+    reps = 10
+    ms = replay_ms(torch, dev, stream, g, reps, group) / (reps * GRAPH_STEPS)
     b3_bytes = sum(l.N * bl.bitnet_b3_row_bytes(l.K) for l in lins)
-    step_bytes = b3_bytes + sum(linear_bytes(l)["x_in"] + 4 + linear_bytes(l)["y_out"] for l in lins)
-    gbs = step_bytes / (ms / 1e3) / 1e9
+    sb = b3_bytes + sum(linear_bytes(l)["x_in"] + 4 + linear_bytes(l)["y_out"] for l in lins)
+    gbs = sb / (ms / 1e3) / 1e9
+    del g, packs
     return {"us_per_step": ms * 1e3, "gbs": gbs, "frac": gbs / float(peaks["hbm_gbs"]),
             "weight_bytes_per_step": b3_bytes, "two_bit_us_per_step": two_bit_step_ms * 1e3,
             "device_status": bl.bitnet_get_device_status(),
-            "timing": f"CUDA graphs of {GRAPH_STEPS} steps over {COPIES} rotating weight copies, per step"}
+            "timing": f"CUDA graphs of {GRAPH_STEPS} steps over {wl.copies} rotating weight copies, per step"}
 
 
 def bench_ste(torch, bl, dev, stream, peaks, peak_src, group):
     """Straight-through-estimator backward GEMMs (tcgen05 kind::f16, bf16 operands, fp32 accumulation) at the
     prefill shapes, M = 4096 tokens: input gradient dX = gamma dY q and weight gradient dW = bf16(dY a)^T x_q,
     per-launch CUDA-event time with L2 flushed (256 MB write) before each launch."""
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     bf16_peak = float(peaks["bf16_tflops"])
     out, tot_flop, tot_ms = {}, 0, 0.0
     for lin in synth.WORKLOADS["prefill_m4096_2p5b_ffn"]:
         M, N, K = lin.M, lin.N, lin.K
-        W = torch.from_numpy(lin.make_w(0)).to(dev)
+        W = torch.from_numpy(weights_for(lin)).to(dev)
         P, G = bl.bitnet_pack_weights(W, EPS_W)
         del W
         x = torch.from_numpy(synth.f32_to_bf16_bits(lin.make_x(0)).view(np.int16).copy()).to(dev).view(torch.bfloat16)
@@ -640,13 +845,12 @@ def bench_ste(torch, bl, dev, stream, peaks, peak_src, group):
             tx, tw = [], []
             for it in range(13):
                 flush.zero_()
-                e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+                e0, e1, e2, e3 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
                 e0.record(stream)
                 bl.bitnet_ste_backward_input(P, G, dY, dX=dX, workspace=wsx)
                 e1.record(stream)
                 flush.zero_()
                 e2.record(stream)
-                e3 = torch.cuda.Event(enable_timing=True)
                 bl.bitnet_ste_backward_weight(dY, xq, a, dW=dW, workspace=ws)
                 e3.record(stream)
                 torch.cuda.synchronize(dev)
@@ -679,7 +883,7 @@ def bench_ffn_block(torch, bl, dev, stream, peaks, peak_src, group, name="ffn_bl
         W = torch.from_numpy(blk.make_w(which, 0)).to(dev)
         P[which] = bl.bitnet_pack_weights(W, EPS_W)
         del W
-    copies = max(2, int(2 * 126e6 // blk.weight_bytes) + 1)
+    copies = max(2, int(3 * L2_BYTES // blk.weight_bytes) + 1)
     cps = [[P[w][0]] + [P[w][0].clone() for _ in range(copies - 1)] for w in ("up", "gate", "down")]
     bf = lambda a: torch.from_numpy(synth.f32_to_bf16_bits(a).view(np.int16).copy()).to(dev).view(torch.bfloat16)
     x = bf(blk.make_x(0))
@@ -699,25 +903,13 @@ def bench_ffn_block(torch, bl, dev, stream, peaks, peak_src, group, name="ffn_bl
         bl.bitnet_bitlinear_gemv(x, cps[1][c % copies], G[1], gi, EPS_RMS, y=h)
         bl.bitnet_bitlinear_gemv(h, cps[2][c % copies], G[2], gs, EPS_RMS, y=y)
 
-    def timed(fn, per=64, reps=40):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for c in range(per):
-                fn(c)
+    def timed(fn, per=32, reps=10):
+        g = capture(torch, stream, fn, per)
         with torch.cuda.stream(stream):
-            for _ in range(3):
+            for _ in range(2):
                 g.replay()
         torch.cuda.synchronize(dev)
-        barrier(group, dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(reps):
-                g.replay()
-            e1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier(group, dev)
-        return max_over_ranks(e0.elapsed_time(e1), group, dev) / (per * reps)
+        return replay_ms(torch, dev, stream, g, reps, group) / (per * reps)
 
     ms = timed(ffn)
     ms3 = timed(three)
@@ -725,78 +917,36 @@ def bench_ffn_block(torch, bl, dev, stream, peaks, peak_src, group, name="ffn_bl
     nbytes = blk.weight_bytes + 2 * blk.M * blk.D + 2 * (blk.D + blk.F) + 12 + 2 * blk.M * blk.F + 2 * blk.M * blk.D
     gbs = nbytes / (ms / 1e3) / 1e9
     hbm = float(peaks["hbm_gbs"])
-    traffic = profiled_traffic(os.path.join(ROOT, "profiles", "ffn_block_m1_2p5b.md"),
+    traffic = profiled_traffic(os.path.join(PROFILES, f"{name}.md"),
                                kernel_source_hash(["ffn.cuh", "gemv.cuh", "quant.cuh", "ptx.cuh"]))
+    del cps, P
     return {"workload": name, "M": blk.M, "D": blk.D, "F": blk.F, "us_per_ffn": ms * 1e3, "gbs": gbs,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                          "traffic": traffic, "bytes_per_launch": nbytes,
                          "peak_source": f"{peak_src} hbm_gbs"},
             "three_fused_launches_us": ms3 * 1e3, "weight_copies": copies, "device_status": status,
-            "timing": "CUDA graphs of 64 launches over rotating weight copies, CUDA events, per launch"}
-
-
-def bench_prefill(torch, bl, dev, stream, peaks, peak_src, group):
-    """Tensor-core GEMM at M = 4096 (K = 2560 -> N = 6912 and K = 6912 -> N = 2560):
-    per-launch CUDA-event time with L2 flushed (256 MB write) before each launch."""
-    out = {}
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    int8_peak = float(peaks["bf16_tflops"]) * 2.0  # dense int8 = 2x dense bf16 (nominal 4.5 vs 2.25 PFLOP/s)
-    tot_ops, tot_ms = 0, 0.0
-    for lin in synth.WORKLOADS["prefill_m4096_2p5b_ffn"]:
-        W = torch.from_numpy(lin.make_w(0)).to(dev)
-        P, G = bl.bitnet_pack_weights(W, EPS_W)
-        del W
-        x = torch.from_numpy(synth.f32_to_bf16_bits(lin.make_x(0)).view(np.int16).copy()).to(dev).view(torch.bfloat16)
-        with torch.cuda.stream(stream):
-            xq, a, rs = bl.bitnet_quant_act(x, None, EPS_RMS, want_rowsum=True)
-            y = torch.empty((lin.M, lin.N), dtype=torch.bfloat16, device=dev)
-            times = []
-            qtimes = []
-            for it in range(13):
-                flush.zero_()
-                e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-                e0.record(stream)
-                bl.bitnet_quant_act(x, None, EPS_RMS, xq, a, rs)
-                e1.record(stream)
-                bl.bitnet_linear_gemm(P, G, xq, a, rs, y=y)
-                e2.record(stream)
-                torch.cuda.synchronize(dev)
-                if it >= 3:
-                    qtimes.append(e0.elapsed_time(e1))
-                    times.append(e1.elapsed_time(e2))
-        ms = max_over_ranks(statistics.median(times), group, dev)
-        qms = max_over_ranks(statistics.median(qtimes), group, dev)
-        tops = lin.ops / (ms / 1e3) / 1e12
-        qb = linear_bytes(lin)["quant"]
-        out[f"K{lin.K}_N{lin.N}"] = {"gemm_us": ms * 1e3, "tops": tops, "frac": tops / int8_peak,
-                                     "quant_us": qms * 1e3, "quant_gbs": qb / (qms / 1e3) / 1e9,
-                                     "quant_frac": qb / (qms / 1e3) / 1e9 / float(peaks["hbm_gbs"])}
-        tot_ops += lin.ops
-        tot_ms += ms
-    tops = tot_ops / (tot_ms / 1e3) / 1e12
-    return {"workload": "prefill_m4096_2p5b_ffn", "tops": tops, "unit": "TOPS",
-            "roofline": {"bound": "tensor", "achieved": tops, "peak": int8_peak, "unit": "TOP/s",
-                         "frac": tops / int8_peak,
-                         "peak_source": f"{peak_src} bf16_tflops x 2 (dense int8 / dense bf16 nominal ratio)"},
-            "per_shape": out, "timing": "median of 10 single launches, L2 flushed before each"}
+            "timing": "CUDA graphs of 32 launches over rotating weight copies, CUDA events, per launch"}
 
 
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=51200)
-    ap.add_argument("--warmup", type=int, default=1280)
+    ap.add_argument("--steps", type=int, default=2560)
+    ap.add_argument("--warmup", type=int, default=256)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
-    ap.add_argument("--no-prefill", action="store_true", help="skip the secondary prefill GEMM measurement")
-    ap.add_argument("--no-ffn", action="store_true", help="skip the secondary one-launch FFN block measurement")
-    ap.add_argument("--no-b3", action="store_true", help="skip the secondary base-3 decode measurement")
-    ap.add_argument("--no-ste", action="store_true", help="skip the secondary STE backward GEMM measurement")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU oracle time for the headline baseline")
+    ap.add_argument("--config-cpu-seconds", type=float, default=3.0, help="CPU oracle time per configuration")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baselines")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other configurations")
+    ap.add_argument("--no-ffn", action="store_true", help="skip the one-launch FFN block measurement")
+    ap.add_argument("--no-b3", action="store_true", help="skip the base-3 decode measurement")
+    ap.add_argument("--no-ste", action="store_true", help="skip the STE backward GEMM measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.steps < 1:
+        ap.error("--steps must be at least 1")
     ws, rank, local = dist_setup()
     lins = synth.WORKLOADS[args.workload]
     if args.impl == "reference":

@@ -1,0 +1,159 @@
+// Host side of bitnet_linear_gemm: the tcgen05 tensor-core product
+// (gemm.cuh): tensor maps, tile size by M, split-K choice, launch.
+#include "host_common.h"
+#include "gemm.cuh"
+
+namespace {
+
+using namespace bitnet;
+using namespace bitnet_host;
+
+// Launch configuration of a GEMM split over clusters of KS CTAs (KS = 1: plain persistent grid).
+template <int BN, int S, bool U8, int KS>
+cudaLaunchConfig_t gemm_config(int clusters, cudaStream_t s, cudaLaunchAttribute (&attr)[2]) {
+  using C = GemmCfg<BN, S, KS>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(clusters * KS);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = s;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = KS;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = KS > 1 ? 2 : 1;
+  return cfg;
+}
+
+// How many clusters of KS CTAs can be resident at once (clusters live inside
+// one GPC, so this is not simply SMs / KS).  Cached per device.
+template <int BN, int S, bool U8, int KS>
+int gemm_cluster_capacity() {
+  static std::atomic<int> cache[kMaxDevices] = {};
+  const int d = current_device();
+  if (d >= 0 && d < kMaxDevices && cache[d] > 0) return cache[d];
+  static std::atomic<bool> done[kMaxDevices] = {};
+  int n = 0;
+  if (set_smem(gemm_kernel<BN, S, U8, KS>, GemmCfg<BN, S, KS>::kSmemBytes, done) == cudaSuccess) {
+    if (KS == 1) {
+      n = sm_count();
+    } else {
+      cudaLaunchAttribute attr[2];
+      cudaLaunchConfig_t cfg = gemm_config<BN, S, U8, KS>(1, nullptr, attr);
+      if (cudaOccupancyMaxActiveClusters(&n, gemm_kernel<BN, S, U8, KS>, &cfg) != cudaSuccess) n = 0;
+    }
+  }
+  cudaGetLastError();
+  if (n <= 0) n = sm_count() / KS;
+  if (d >= 0 && d < kMaxDevices) cache[d] = n;
+  return n;
+}
+
+template <int BN, int S, bool U8, int KS>
+cudaError_t launch_gemm_ks(const CUtensorMap& mx, const CUtensorMap& mw, const float* gamma, const float* a,
+                           const int32_t* rs, int M, int N, int K, void* y, int yd, cudaStream_t s) {
+  using C = GemmCfg<BN, S, KS>;
+  static std::atomic<bool> done[kMaxDevices] = {};
+  const cudaError_t e = set_smem(gemm_kernel<BN, S, U8, KS>, C::kSmemBytes, done);
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = static_cast<int64_t>((N + kGemmBM - 1) / kGemmBM) * ((M + BN - 1) / BN);
+  const int cap = gemm_cluster_capacity<BN, S, U8, KS>();
+  const int clusters = static_cast<int>(tiles < cap ? tiles : cap);
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = gemm_config<BN, S, U8, KS>(clusters, s, attr);
+  return cudaLaunchKernelEx(&cfg, gemm_kernel<BN, S, U8, KS>, mx, mw, gamma, a, rs, M, N, K, y, yd);
+}
+
+// Split factor for a GEMM of `tiles` output tiles and nk K-steps: the one
+// that keeps the most SMs busy over the whole launch (tiles spread over
+// resident clusters in waves), with a small penalty per extra split for the
+// partial-sum exchange.  Only used with unsigned codes (row sums given).
+// Split factor for a GEMM of `tiles` output tiles and nk K-steps.  With two
+// or more waves of tiles per SM the plain persistent grid is used; with fewer
+// (decode-sized M) the factor in {1, 2, 4, 8} that keeps the most SMs busy
+// over the launch (tiles spread over the resident clusters in waves), with a
+// small penalty per extra split for the partial-sum exchange.  Only used with
+// unsigned codes (row sums given).
+template <int BN, int S>
+int choose_ksplit(int64_t tiles, int nk) {
+  const int sms = sm_count();
+  const int cap1 = gemm_cluster_capacity<BN, S, true, 1>();
+  if (tiles >= 2 * static_cast<int64_t>(cap1)) return 1;
+  const int ks[4] = {1, 2, 4, 8};
+  const int caps[4] = {cap1, gemm_cluster_capacity<BN, S, true, 2>(), gemm_cluster_capacity<BN, S, true, 4>(),
+                       gemm_cluster_capacity<BN, S, true, 8>()};
+  int best = 1;
+  double best_score = -1.0;
+  for (int i = 0; i < 4; ++i) {
+    const int k = ks[i];
+    if (k > nk) break;
+    const int64_t cl = tiles < caps[i] ? tiles : caps[i];
+    if (cl <= 0) continue;
+    const int64_t waves = (tiles + cl - 1) / cl;
+    const double busy = static_cast<double>(tiles) * k / (static_cast<double>(waves) * sms);
+    const double score = busy - 0.03 * (k - 1);
+    if (score > best_score + 1e-9) {
+      best_score = score;
+      best = k;
+    }
+  }
+  return best;
+}
+
+template <int BN, int S, bool U8>
+cudaError_t launch_gemm_t(const CUtensorMap& mx, const CUtensorMap& mw, const float* gamma, const float* a,
+                          const int32_t* rs, int M, int N, int K, void* y, int yd, cudaStream_t s) {
+  if constexpr (U8) {
+    const int64_t tiles = static_cast<int64_t>((N + kGemmBM - 1) / kGemmBM) * ((M + BN - 1) / BN);
+    const int nk = (K + kGemmBK - 1) / kGemmBK;
+    switch (choose_ksplit<BN, S>(tiles, nk)) {
+      case 2: return launch_gemm_ks<BN, S, U8, 2>(mx, mw, gamma, a, rs, M, N, K, y, yd, s);
+      case 4: return launch_gemm_ks<BN, S, U8, 4>(mx, mw, gamma, a, rs, M, N, K, y, yd, s);
+      case 8: return launch_gemm_ks<BN, S, U8, 8>(mx, mw, gamma, a, rs, M, N, K, y, yd, s);
+      default: break;
+    }
+  }
+  return launch_gemm_ks<BN, S, U8, 1>(mx, mw, gamma, a, rs, M, N, K, y, yd, s);
+}
+
+template <int BN, int S>
+cudaError_t launch_gemm_bn(const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
+                           const int32_t* rs, int M, void* y, int yd, cudaStream_t s) {
+  CUtensorMap mx, mw;
+  // activations: 128-byte-wide boxes (two per stage); packed codes: one
+  // 64-byte-wide box of 128 rows per stage
+  if (!make_map_u8(&mx, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(K), 128, BN,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!make_map_u8(&mw, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4),
+                   kGemmBK / 4, kGemmBM, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  if (rs != nullptr) return launch_gemm_t<BN, S, true>(mx, mw, gamma, a, rs, M, N, K, y, yd, s);
+  return launch_gemm_t<BN, S, false>(mx, mw, gamma, a, rs, M, N, K, y, yd, s);
+}
+
+}  // namespace
+
+BITNET_DEFINE_TAKE_ERROR(gemm)
+
+extern "C" {
+
+bitnet_status bitnet_linear_gemm(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, const int8_t* x_q,
+                                 const float* a_scale, const int32_t* x_rowsum, int64_t M, void* y, int y_dtype,
+                                 void* stream) {
+  const bitnet_status st = check_linear(W_packed, gamma, N, K, x_q, a_scale, x_rowsum, M, y, y_dtype);
+  if (st != BITNET_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int n = static_cast<int>(N), k = static_cast<int>(K), m = static_cast<int>(M);
+  cudaError_t e;
+  if (m <= 16) e = launch_gemm_bn<16, 6>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
+  else if (m <= 32) e = launch_gemm_bn<32, 6>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
+  else if (m <= 64) e = launch_gemm_bn<64, 6>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
+  else e = launch_gemm_bn<128, 4>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
+  return from_cuda(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,134 @@
+// Host side of the decode products on CUDA cores: bitnet_linear_gemv and the
+// fused decode BitLinear bitnet_bitlinear_gemv (gemv.cuh).
+#include "host_common.h"
+#include "gemv.cuh"
+
+namespace {
+
+using namespace bitnet;
+using namespace bitnet_host;
+
+template <int MT, bool U8, bool XS>
+cudaError_t launch_gemv_x(const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
+                          const int32_t* rs, void* y, int yd, cudaStream_t s) {
+  static std::atomic<bool> done[kMaxDevices] = {};
+  const cudaError_t e = set_smem(gemv_kernel<MT, U8, XS>, gemv_smem_bytes(MT, kGemvXMaxBytes / MT, XS), done);
+  if (e != cudaSuccess) return e;
+  const int64_t groups = (N + kGemvRows - 1) / kGemvRows;
+  const int grid = static_cast<int>(groups < sm_count() ? groups : sm_count());
+  return launch_pdl(gemv_kernel<MT, U8, XS>, dim3(grid), dim3(kGemvThreads), gemv_smem_bytes(MT, K, XS), s, Wp, gamma,
+                    N, K, xq, a, rs, static_cast<const float*>(nullptr), static_cast<const float*>(nullptr), 0.0f, y,
+                    yd);
+}
+
+template <int MT, bool U8>
+cudaError_t launch_gemv_t(const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
+                          const int32_t* rs, void* y, int yd, cudaStream_t s) {
+  if (static_cast<int64_t>(MT) * K <= kGemvXMaxBytes)
+    return launch_gemv_x<MT, U8, true>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+  return launch_gemv_x<MT, U8, false>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+}
+
+template <bool U8>
+cudaError_t launch_gemv_u(int M, const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
+                          const int32_t* rs, void* y, int yd, cudaStream_t s) {
+  switch (M) {
+    case 1: return launch_gemv_t<1, U8>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+    case 2: return launch_gemv_t<2, U8>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+    case 3: return launch_gemv_t<3, U8>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+    case 4: return launch_gemv_t<4, U8>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+    case 5: return launch_gemv_t<5, U8>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+    case 6: return launch_gemv_t<6, U8>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+    case 7: return launch_gemv_t<7, U8>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+    case 8: return launch_gemv_t<8, U8>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// Fused decode BitLinear: quantisation (and RMSNorm) of M <= 8 token rows in
+// every CTA's prologue, then the GEMV.
+template <int MT, typename T, int MAXC>
+cudaError_t launch_fused_t(const void* x, const void* gain, float eps, const uint8_t* Wp, const float* gamma, int N,
+                           int K, void* y, int yd, cudaStream_t s) {
+  static std::atomic<bool> done[kMaxDevices] = {};
+  auto kern = gemv_kernel<MT, true, true, true, T, MAXC>;
+  const cudaError_t e = set_smem(kern, gemv_smem_bytes(MT, kGemvXMaxBytes / MT, true), done);
+  if (e != cudaSuccess) return e;
+  const int64_t groups = (N + kGemvRows - 1) / kGemvRows;
+  const int grid = static_cast<int>(groups < sm_count() ? groups : sm_count());
+  return launch_pdl(kern, dim3(grid), dim3(kGemvThreads), gemv_smem_bytes(MT, K, true), s, Wp, gamma, N, K,
+                    static_cast<const int8_t*>(nullptr), static_cast<const float*>(nullptr),
+                    static_cast<const int32_t*>(nullptr), static_cast<const T*>(x), static_cast<const T*>(gain), eps, y,
+                    yd);
+}
+
+template <int MT, typename T>
+cudaError_t launch_fused_c(const void* x, const void* gain, float eps, const uint8_t* Wp, const float* gamma, int N,
+                           int K, void* y, int yd, cudaStream_t s) {
+  const int per_thread = (K / 8 + kQuantThreads - 1) / kQuantThreads;
+  if (per_thread <= 1) return launch_fused_t<MT, T, 1>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+  if (per_thread <= 2) return launch_fused_t<MT, T, 2>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+  if (per_thread <= 4) return launch_fused_t<MT, T, 4>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+  if (per_thread <= 8) return launch_fused_t<MT, T, 8>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+  if constexpr (sizeof(T) == 2) return launch_fused_t<MT, T, 16>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+  return cudaErrorInvalidValue;
+}
+
+template <typename T>
+cudaError_t launch_fused(int M, const void* x, const void* gain, float eps, const uint8_t* Wp, const float* gamma,
+                         int N, int K, void* y, int yd, cudaStream_t s) {
+  switch (M) {
+    case 1: return launch_fused_c<1, T>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+    case 2: return launch_fused_c<2, T>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+    case 3: return launch_fused_c<3, T>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+    case 4: return launch_fused_c<4, T>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+    case 5: return launch_fused_c<5, T>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+    case 6: return launch_fused_c<6, T>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+    case 7: return launch_fused_c<7, T>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+    case 8: return launch_fused_c<8, T>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+BITNET_DEFINE_TAKE_ERROR(gemv)
+
+extern "C" {
+
+bitnet_status bitnet_linear_gemv(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, const int8_t* x_q,
+                                 const float* a_scale, const int32_t* x_rowsum, int64_t M, void* y, int y_dtype,
+                                 void* stream) {
+  const bitnet_status st = check_linear(W_packed, gamma, N, K, x_q, a_scale, x_rowsum, M, y, y_dtype);
+  if (st != BITNET_OK) return st;
+  if (M > 8) return BITNET_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int n = static_cast<int>(N), k = static_cast<int>(K), m = static_cast<int>(M);
+  const cudaError_t e = x_rowsum != nullptr
+                            ? launch_gemv_u<true>(m, W_packed, gamma, n, k, x_q, a_scale, x_rowsum, y, y_dtype, s)
+                            : launch_gemv_u<false>(m, W_packed, gamma, n, k, x_q, a_scale, x_rowsum, y, y_dtype, s);
+  return from_cuda(e);
+}
+
+bitnet_status bitnet_bitlinear_gemv(const void* x, int x_dtype, const void* rms_gain, float rms_eps,
+                                    const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, int64_t M,
+                                    void* y, int y_dtype, void* stream) {
+  if (x == nullptr || W_packed == nullptr || gamma == nullptr || y == nullptr) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(rms_gain, 16) || !aligned(W_packed, 16) || !aligned(y, 16) || !aligned(gamma, 4))
+    return BITNET_ERR_INVALID_ARG;
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
+  if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16 && y_dtype != BITNET_I32) return BITNET_ERR_INVALID_ARG;
+  if (rms_gain != nullptr && (!std::isfinite(rms_eps) || !(rms_eps > 0.0f))) return BITNET_ERR_INVALID_ARG;
+  const int64_t kmax = x_dtype == BITNET_BF16 ? 32768 : 16384;
+  if (!valid_k(K) || K > kmax || N < 1 || N > INT32_MAX || M < 1 || M > 8 || M * K > kGemvXMaxBytes)
+    return BITNET_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int n = static_cast<int>(N), k = static_cast<int>(K), m = static_cast<int>(M);
+  const cudaError_t e =
+      x_dtype == BITNET_BF16
+          ? launch_fused<__nv_bfloat16>(m, x, rms_gain, rms_eps, W_packed, gamma, n, k, y, y_dtype, s)
+          : launch_fused<float>(m, x, rms_gain, rms_eps, W_packed, gamma, n, k, y, y_dtype, s);
+  return from_cuda(e);
+}
+
+}  // extern "C"

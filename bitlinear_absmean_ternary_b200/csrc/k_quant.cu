@@ -1,0 +1,104 @@
+// Host side of bitnet_quant_act: per-token absmax int8 quantisation with the
+// optional fused RMSNorm (quant.cuh: a CTA per row; quant_rows.cuh: a warp
+// per row for many bf16 rows).
+#include "host_common.h"
+#include "quant.cuh"
+#include "quant_rows.cuh"
+
+namespace {
+
+using namespace bitnet;
+using namespace bitnet_host;
+
+template <typename T, int MAXC, int NTHR = kQuantThreads>
+cudaError_t launch_quant_t(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
+                           int32_t* rs, cudaStream_t s, int threads = kQuantThreads) {
+  static std::atomic<bool> done[kMaxDevices] = {};
+  const cudaError_t e = set_smem(quant_act_kernel<T, MAXC, NTHR>, 0, done);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(quant_act_kernel<T, MAXC, NTHR>, dim3(static_cast<unsigned>(M)), dim3(threads), 0, s,
+                    static_cast<const T*>(x), K, static_cast<const T*>(gain), eps, xq, a, rs);
+}
+
+template <int MAXC, bool NORM>
+cudaError_t launch_quant_rows_t(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
+                                int32_t* rs, cudaStream_t s) {
+  static std::atomic<bool> done[kMaxDevices] = {};
+  const cudaError_t e = set_smem(quant_rows_kernel<MAXC, NORM>, 0, done);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = (M + kQuantRowsWarps - 1) / kQuantRowsWarps;
+  return launch_pdl(quant_rows_kernel<MAXC, NORM>, dim3(static_cast<unsigned>(grid)), dim3(kQuantRowsThreads), 0, s,
+                    static_cast<const __nv_bfloat16*>(x), M, K, static_cast<const __nv_bfloat16*>(gain), eps, xq, a,
+                    rs);
+}
+
+template <bool NORM>
+cudaError_t launch_quant_rows(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
+                              int32_t* rs, cudaStream_t s) {
+  const int per_lane = (K / 8 + 31) / 32;
+#define BN_QROWS(C) \
+  if (per_lane <= C) return launch_quant_rows_t<C, NORM>(x, M, K, gain, eps, xq, a, rs, s);
+  BN_QROWS(2) BN_QROWS(4) BN_QROWS(6) BN_QROWS(8) BN_QROWS(10) BN_QROWS(12) BN_QROWS(16) BN_QROWS(20)
+  BN_QROWS(24)
+#undef BN_QROWS
+  return cudaErrorInvalidValue;
+}
+
+// Token count from which the warp-per-row kernel takes over (bf16 input,
+// K <= 6144): from there on it keeps more rows in flight per SM; below, a CTA
+// per row spreads a short batch over more SMs.
+constexpr int64_t kQuantRowsMinM = 512;
+
+template <typename T>
+cudaError_t launch_quant(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
+                         int32_t* rs, cudaStream_t s) {
+  if constexpr (sizeof(T) == 2) {
+    if (M >= kQuantRowsMinM && K <= 32 * 8 * kQuantRowsMaxChunks)
+      return gain != nullptr ? launch_quant_rows<true>(x, M, K, gain, eps, xq, a, rs, s)
+                             : launch_quant_rows<false>(x, M, K, gain, eps, xq, a, rs, s);
+  }
+  const int per_thread = (K / 8 + kQuantThreads - 1) / kQuantThreads;
+  if (gain == nullptr) {
+    // No norm, so no fixed order: the fewest whole warps (at most 256 threads)
+    // that give every thread the same number of 8-element chunks.
+    const int mc = per_thread <= 1 ? 1 : per_thread <= 2 ? 2 : per_thread <= 4 ? 4 : per_thread <= 8 ? 8 : 16;
+    const int threads = ((K / 8 + mc - 1) / mc + 31) / 32 * 32;
+    if (mc == 1) return launch_quant_t<T, 1>(x, M, K, gain, eps, xq, a, rs, s, threads);
+    if (mc == 2) return launch_quant_t<T, 2>(x, M, K, gain, eps, xq, a, rs, s, threads);
+    if (mc == 4) return launch_quant_t<T, 4>(x, M, K, gain, eps, xq, a, rs, s, threads);
+    if (mc == 8) return launch_quant_t<T, 8>(x, M, K, gain, eps, xq, a, rs, s, threads);
+    if constexpr (sizeof(T) == 2) return launch_quant_t<T, 16>(x, M, K, gain, eps, xq, a, rs, s, threads);
+    return cudaErrorInvalidValue;
+  }
+  if (per_thread <= 1) return launch_quant_t<T, 1>(x, M, K, gain, eps, xq, a, rs, s);
+  if (per_thread <= 2) return launch_quant_t<T, 2>(x, M, K, gain, eps, xq, a, rs, s);
+  if (per_thread <= 4) return launch_quant_t<T, 4>(x, M, K, gain, eps, xq, a, rs, s);
+  if (per_thread <= 8) return launch_quant_t<T, 8>(x, M, K, gain, eps, xq, a, rs, s);
+  if constexpr (sizeof(T) == 2) return launch_quant_t<T, 16>(x, M, K, gain, eps, xq, a, rs, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+BITNET_DEFINE_TAKE_ERROR(quant)
+
+extern "C" {
+
+bitnet_status bitnet_quant_act(const void* x, int x_dtype, int64_t M, int64_t K, const void* rms_gain, float rms_eps,
+                               int8_t* x_q, float* a_scale, int32_t* x_rowsum, void* stream) {
+  if (x == nullptr || x_q == nullptr || a_scale == nullptr) return BITNET_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(x_q, 16) || !aligned(rms_gain, 16) || !aligned(a_scale, 4) || !aligned(x_rowsum, 4))
+    return BITNET_ERR_INVALID_ARG;
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_INVALID_ARG;
+  if (rms_gain != nullptr && (!std::isfinite(rms_eps) || !(rms_eps > 0.0f))) return BITNET_ERR_INVALID_ARG;
+  const int64_t kmax = x_dtype == BITNET_BF16 ? 32768 : 16384;
+  if (!valid_k(K) || K > kmax || M < 1 || M > INT32_MAX) return BITNET_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t e =
+      x_dtype == BITNET_BF16
+          ? launch_quant<__nv_bfloat16>(x, M, static_cast<int>(K), rms_gain, rms_eps, x_q, a_scale, x_rowsum, s)
+          : launch_quant<float>(x, M, static_cast<int>(K), rms_gain, rms_eps, x_q, a_scale, x_rowsum, s);
+  return from_cuda(e);
+}
+
+}  // extern "C"

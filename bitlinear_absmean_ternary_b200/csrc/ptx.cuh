@@ -10,9 +10,10 @@
 
 namespace bitnet {
 
-// Device-wide error word: set when a bounded wait gives up.  Read and cleared
-// by bitnet_get_device_status.
-__device__ unsigned int g_device_error;
+// Device-wide error word: set when a bounded wait gives up.  Each translation
+// unit of the library has its own copy (internal linkage); bitnet_get_device_status
+// reads and clears all of them.
+static __device__ unsigned int g_device_error;
 
 constexpr unsigned int kErrTimeout = 1u;
 // A wait on a barrier gives up after this many nanoseconds of %globaltimer.
