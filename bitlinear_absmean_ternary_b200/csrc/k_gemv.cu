@@ -8,17 +8,61 @@ namespace {
 using namespace bitnet;
 using namespace bitnet_host;
 
+// Launch plan of gemv_kernel (grid, K-chunk, ring depth, shared memory).
+//
+// A CTA whose share of W is small (the 2.5B-class decode shapes, about
+// 30 KB per SM) has all of it in flight from the start with the default
+// ring, and its few rows are cut into chunks of at most 2560 weights so
+// that they spread over all 16 warps.  A large share (the 27B-class shapes,
+// about 195 KB per SM) is streamed with long chunks through a deep ring, so
+// that each SM keeps tens of KB of weights in flight with few, large bulk
+// copies.  The thresholds are compile-time constants (a tuning build may
+// define them).
+#ifndef BITNET_GEMV_SMALL_SHARE
+#define BITNET_GEMV_SMALL_SHARE (64 * 1024)
+#endif
+#ifndef BITNET_GEMV_BIG_CHUNK
+#define BITNET_GEMV_BIG_CHUNK 2688
+#endif
+#ifndef BITNET_GEMV_BIG_RING
+#define BITNET_GEMV_BIG_RING (86 * 1024)
+#endif
+constexpr int kGemvSmemMax = 232448 - 2048;  // 227 KB less the fused kernel's static scratch
+
+struct GemvPlan {
+  int grid, kchunk, nslots, smem;
+};
+
+GemvPlan gemv_plan(int mt, int N, int K, bool xs) {
+  GemvPlan p;
+  const int64_t groups = (N + kGemvRows - 1) / kGemvRows;
+  p.grid = static_cast<int>(groups < sm_count() ? groups : sm_count());
+  const int64_t rows = (N + p.grid - 1) / p.grid;
+  const int64_t share = rows * (K / 4);
+  if (share <= BITNET_GEMV_SMALL_SHARE) {
+    p.kchunk = gemv_kchunk(K);
+    p.nslots = kGemvSlots;
+  } else {
+    p.kchunk = gemv_kchunk_max(K, BITNET_GEMV_BIG_CHUNK);
+    const int per_warp = BITNET_GEMV_BIG_RING / (kGemvWarps * p.kchunk);
+    p.nslots = per_warp < 2 ? 2 : (per_warp > kGemvMaxSlots ? kGemvMaxSlots : per_warp);
+  }
+  while (p.nslots > 1 && gemv_plan_smem_bytes(mt, K, xs, p.kchunk, p.nslots) > kGemvSmemMax) --p.nslots;
+  p.smem = gemv_plan_smem_bytes(mt, K, xs, p.kchunk, p.nslots);
+  return p;
+}
+
 template <int MT, bool U8, bool XS>
 cudaError_t launch_gemv_x(const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
                           const int32_t* rs, void* y, int yd, cudaStream_t s) {
   static std::atomic<bool> done[kMaxDevices] = {};
-  const cudaError_t e = set_smem(gemv_kernel<MT, U8, XS>, gemv_smem_bytes(MT, kGemvXMaxBytes / MT, XS), done);
+  const cudaError_t e = set_smem(gemv_kernel<MT, U8, XS>, kGemvSmemMax, done);
   if (e != cudaSuccess) return e;
-  const int64_t groups = (N + kGemvRows - 1) / kGemvRows;
-  const int grid = static_cast<int>(groups < sm_count() ? groups : sm_count());
-  return launch_pdl(gemv_kernel<MT, U8, XS>, dim3(grid), dim3(kGemvThreads), gemv_smem_bytes(MT, K, XS), s, Wp, gamma,
-                    N, K, xq, a, rs, static_cast<const float*>(nullptr), static_cast<const float*>(nullptr), 0.0f, y,
-                    yd);
+  const GemvPlan p = gemv_plan(MT, N, K, XS);
+  if (p.smem > kGemvSmemMax) return cudaErrorInvalidValue;
+  return launch_pdl(gemv_kernel<MT, U8, XS>, dim3(p.grid), dim3(kGemvThreads), p.smem, s, Wp, gamma, N, K, xq, a, rs,
+                    static_cast<const float*>(nullptr), static_cast<const float*>(nullptr), 0.0f, y, yd, p.kchunk,
+                    p.nslots);
 }
 
 template <int MT, bool U8>
@@ -52,14 +96,14 @@ cudaError_t launch_fused_t(const void* x, const void* gain, float eps, const uin
                            int K, void* y, int yd, cudaStream_t s) {
   static std::atomic<bool> done[kMaxDevices] = {};
   auto kern = gemv_kernel<MT, true, true, true, T, MAXC>;
-  const cudaError_t e = set_smem(kern, gemv_smem_bytes(MT, kGemvXMaxBytes / MT, true), done);
+  const cudaError_t e = set_smem(kern, kGemvSmemMax, done);
   if (e != cudaSuccess) return e;
-  const int64_t groups = (N + kGemvRows - 1) / kGemvRows;
-  const int grid = static_cast<int>(groups < sm_count() ? groups : sm_count());
-  return launch_pdl(kern, dim3(grid), dim3(kGemvThreads), gemv_smem_bytes(MT, K, true), s, Wp, gamma, N, K,
+  const GemvPlan p = gemv_plan(MT, N, K, true);
+  if (p.smem > kGemvSmemMax) return cudaErrorInvalidValue;
+  return launch_pdl(kern, dim3(p.grid), dim3(kGemvThreads), p.smem, s, Wp, gamma, N, K,
                     static_cast<const int8_t*>(nullptr), static_cast<const float*>(nullptr),
                     static_cast<const int32_t*>(nullptr), static_cast<const T*>(x), static_cast<const T*>(gain), eps, y,
-                    yd);
+                    yd, p.kchunk, p.nslots);
 }
 
 template <int MT, typename T>

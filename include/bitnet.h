@@ -24,6 +24,20 @@
  *   - Every pointer must be 16-byte aligned.
  *   - Errors are returned as bitnet_status; nothing is launched when an
  *     argument is rejected.  No C++ exception crosses this boundary.
+ *   - The product entry points (bitnet_linear_gemv, bitnet_linear_gemm,
+ *     bitnet_bitlinear_gemv, bitnet_bitlinear_ffn_gemv,
+ *     bitnet_bitlinear_gemv_b3) are launched with programmatic dependent
+ *     launch: they start while the previous kernel on the stream finishes,
+ *     and request their first packed-weight tiles BEFORE waiting for it
+ *     (the weights of a layer never depend on the layer before).  So the
+ *     kernel launched immediately before one of them on the same stream must
+ *     not write the packed weights it reads.  Any kernel between the writer
+ *     and the product call, a synchronisation, or an event wait restores the
+ *     ordering; a kernel that writes the weights and does not signal early
+ *     completion (cudaTriggerProgrammaticLaunchCompletion) is also safe in
+ *     practice, and the tests check a torch copy followed directly by the
+ *     decode entry points.  Activations, scales and outputs are only touched
+ *     after the wait.
  *
  * Packed weight layout (2 bits per weight; the pages say only that the three
  * states are stored on two bits plus some structure -- inferownia.pl,
@@ -107,6 +121,9 @@ bitnet_status bitnet_pack_weights(const float* W, int64_t N, int64_t K, float ep
  *   - All calls share the array and it keeps the previous call's contents;
  *     the call clears what must start at zero.  Calls that overlap on the GPU
  *     (for example from two host threads on two streams) race on it.
+ *   - The looked-up address is kept for the life of the process, so the
+ *     library must not be used on a device after cudaDeviceReset of that
+ *     device (the array's address belongs to the destroyed context).
  * Synchronises `stream`.
  */
 #define BITNET_PACK_NOALLOC_MAX_ROWS 65536

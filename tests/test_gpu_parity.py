@@ -246,7 +246,9 @@ def _check_linear(dev, orc, fn, M, N, K, seed=0, zero_row=None, zero_tok=None, s
 
 
 GEMV_CASES = [(1, 256, 256), (4, 256, 256), (8, 6912, 2560), (1, 2560, 6912), (3, 129, 192), (5, 1, 64),
-              (2, 37, 4160), (7, 300, 640), (1, 1000, 21504), (6, 77, 8192)]
+              (2, 37, 4160), (7, 300, 640), (1, 1000, 21504), (6, 77, 8192),
+              # 27B-class shapes: the deep-ring launch plan (long chunks, several slots per warp)
+              (1, 21504, 5376), (3, 21504, 5376), (2, 5376, 21504), (1, 5373, 21504)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMV_CASES)
@@ -294,6 +296,9 @@ FUSED_CASES = [
     (8, 300, 2688, "bf16", True, "i32"),
     (3, 129, 64, "f32", True, "bf16"),
     (2, 1000, 4096, "bf16", False, "bf16"),
+    (1, 21504, 5376, "bf16", False, "bf16"),   # 27B up: deep-ring plan, one token (masked fields)
+    (2, 5376, 10752, "bf16", True, "f32"),     # deep-ring plan with two tokens
+    (1, 21501, 5376, "bf16", True, "i32"),     # ragged last group of the last CTA
 ]
 
 
@@ -391,3 +396,34 @@ def test_repeatable_and_status_clean(dev, orc):
         for u, v in zip(outs[0], o):
             assert torch.equal(u, v)
     assert bl.bitnet_get_device_status() == bl.BITNET_OK
+
+
+def test_gemv_after_a_kernel_that_writes_the_weights(dev, orc):
+    """The decode kernels request their first weight tiles before waiting on
+    the previous kernel (programmatic dependent launch).  A torch kernel that
+    writes W_packed just before them on the same stream (here a copy from a
+    second buffer) does not signal early completion, so the kernels still see
+    the new weights: checked against the oracle for both decode entry points."""
+    import torch
+    N, K = 21504, 5376
+    rng = np.random.default_rng(3)
+    q = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    packed = orc.pack_codes(q)
+    x = synth.activations(1, K, 4, 2, "normal", 0.01, 20.0, "bf16")
+    xq_r, a_r, _ = orc.quant_act(x)
+    gamma = np.float32(0.0125)
+    _, y_r = orc.bitlinear(packed, gamma, K, xq_r, a_r)
+    src = _t(packed, dev)
+    G = _t(np.array([gamma], np.float32), dev)
+    xd = _x_dev(x, "bf16", dev)
+    xq, a, rs = bl.bitnet_quant_act(xd, want_rowsum=True)
+    for trial in range(3):
+        P = torch.zeros_like(src)
+        torch.cuda.synchronize()
+        P.copy_(src)                      # writes W_packed on the current stream ...
+        y1 = bl.bitnet_bitlinear_gemv(xd, P, G, out_dtype=torch.float32)   # ... read right after
+        P2 = torch.zeros_like(src)
+        P2.copy_(src)
+        y2 = bl.bitnet_linear_gemv(P2, G, xq, a, rs, out_dtype=torch.float32)
+        assert ulp_diff_f32(y1.cpu().numpy(), y_r).max() == 0
+        assert ulp_diff_f32(y2.cpu().numpy(), y_r).max() == 0
