@@ -404,11 +404,15 @@ class Workload:
                 "a": torch.empty(lin.M, dtype=torch.float32, device=dev),
                 "rs": torch.empty(lin.M, dtype=torch.int32, device=dev),
                 "y": torch.empty((lin.M, lin.N), dtype=ydt, device=dev)})
+        # one GEMM workspace for the whole step (its calls run one after another on one stream)
+        wsb = max([bl.bitnet_linear_gemm_workspace_bytes(l.M, l.N, l.K) for l in lins if l.M > 8] or [0])
+        self.ws = torch.zeros(wsb, dtype=torch.uint8, device=dev) if wsb else None
         self.fused = all(l.M <= 8 and l.M * l.K <= 21504 for l in lins)
         self.kernels_per_step = (1 if self.fused else 2) * len(lins)
         self.product_kernel = ("gemv_kernel (fused quantisation + GEMV, bitnet_bitlinear_gemv)" if self.fused else
                                "gemv_kernel (bitnet_linear_gemv)" if all(l.M <= 8 for l in lins) else
-                               "gemm_kernel (tcgen05, bitnet_linear_gemm)")
+                               "gemm_sk_kernel (tcgen05 stream-K, bitnet_linear_gemm)" if all(l.M <= 64 for l in lins)
+                               else "gemm_kernel (tcgen05, bitnet_linear_gemm)")
 
     def _act(self, a, dtype):
         torch = self.torch
@@ -422,8 +426,12 @@ class Workload:
 
     def product(self, i, c):
         lin, b = self.lins[i], self.bufs[i]
-        fn = self.bl.bitnet_linear_gemv if lin.M <= 8 else self.bl.bitnet_linear_gemm
-        fn(self.packs[i][0][c % self.copies], self.packs[i][1], b["xq"], b["a"], b["rs"], y=b["y"])
+        if lin.M <= 8:
+            self.bl.bitnet_linear_gemv(self.packs[i][0][c % self.copies], self.packs[i][1], b["xq"], b["a"],
+                                       b["rs"], y=b["y"])
+        else:
+            self.bl.bitnet_linear_gemm(self.packs[i][0][c % self.copies], self.packs[i][1], b["xq"], b["a"],
+                                       b["rs"], y=b["y"], workspace=self.ws)
 
     def fused_linear(self, i, c):
         self.bl.bitnet_bitlinear_gemv(self.xs[i], self.packs[i][0][c % self.copies], self.packs[i][1],

@@ -54,10 +54,12 @@ def lib() -> ctypes.CDLL:
         L.bitnet_pack_weights.restype = I
         L.bitnet_quant_act.argtypes = [P, I, I64, I64, P, F, P, P, P, P]
         L.bitnet_quant_act.restype = I
-        for name in ("bitnet_linear_gemv", "bitnet_linear_gemm"):
-            fn = getattr(L, name)
-            fn.argtypes = [P, P, I64, I64, P, P, P, I64, P, I, P]
-            fn.restype = I
+        L.bitnet_linear_gemv.argtypes = [P, P, I64, I64, P, P, P, I64, P, I, P]
+        L.bitnet_linear_gemv.restype = I
+        L.bitnet_linear_gemm.argtypes = [P, P, I64, I64, P, P, P, I64, P, I, P, ctypes.c_size_t, P]
+        L.bitnet_linear_gemm.restype = I
+        L.bitnet_linear_gemm_workspace_bytes.argtypes = [I64, I64, I64]
+        L.bitnet_linear_gemm_workspace_bytes.restype = ctypes.c_size_t
         L.bitnet_bitlinear_gemv.argtypes = [P, I, P, F, P, P, I64, I64, I64, P, I, P]
         L.bitnet_bitlinear_gemv.restype = I
         L.bitnet_bitlinear_ffn_gemv.argtypes = [P, I, I64, I64, I64, P, F, P, P, P, P, P, F, P, P, P, P, I, P, P]
@@ -213,7 +215,7 @@ def bitnet_quant_act(x, rms_gain=None, rms_eps: float = 1e-5, x_q=None, a_scale=
     return x_q, a_scale, x_rowsum
 
 
-def _linear(name: str, W_packed, gamma, x_q, a_scale, x_rowsum=None, y=None, out_dtype=None):
+def _linear_args(W_packed, gamma, x_q, a_scale, x_rowsum, y, out_dtype):
     torch = _torch()
     _need_cuda(W_packed, gamma, x_q, a_scale, x_rowsum, y)
     N = W_packed.shape[0]
@@ -223,20 +225,45 @@ def _linear(name: str, W_packed, gamma, x_q, a_scale, x_rowsum=None, y=None, out
         raise ValueError("x_q and W_packed disagree on K")
     if y is None:
         y = torch.empty((M, N), dtype=out_dtype or torch.bfloat16, device=x_q.device)
-    st = getattr(lib(), name)(_ptr(W_packed), _ptr(gamma), N, K, _ptr(x_q), _ptr(a_scale), _ptr(x_rowsum), M,
-                              _ptr(y), _dtype_code(y.dtype), _stream(x_q.device))
-    _check(name, st)
-    return y
+    return M, N, K, y
 
 
 def bitnet_linear_gemv(W_packed, gamma, x_q, a_scale, x_rowsum=None, y=None, out_dtype=None):
     """W1.58A8 product for M <= 8 tokens (CUDA cores).  Returns y (M x N)."""
-    return _linear("bitnet_linear_gemv", W_packed, gamma, x_q, a_scale, x_rowsum, y, out_dtype)
+    M, N, K, y = _linear_args(W_packed, gamma, x_q, a_scale, x_rowsum, y, out_dtype)
+    st = lib().bitnet_linear_gemv(_ptr(W_packed), _ptr(gamma), N, K, _ptr(x_q), _ptr(a_scale), _ptr(x_rowsum), M,
+                                  _ptr(y), _dtype_code(y.dtype), _stream(x_q.device))
+    _check("bitnet_linear_gemv", st)
+    return y
 
 
-def bitnet_linear_gemm(W_packed, gamma, x_q, a_scale, x_rowsum=None, y=None, out_dtype=None):
-    """W1.58A8 product for any M (tcgen05 tensor cores).  Returns y (M x N)."""
-    return _linear("bitnet_linear_gemm", W_packed, gamma, x_q, a_scale, x_rowsum, y, out_dtype)
+def bitnet_linear_gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    """Workspace bytes of bitnet_linear_gemm on the current device (0 when none is used)."""
+    return int(lib().bitnet_linear_gemm_workspace_bytes(M, N, K))
+
+
+def bitnet_linear_gemm(W_packed, gamma, x_q, a_scale, x_rowsum=None, y=None, out_dtype=None, workspace=None,
+                       stream_k: bool = True):
+    """W1.58A8 product for any M (tcgen05 tensor cores).  Returns y (M x N).
+
+    workspace: a zeroed uint8 device tensor of bitnet_linear_gemm_workspace_bytes
+    bytes, reused across calls on one stream (the calls leave it zeroed), or None
+    to allocate a zeroed one for this call when M <= 64.  stream_k=False passes
+    no workspace (the persistent-tile path; same results)."""
+    torch = _torch()
+    M, N, K, y = _linear_args(W_packed, gamma, x_q, a_scale, x_rowsum, y, out_dtype)
+    if not stream_k:
+        workspace = None
+    elif workspace is None:
+        nbytes = bitnet_linear_gemm_workspace_bytes(M, N, K)
+        if nbytes:
+            workspace = torch.zeros(nbytes, dtype=torch.uint8, device=x_q.device)
+    _need_cuda(workspace)
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().bitnet_linear_gemm(_ptr(W_packed), _ptr(gamma), N, K, _ptr(x_q), _ptr(a_scale), _ptr(x_rowsum), M,
+                                  _ptr(y), _dtype_code(y.dtype), _ptr(workspace), wsb, _stream(x_q.device))
+    _check("bitnet_linear_gemm", st)
+    return y
 
 
 def bitnet_bitlinear_gemv(x, W_packed, gamma, rms_gain=None, rms_eps: float = 1e-5, y=None, out_dtype=None):

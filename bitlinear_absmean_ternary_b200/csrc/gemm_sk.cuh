@@ -1,0 +1,402 @@
+// W1.58A8 product for decode-sized batches (M <= 64 tokens) on the Blackwell
+// tensor cores, balanced by splitting the work stream, not the tiles.
+//
+// Same operands and arithmetic as gemm.cuh (the pages' "low-bit matrix
+// product followed by rescaling", comrad404.com review, "Метод: как устроен
+// BitNet b1.58"): A = the ternary codes of 128 weight rows expanded to 8 bits
+// in registers and written to tensor memory, B = the int8 activations of the
+// BN token columns in shared memory (128-byte swizzled, K-major), int32
+// accumulators in tensor memory, 256 bytes of K per stage (8 MMAs of K = 32).
+//
+// At these sizes the product is bound by streaming the packed weights from
+// HBM (Habr repost on juhe.plus, "Но есть одно - НО": the weights are the
+// cost), so the design keeps every SM streaming an equal share of them:
+//
+//   * Work split (stream-K): the units are (row tile, K stage) pairs in
+//     tile-major order, U = ceil(N/128) * ceil(K/256) of them, and CTA c of
+//     the G CTAs (one per SM) takes the contiguous range [U*c/G, U*(c+1)/G).
+//     A range is a run of segments, one per row tile it touches.  A tile
+//     that lies wholly in one range is finished by that CTA.  A tile cut by
+//     range boundaries has one "finisher", the CTA holding its first K stage
+//     (the tile is the last segment of that CTA's range), and helpers, the
+//     later CTAs holding its other stages (for each helper the tile is its
+//     FIRST segment, so a CTA is the helper of at most one tile).  A helper
+//     stores its int32 partial tile into its own slot of the workspace and
+//     raises its flag; the finisher, which reaches the tile last, waits for
+//     the flags of its helpers, adds their partials (integer adds: the result
+//     is bit-identical to an unsplit product), dequantises, stores y and
+//     lowers the flags again, so the workspace is all zero between calls.
+//
+//   * Feed: the packed weights have a ring of their own (SW stages of 8 KB),
+//     freed as soon as the unpack warps have read a stage into registers, so
+//     the weight producer runs SW stages ahead of the tensor-memory writes.
+//     Its first SW stages are requested before waiting on the previous
+//     kernel (programmatic dependent launch): the weights never depend on it.
+//     The activations (a few KB per stage, read from L2) come through a
+//     shallower ring freed by the MMA commits.  The unpacked A operand has T
+//     tensor-memory slots of 64 columns, freed by the MMA commits.
+//
+// Warp roles (480 threads):
+//   warp 0, lane 0     weight producer (TMA, one 128-row x 64-byte box per stage);
+//   warp 1, lane 0     activation producer (TMA, two BN x 128-byte boxes per stage);
+//   warp 2             tensor-memory allocator; lane 0 issues the MMAs;
+//   warps 3..10        unpack: two warps per TMEM lane quarter (warp % 4),
+//                      taking alternate stages; thread = weight row;
+//   warps 11..14       epilogue, one per lane quarter; thread = weight row.
+// Every wait is bounded; a timeout flags the device error word, the role
+// stops, and the kernel drains what is in flight and exits.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "gemm.cuh"
+#include "ptx.cuh"
+
+namespace bitnet {
+
+constexpr int kSkFirstUnpack = 3;
+constexpr int kSkUnpackWarps = 8;
+constexpr int kSkFirstEpi = kSkFirstUnpack + kSkUnpackWarps;
+constexpr int kSkEpiWarps = 4;
+constexpr int kSkThreads = (kSkFirstEpi + kSkEpiWarps) * 32;
+
+template <int BN>
+struct SkCfg {
+  static constexpr int kWStage = kGemmBM * (kGemmBK / 4);  // packed codes of 128 rows x 256 K: 8 KB
+  static constexpr int kXSub = BN * 128;                   // one 128-byte-wide activation box
+  static constexpr int kXStage = kXSub * (kGemmBK / 128);  // activations of a stage
+  static constexpr int SW = BN <= 32 ? 16 : 12;            // weight ring stages
+  static constexpr int SX = BN <= 32 ? 8 : 6;              // activation ring stages
+  static constexpr int kAslot = kGemmBK / 4;               // TMEM columns per A slot
+  static constexpr int kAcol = 2 * BN;                     // two accumulators first
+  static constexpr int T = (512 - kAcol) / kAslot;         // A slots in TMEM
+  static constexpr int kXOff = SW * kWStage;
+  static constexpr int kBarOff = kXOff + SX * kXStage;
+  static constexpr int kNumBars = 2 * SW + 2 * SX + 2 * T + 6;
+  static constexpr int kScaleOff = kBarOff + ((kNumBars * 8 + 8 + 127) / 128) * 128;
+  static constexpr int kNeeded = 1024 + kScaleOff + BN * 8;
+  // The CTA holds all 512 TMEM columns: ask for enough shared memory that a
+  // second CTA never fits on the SM, so none waits in tcgen05.alloc.
+  static constexpr int kMinSmem = 233472 / 2;
+  static constexpr int kSmemBytes = kNeeded > kMinSmem ? kNeeded : kMinSmem;
+  // workspace: G flags (rounded to 256 bytes), then G partial tiles int32 [BN][128]
+  static constexpr int kPartInts = BN * kGemmBM;
+  static_assert(kWStage % 1024 == 0 && kXStage % 1024 == 0, "stages stay 1024-byte aligned");
+  static_assert(kAcol + T * kAslot <= 512 && T >= 2, "TMEM budget");
+  static_assert(kNeeded <= 232448, "shared memory budget");
+  static_assert(BN == 16 || BN == 32 || BN == 64, "token tile");
+};
+
+__host__ __device__ inline size_t sk_flag_bytes(int G) { return (static_cast<size_t>(G) * 4 + 255) / 256 * 256; }
+
+// CTA (of G) whose unit range [U*c/G, U*(c+1)/G) holds unit u.
+__device__ __forceinline__ int sk_cta_of(long long u, long long U, int G) {
+  return static_cast<int>(((u + 1) * G - 1) / U);
+}
+
+BN_DEV void st_release_gpu_u32(unsigned int* p, unsigned int v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+BN_DEV unsigned int ld_acquire_gpu_u32(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Barrier over the four epilogue warps on an mbarrier of 4 arrivals, with
+// a bounded wait (a warp that gave up earlier cannot hang the others).
+// `phase` counts the uses; every epilogue warp makes the same calls.
+BN_DEV bool sk_epi_sync(uint64_t* bar, int& phase) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, static_cast<uint32_t>(phase & 1));
+  ++phase;
+  return ok;
+}
+
+template <int BN, bool U8>
+__global__ void __launch_bounds__(kSkThreads, 1)
+    gemm_sk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
+                   const float* __restrict__ gamma_ptr, const float* __restrict__ a_scale,
+                   const int32_t* __restrict__ rowsum, int M, int N, int K, void* __restrict__ y, int y_dtype,
+                   unsigned int* __restrict__ flags, int* __restrict__ parts) {
+  using C = SkCfg<BN>;
+  constexpr int SW = C::SW, SX = C::SX, T = C::T;
+  constexpr int NMMA = kGemmBK / 32;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* w_full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* w_empty = w_full + SW;
+  uint64_t* x_full = w_empty + SW;
+  uint64_t* x_empty = x_full + SX;
+  uint64_t* a_full = x_empty + SX;
+  uint64_t* a_empty = a_full + T;
+  uint64_t* acc_full = a_empty + T;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* done = acc_empty + 2;
+  uint64_t* epi_bar = done + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi_bar + 1);
+  float* s_a = reinterpret_cast<float*>(smem + C::kScaleOff);
+  int* s_rs = reinterpret_cast<int*>(s_a + BN);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = (N + kGemmBM - 1) / kGemmBM;
+  const int nk = (K + kGemmBK - 1) / kGemmBK;
+  const long long U = static_cast<long long>(n_tiles) * nk;
+  const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
+  const long long u0 = U * cta / G, u1 = U * (cta + 1) / G;
+  const int total = static_cast<int>(u1 - u0);  // stages of this CTA
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < SW; ++s) {
+      mbar_init(&w_full[s], 1);
+      mbar_init(&w_empty[s], 4);
+    }
+    for (int s = 0; s < SX; ++s) {
+      mbar_init(&x_full[s], 1);
+      mbar_init(&x_empty[s], 1);
+    }
+    for (int s = 0; s < T; ++s) {
+      mbar_init(&a_full[s], 4);
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kSkEpiWarps);
+    }
+    mbar_init(done, 1);
+    mbar_init(epi_bar, kSkEpiWarps);
+    fence_barrier_init();
+    tma_prefetch_desc(&tmap_x);
+    tma_prefetch_desc(&tmap_w);
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ weight producer
+      // The packed weights never depend on the previous kernel: no wait at all.
+      bool ok = true;
+      int g = 0;
+      for (; g < total; ++g) {
+        const int s = g % SW;
+        if (g >= SW && !mbar_wait(&w_empty[s], ((g / SW) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
+        const long long u = u0 + g;
+        const int t = static_cast<int>(u / nk), kb = static_cast<int>(u - static_cast<long long>(t) * nk);
+        mbar_arrive_expect_tx(&w_full[s], C::kWStage);
+        tma_load_2d(smem + s * C::kWStage, &tmap_w, kb * (kGemmBK / 4), t * kGemmBM, &w_full[s]);
+      }
+      if (!ok)  // let the copies in flight land before the shared memory goes away
+        for (int h = g - SW > 0 ? g - SW : 0; h < g; ++h) mbar_wait(&w_full[h % SW], (h / SW) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ activation producer
+      pdl_wait();  // x_q comes from the previous kernel
+      bool ok = true;
+      int g = 0;
+      for (; g < total; ++g) {
+        const int s = g % SX;
+        if (g >= SX && !mbar_wait(&x_empty[s], ((g / SX) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
+        const long long u = u0 + g;
+        const int kb = static_cast<int>(u % nk);
+        uint8_t* xs = smem + C::kXOff + s * C::kXStage;
+        mbar_arrive_expect_tx(&x_full[s], C::kXStage);
+#pragma unroll
+        for (int i = 0; i < kGemmBK / 128; ++i) tma_load_2d(xs + i * C::kXSub, &tmap_x, kb * kGemmBK + 128 * i, 0, &x_full[s]);
+      }
+      if (!ok)
+        for (int h = g - SX > 0 ? g - SX : 0; h < g; ++h) mbar_wait(&x_full[h % SX], (h / SX) & 1);
+    }
+  } else if (warp == 2) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc = idesc_i8(kGemmBM, BN, !U8);
+      bool ok = true;
+      int g = 0, seg = 0;
+      for (long long u = u0; ok && u < u1; ++seg) {
+        const long long t = u / nk;
+        const long long seg_end = (t + 1) * nk < u1 ? (t + 1) * nk : u1;
+        const int b = seg & 1;
+        if (!mbar_wait(&acc_empty[b], ((seg >> 1) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (long long v = u; v < seg_end; ++v, ++g) {
+          const int a = g % T, sx = g % SX;
+          if (!mbar_wait(&a_full[a], (g / T) & 1) || !mbar_wait(&x_full[sx], (g / SX) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t xaddr = smem_addr(smem + C::kXOff + sx * C::kXStage);
+#pragma unroll
+          for (int kk = 0; kk < NMMA; ++kk)
+            mma_i8_tmemA(tmem + b * BN, tmem + C::kAcol + C::kAslot * a + 8 * kk,
+                         smem_desc_k_sw128(xaddr + (kk >> 2) * C::kXSub + 32 * (kk & 3)), idesc,
+                         (v > u || kk > 0) ? 1u : 0u);
+          tc_commit(&a_empty[a]);
+          tc_commit(&x_empty[sx]);
+        }
+        if (ok) tc_commit(&acc_full[b]);
+        u = seg_end;
+      }
+      tc_commit(done);  // arrives once every MMA issued above has finished
+      mbar_wait(done, 0);
+    }
+  } else if (warp < kSkFirstEpi) {
+    // ------------------------------------------------------------ unpack
+    const int q = warp & 3;
+    const int par = (warp - kSkFirstUnpack) >> 2;  // this warp takes stages with g % 2 == par
+    const int r = 32 * q + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    // 64-byte swizzle of the packed tile: 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3)
+    const uint32_t swz = static_cast<uint32_t>((r >> 1) & 3);
+    for (int g = par; g < total; g += 2) {
+      const int s = g % SW;
+      if (!__all_sync(0xffffffffu, mbar_wait(&w_full[s], (g / SW) & 1))) break;
+      const uint32_t wrow = smem_addr(smem + s * C::kWStage) + r * (kGemmBK / 4);
+      uint4 p[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) p[c] = lds128(wrow + ((static_cast<uint32_t>(c) ^ swz) << 4));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&w_empty[s]);  // the weight slot may be refilled
+      const int a = g % T;
+      if (!__all_sync(0xffffffffu, mbar_wait(&a_empty[a], ((g / T) & 1) ^ 1))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {  // two halves of 128 K each -> 32 TMEM columns each
+        const uint32_t pw[8] = {p[2 * h].x, p[2 * h].y, p[2 * h].z, p[2 * h].w,
+                                p[2 * h + 1].x, p[2 * h + 1].y, p[2 * h + 1].z, p[2 * h + 1].w};
+        uint32_t v[32];
+#pragma unroll
+        for (int wi = 0; wi < 8; ++wi)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t c4 = (pw[wi] >> (2 * j)) & 0x03030303u;
+            v[4 * wi + j] = U8 ? c4 : codes_to_signed(c4);
+          }
+        tmem_st_32x32b_x32(lane_base + C::kAcol + C::kAslot * a + 32 * h, v);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&a_full[a]);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int r = 32 * q + lane;  // accumulator row (TMEM lane) of this thread
+    const int et = (warp - kSkFirstEpi) * 32 + lane;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    pdl_wait();  // a_scale, rowsum and the workspace follow the previous kernel
+    const float gamma = __ldg(gamma_ptr);
+    if (et < BN) {
+      s_a[et] = et < M ? __ldg(a_scale + et) : 0.0f;
+      s_rs[et] = (U8 && et < M) ? __ldg(rowsum + et) : 0;
+    }
+    int ephase = 0;
+    sk_epi_sync(epi_bar, ephase);
+    int seg = 0;
+    for (long long u = u0; u < u1; ++seg) {
+      const long long t = u / nk;
+      const int kb_lo = static_cast<int>(u - t * nk);
+      const long long seg_end = (t + 1) * nk < u1 ? (t + 1) * nk : u1;
+      const int kb_hi = static_cast<int>(seg_end - t * nk);
+      u = seg_end;
+      const int b = seg & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[b], (seg >> 1) & 1))) break;
+      tc_fence_after();
+      uint32_t v[BN];
+#pragma unroll
+      for (int c0 = 0; c0 < BN; c0 += 16) {
+        uint32_t w16[16];
+        tmem_ld_32x32b_x16(lane_base + b * BN + c0, w16);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[c0 + j] = w16[j];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);  // the accumulator may be reused
+      if (kb_lo > 0) {
+        // helper: this CTA's partial of a tile finished by an earlier CTA
+        int* slot = parts + static_cast<size_t>(cta) * C::kPartInts;
+#pragma unroll
+        for (int j = 0; j < BN; ++j) slot[j * kGemmBM + r] = static_cast<int>(v[j]);
+        __threadfence();
+        if (sk_epi_sync(epi_bar, ephase) && et == 0) st_release_gpu_u32(&flags[cta], 1u);
+        continue;
+      }
+      if (kb_hi < nk) {
+        // finisher: add the partials of the helpers (the CTAs after this one that hold the tile's other stages)
+        const int last = sk_cta_of(t * nk + nk - 1, U, G);
+        bool ok = true;
+        if (et == 0) {
+          const uint64_t t0 = global_timer_ns();
+          for (int h = cta + 1; h <= last && ok; ++h) {
+            for (uint32_t i = 1; ld_acquire_gpu_u32(&flags[h]) == 0u; ++i) {
+              if ((i & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+                flag_timeout();
+                ok = false;
+                break;
+              }
+            }
+          }
+        }
+        sk_epi_sync(epi_bar, ephase);
+        __threadfence();
+        for (int h = cta + 1; h <= last; ++h) {
+          const int* slot = parts + static_cast<size_t>(h) * C::kPartInts;
+#pragma unroll
+          for (int j = 0; j < BN; ++j) v[j] += static_cast<uint32_t>(__ldcg(slot + j * kGemmBM + r));
+        }
+        sk_epi_sync(epi_bar, ephase);
+        if (et == 0)
+          for (int h = cta + 1; h <= last; ++h) flags[h] = 0u;  // all zero again for the next call
+      }
+      // dequantise and store: thread = output feature n, columns = tokens
+      const int n = static_cast<int>(t) * kGemmBM + r;
+      if (n < N) {
+#pragma unroll
+        for (int j = 0; j < BN; ++j) {
+          if (j < M) {
+            const int a = static_cast<int>(v[j]) - s_rs[j];
+            const int64_t o = static_cast<int64_t>(j) * N + n;
+            if (y_dtype == 2) {
+              static_cast<int32_t*>(y)[o] = a;
+            } else {
+              const float val = __fmul_rn(__fmul_rn(__int2float_rn(a), gamma), s_a[j]);
+              if (y_dtype == 0) static_cast<float*>(y)[o] = val;
+              else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(val);
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace bitnet

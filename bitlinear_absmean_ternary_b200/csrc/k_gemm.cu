@@ -1,7 +1,9 @@
-// Host side of bitnet_linear_gemm: the tcgen05 tensor-core product
-// (gemm.cuh): tensor maps, tile size by M, split-K choice, launch.
+// Host side of bitnet_linear_gemm: the tcgen05 tensor-core products --
+// gemm_sk.cuh (stream-K, M <= 64 with a workspace) and gemm.cuh (persistent
+// tiles, cluster split-K for few tiles): tensor maps, tile size by M, launch.
 #include "host_common.h"
 #include "gemm.cuh"
+#include "gemm_sk.cuh"
 
 namespace {
 
@@ -135,24 +137,81 @@ cudaError_t launch_gemm_bn(const uint8_t* Wp, const float* gamma, int N, int K, 
   return launch_gemm_t<BN, S, false>(mx, mw, gamma, a, rs, M, N, K, y, yd, s);
 }
 
+// Token tile of the stream-K kernel for M <= 64 tokens.
+int sk_bn(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
+
+// Workspace of the stream-K kernel on the current device: a flag per CTA
+// (one CTA per SM at most) and a partial int32 tile [BN][128] per CTA.
+size_t sk_workspace_bytes(int64_t M) {
+  const int G = sm_count();
+  return sk_flag_bytes(G) + static_cast<size_t>(G) * sk_bn(M) * kGemmBM * 4;
+}
+
+template <int BN, bool U8>
+cudaError_t launch_sk(const CUtensorMap& mx, const CUtensorMap& mw, const float* gamma, const float* a,
+                      const int32_t* rs, int M, int N, int K, void* y, int yd, void* ws, cudaStream_t s) {
+  using C = SkCfg<BN>;
+  static std::atomic<bool> done[kMaxDevices] = {};
+  const cudaError_t e = set_smem(gemm_sk_kernel<BN, U8>, C::kSmemBytes, done);
+  if (e != cudaSuccess) return e;
+  const int64_t units = static_cast<int64_t>((N + kGemmBM - 1) / kGemmBM) * ((K + kGemmBK - 1) / kGemmBK);
+  const int sms = sm_count();
+  const int G = static_cast<int>(units < sms ? units : sms);
+  unsigned int* flags = static_cast<unsigned int*>(ws);
+  int* parts = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + sk_flag_bytes(sms));
+  return launch_pdl(gemm_sk_kernel<BN, U8>, dim3(G), dim3(kSkThreads), C::kSmemBytes, s, mx, mw, gamma, a, rs, M, N,
+                    K, y, yd, flags, parts);
+}
+
+template <int BN>
+cudaError_t launch_sk_bn(const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
+                         const int32_t* rs, int M, void* y, int yd, void* ws, cudaStream_t s) {
+  CUtensorMap mx, mw;
+  if (!make_map_u8(&mx, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(K), 128, BN,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (!make_map_u8(&mw, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4),
+                   kGemmBK / 4, kGemmBM, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
+  if (rs != nullptr) return launch_sk<BN, true>(mx, mw, gamma, a, rs, M, N, K, y, yd, ws, s);
+  return launch_sk<BN, false>(mx, mw, gamma, a, rs, M, N, K, y, yd, ws, s);
+}
+
 }  // namespace
 
 BITNET_DEFINE_TAKE_ERROR(gemm)
 
 extern "C" {
 
+size_t bitnet_linear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M < 1 || M > 64 || N < 1 || N > INT32_MAX || !valid_k(K)) return 0;
+  return sk_workspace_bytes(M);
+}
+
 bitnet_status bitnet_linear_gemm(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, const int8_t* x_q,
                                  const float* a_scale, const int32_t* x_rowsum, int64_t M, void* y, int y_dtype,
-                                 void* stream) {
+                                 void* workspace, size_t workspace_bytes, void* stream) {
   const bitnet_status st = check_linear(W_packed, gamma, N, K, x_q, a_scale, x_rowsum, M, y, y_dtype);
   if (st != BITNET_OK) return st;
+  if (!aligned(workspace, 16)) return BITNET_ERR_INVALID_ARG;
+  const bool stream_k = workspace != nullptr && M <= 64;
+  if (stream_k && workspace_bytes < sk_workspace_bytes(M)) return BITNET_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int n = static_cast<int>(N), k = static_cast<int>(K), m = static_cast<int>(M);
   cudaError_t e;
-  if (m <= 16) e = launch_gemm_bn<16, 6>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
-  else if (m <= 32) e = launch_gemm_bn<32, 6>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
-  else if (m <= 64) e = launch_gemm_bn<64, 6>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
-  else e = launch_gemm_bn<128, 4>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
+  if (stream_k) {
+    if (m <= 16) e = launch_sk_bn<16>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, workspace, s);
+    else if (m <= 32) e = launch_sk_bn<32>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, workspace, s);
+    else e = launch_sk_bn<64>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, workspace, s);
+  } else if (m <= 16) {
+    e = launch_gemm_bn<16, 6>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
+  } else if (m <= 32) {
+    e = launch_gemm_bn<32, 6>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
+  } else if (m <= 64) {
+    e = launch_gemm_bn<64, 6>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
+  } else {
+    e = launch_gemm_bn<128, 4>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
+  }
   return from_cuda(e);
 }
 

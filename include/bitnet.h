@@ -187,18 +187,46 @@ bitnet_status bitnet_linear_gemv(const uint8_t* W_packed, const float* gamma, in
                                  int64_t M, void* y, int y_dtype, void* stream);
 
 /*
+ * Bytes of workspace bitnet_linear_gemm uses for an M x K by N x K product on
+ * the CURRENT device (it depends on the device's SM count): for M <= 64 a
+ * flag per SM and one partial int32 tile of 128 rows x 16, 32 or 64 tokens
+ * per SM (about 1.2, 2.4 or 4.8 MB on a B200); 0 for M > 64, where no
+ * workspace is used.
+ */
+size_t bitnet_linear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
  * The same product for any M >= 1 on the 5th-generation tensor cores
  * (tcgen05 kind::i8, int32 accumulators in tensor memory): packed weight
  * tiles and activation tiles arrive in shared memory by TMA, the ternary
  * codes are expanded to 8-bit in registers and written to tensor memory as
  * the A operand, the activations are the B operand in shared memory.
- * Same arguments, formulas and results as bitnet_linear_gemv.
+ * Same formulas and results as bitnet_linear_gemv (the low-bit product
+ * followed by rescaling of the comrad404.com review, section "Метод").
+ *
+ * workspace [in,out] device memory of at least
+ *           bitnet_linear_gemm_workspace_bytes(M, N, K) bytes, 16-byte
+ *           aligned, or NULL.  With M <= 64 and a workspace, the product
+ *           runs "stream-K": every SM takes an equal share of the (row tile,
+ *           K step) work and partial tiles cut between SMs are added
+ *           exactly in int32 through the workspace, so decode-sized batches
+ *           stream the packed weights at HBM rate.  Zero the workspace before
+ *           its first use (e.g. cudaMemset): its first bytes are flags that
+ *           must start at zero, and every call leaves them zero again (the
+ *           rest is scratch that every call overwrites before reading).  Two calls that may run at the same time (on two
+ *           streams) must not share a workspace.  If a call reports
+ *           BITNET_ERR_TIMEOUT through bitnet_get_device_status, zero the
+ *           workspace again before reusing it.  Without a workspace (NULL,
+ *           with workspace_bytes ignored) or for M > 64, the product runs on
+ *           persistent tiles, split over thread-block clusters when there
+ *           are few tiles; the results are identical.
  * M <= 2^31 - 1, N <= 2^31 - 1, K <= 2^31 - 1 with M*N fitting the output.
  * Asynchronous.
  */
 bitnet_status bitnet_linear_gemm(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K,
                                  const int8_t* x_q, const float* a_scale, const int32_t* x_rowsum,
-                                 int64_t M, void* y, int y_dtype, void* stream);
+                                 int64_t M, void* y, int y_dtype, void* workspace, size_t workspace_bytes,
+                                 void* stream);
 
 /*
  * Fused decode BitLinear: bitnet_quant_act followed by bitnet_linear_gemv in

@@ -89,7 +89,9 @@ def test_quant_rejects_bad_arguments(L):
 def test_linear_rejects_bad_arguments(L, name):
     fn = getattr(L, name)
 
-    def call(W=FAKE, g=FAKE, N=8, K=64, xq=FAKE, a=FAKE, rs=None, M=1, y=FAKE, yd=bl.BITNET_BF16):
+    def call(W=FAKE, g=FAKE, N=8, K=64, xq=FAKE, a=FAKE, rs=None, M=1, y=FAKE, yd=bl.BITNET_BF16, ws=None, wsb=0):
+        if name == "bitnet_linear_gemm":
+            return fn(W, g, N, K, xq, a, rs, M, y, yd, ws, wsb, None)
         return fn(W, g, N, K, xq, a, rs, M, y, yd, None)
 
     assert call(W=None) == bl.BITNET_ERR_INVALID_ARG
@@ -106,6 +108,24 @@ def test_linear_rejects_bad_arguments(L, name):
     assert call(N=1 << 31) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
     if name == "bitnet_linear_gemv":
         assert call(M=9) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    else:
+        need = bl.bitnet_linear_gemm_workspace_bytes(16, 8, 64)
+        assert call(ws=MIS, wsb=need) == bl.BITNET_ERR_INVALID_ARG      # misaligned workspace
+        assert call(M=16, ws=FAKE, wsb=need - 16) == bl.BITNET_ERR_INVALID_ARG  # workspace too small
+
+
+def test_gemm_workspace_bytes(L):
+    # one flag per SM (rounded to 256 bytes) and one int32 tile of 128 rows x BN tokens per SM
+    sms = [bl.bitnet_linear_gemm_workspace_bytes(m, 256, 256) for m in (1, 16, 17, 32, 33, 64)]
+    assert sms[0] == sms[1] and sms[2] == sms[3] and sms[4] == sms[5]
+    assert sms[0] > 0 and sms[0] % 256 == 0
+    per_sm_16 = sms[0]
+    # BN = 16, 32, 64: the partial tiles double with BN, the flags do not
+    assert sms[2] - sms[0] == sms[4] - sms[2] - (sms[2] - sms[0])
+    assert bl.bitnet_linear_gemm_workspace_bytes(65, 256, 256) == 0
+    assert bl.bitnet_linear_gemm_workspace_bytes(0, 256, 256) == 0
+    assert bl.bitnet_linear_gemm_workspace_bytes(8, 256, 100) == 0
+    assert per_sm_16 >= 16 * 128 * 4
 
 
 def test_fused_rejects_bad_arguments(L):

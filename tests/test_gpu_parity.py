@@ -427,3 +427,80 @@ def test_gemv_after_a_kernel_that_writes_the_weights(dev, orc):
         y2 = bl.bitnet_linear_gemv(P2, G, xq, a, rs, out_dtype=torch.float32)
         assert ulp_diff_f32(y1.cpu().numpy(), y_r).max() == 0
         assert ulp_diff_f32(y2.cpu().numpy(), y_r).max() == 0
+
+
+# --------------------------------------------------------------------------- stream-K GEMM (M <= 64)
+
+SK_CASES = [(1, 128, 64), (16, 21504, 5376), (16, 5376, 21504), (64, 3840, 2560), (64, 2560, 6912),
+            (5, 300, 320), (33, 1000, 2624), (17, 777, 5376), (64, 13824, 2560), (2, 129, 21504)]
+
+
+@pytest.mark.parametrize("M,N,K", SK_CASES)
+def test_gemm_stream_k_matches_tiles_and_oracle(dev, orc, M, N, K):
+    """Stream-K (equal work per SM, partial tiles added through the workspace)
+    against the persistent-tile path and the oracle, with one workspace reused
+    by every call (the calls must leave its flags zero)."""
+    import torch
+    rng = np.random.default_rng(M + N + K)
+    q = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    packed = orc.pack_codes(q)
+    x = synth.activations(M, K, 11, 5, "student_t4", 0.0, 1.0, "f32")
+    xq, a, rs = orc.quant_act(x)
+    gamma = np.float32(0.0211)
+    P, G = _t(packed, dev), _t(np.array([gamma], np.float32), dev)
+    XQ, A, RS = _t(xq, dev), _t(a, dev), _t(rs, dev)
+    ws = torch.zeros(bl.bitnet_linear_gemm_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
+    ms = rng.integers(0, M, 4000)
+    ns = rng.integers(0, N, 4000)
+    acc_r, y_r = orc.bitlinear_sampled(packed, gamma, K, xq, a, ms, ns)
+    for rowsum in (RS, None):
+        for out in (torch.int32, torch.float32, torch.bfloat16):
+            y_sk = bl.bitnet_linear_gemm(P, G, XQ, A, rowsum, out_dtype=out, workspace=ws)
+            y_t = bl.bitnet_linear_gemm(P, G, XQ, A, rowsum, out_dtype=out, stream_k=False)
+            assert torch.equal(y_sk, y_t)
+            if out == torch.int32:
+                np.testing.assert_array_equal(y_sk.cpu().numpy()[ms, ns], acc_r)
+            elif out == torch.float32:
+                assert ulp_diff_f32(y_sk.cpu().numpy()[ms, ns], y_r).max() == 0
+            else:
+                yb = y_sk.view(torch.int16).cpu().numpy().view(np.uint16)[ms, ns]
+                assert ulp_diff_bf16(yb, orc.f32_to_bf16(y_r)).max() == 0
+    torch.cuda.synchronize()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    assert int(ws[:4 * sms].view(torch.int32).abs().sum()) == 0, "flags left raised"
+    assert bl.bitnet_get_device_status() == bl.BITNET_OK
+
+
+def test_gemm_stream_k_in_a_cuda_graph(dev, orc):
+    """Several stream-K calls sharing one workspace inside a CUDA graph, the
+    graph replayed three times: every replay exact, flags zero at the end."""
+    import torch
+    M, N, K = 16, 6912, 2560
+    rng = np.random.default_rng(5)
+    q = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    packed = orc.pack_codes(q)
+    x = synth.activations(M, K, 2, 5, "normal", 0.01, 20.0, "bf16")
+    xq, a, rs = orc.quant_act(x)
+    gamma = np.float32(0.0187)
+    acc_r, _ = orc.bitlinear(packed, gamma, K, xq, a)
+    P, G = _t(packed, dev), _t(np.array([gamma], np.float32), dev)
+    XQ, A, RS = _t(xq, dev), _t(a, dev), _t(rs, dev)
+    ws = torch.zeros(bl.bitnet_linear_gemm_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
+    ys = [torch.empty((M, N), dtype=torch.int32, device=dev) for _ in range(3)]
+    s = torch.cuda.Stream(dev)
+    bl.bitnet_linear_gemm(P, G, XQ, A, RS, y=ys[0], workspace=ws)  # first call outside the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for y in ys:
+            bl.bitnet_linear_gemm(P, G, XQ, A, RS, y=y, workspace=ws)
+    for _ in range(3):
+        for y in ys:
+            y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        for y in ys:
+            np.testing.assert_array_equal(y.cpu().numpy(), acc_r)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    assert int(ws[:4 * sms].view(torch.int32).abs().sum()) == 0
+    assert bl.bitnet_get_device_status() == bl.BITNET_OK
