@@ -280,13 +280,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     constexpr int CW = BN / EH < 32 ? BN / EH : 32;
     const int half = (warp - kGemmFirstEpiWarp) >> 2;
     const int col_lo = half * (BN / EH), col_hi = half < EH ? (half + 1) * (BN / EH) : col_lo;
+    constexpr int NCH = (BN / EH) / CW;  // column chunks of this warp per tile
     int tc = 0;
     for (int t = cid; t < tiles; t += ncl, ++tc) {
       const int b = tc % NB;
-      if (!__all_sync(0xffffffffu, mbar_wait(&accfull[b], (tc / NB) & 1))) break;
-      tc_fence_after();
       const int n0 = (t % n_tiles) * kGemmBM;
       const int m0 = (t / n_tiles) * BN;
+      // per-token scale and row sum of this warp's columns, one token per lane and
+      // chunk, requested before the accumulator wait so the loads overlap it
+      float pa[NCH];
+      int prs[NCH];
+#pragma unroll
+      for (int ch = 0; ch < NCH; ++ch) {
+        const int mm = m0 + col_lo + ch * CW + (lane < CW ? lane : 0);
+        const bool inb = col_lo < col_hi && lane < CW && mm < M;
+        pa[ch] = inb ? __ldg(a_scale + mm) : 0.0f;
+        prs[ch] = (U8 && inb) ? __ldg(rowsum + mm) : 0;
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&accfull[b], (tc / NB) & 1))) break;
+      tc_fence_after();
       if constexpr (KSPLIT > 1) {
         // ---- split-K: partial -> shared memory, exchange, reduce this CTA's slice of rows
         const int r = 32 * q + lane;  // accumulator row (TMEM lane) this thread drains
@@ -355,19 +367,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       } else {
         // ---- one CTA per tile: dequantise straight from TMEM
         const int n = n0 + 32 * q + lane;
-#pragma unroll 1
-        for (int cc = col_lo; cc < col_hi; cc += CW) {
+#pragma unroll
+        for (int ch = 0; ch < NCH; ++ch) {
+          const int cc = col_lo + ch * CW;
+          if (cc >= col_hi) break;
           uint32_t v[CW];
           if constexpr (CW == 32) {
             tmem_ld_32x32b_x32(lane_base + b * BN + cc, v);
           } else {
             tmem_ld_32x32b_x16(lane_base + b * BN + cc, v);
           }
-          // per-token scale and row sum of the CW tokens of this chunk, one per lane
-          const int mm = m0 + cc + (lane < CW ? lane : 0);
-          const bool inb = lane < CW && mm < M;
-          const float my_a = inb ? __ldg(a_scale + mm) : 0.0f;
-          const int my_rs = (U8 && inb) ? __ldg(rowsum + mm) : 0;
+          const float my_a = pa[ch];
+          const int my_rs = prs[ch];
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < CW; ++j) {

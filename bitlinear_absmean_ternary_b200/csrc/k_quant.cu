@@ -16,8 +16,9 @@ cudaError_t launch_quant_t(const void* x, int64_t M, int K, const void* gain, fl
   static std::atomic<bool> done[kMaxDevices] = {};
   const cudaError_t e = set_smem(quant_act_kernel<T, MAXC, NTHR>, 0, done);
   if (e != cudaSuccess) return e;
+  const int early = M <= sm_count() ? 1 : 0;  // the whole grid is resident at once
   return launch_pdl(quant_act_kernel<T, MAXC, NTHR>, dim3(static_cast<unsigned>(M)), dim3(threads), 0, s,
-                    static_cast<const T*>(x), K, static_cast<const T*>(gain), eps, xq, a, rs);
+                    static_cast<const T*>(x), K, static_cast<const T*>(gain), eps, xq, a, rs, early);
 }
 
 template <int MAXC, bool NORM>

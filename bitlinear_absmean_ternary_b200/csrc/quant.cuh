@@ -268,18 +268,24 @@ BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict_
 // fixed summation order is defined on 256 lanes); without it the launcher
 // takes the fewest whole warps that give every thread the same number of
 // chunks (160 threads x 2 chunks for K = 2560, 224 x 4 for K = 6912).
+// early: every CTA of the grid is resident at once (a decode-sized batch),
+// so the next kernel on the stream may be launched right away -- the
+// product kernels then fetch their weights while this one runs; with more
+// rows than fit at once, the next kernel launches once every CTA is past
+// its quantisation, so that it takes no SM from the rows still waiting.
 template <typename T, int MAXC, int NTHR = kQuantThreads>
 __global__ void __launch_bounds__(NTHR) quant_act_kernel(const T* __restrict__ x, int K,
                                                                   const T* __restrict__ gain, float rms_eps,
                                                                   int8_t* __restrict__ xq, float* __restrict__ a_out,
-                                                                  int32_t* __restrict__ rowsum_out) {
+                                                                  int32_t* __restrict__ rowsum_out, int early) {
   __shared__ QuantScratch sc;
   const int64_t m = blockIdx.x;
+  if (early) pdl_launch_dependents();
   pdl_wait();
   float amax;
   int sum;
   quant_row_cta<T, MAXC>(x + m * K, K, gain, rms_eps, xq + m * K, sc, amax, sum);
-  pdl_launch_dependents();
+  if (!early) pdl_launch_dependents();
   if (threadIdx.x == 0) {
     a_out[m] = amax == 0.0f ? 0.0f : __fdiv_rn(amax, 127.0f);
     if (rowsum_out != nullptr) rowsum_out[m] = sum;
