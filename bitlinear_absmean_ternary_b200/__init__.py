@@ -60,6 +60,10 @@ def lib() -> ctypes.CDLL:
         L.bitnet_linear_gemm.restype = I
         L.bitnet_linear_gemm_workspace_bytes.argtypes = [I64, I64, I64]
         L.bitnet_linear_gemm_workspace_bytes.restype = ctypes.c_size_t
+        L.bitnet_linear_upgate_workspace_bytes.argtypes = [I64, I64, I64]
+        L.bitnet_linear_upgate_workspace_bytes.restype = ctypes.c_size_t
+        L.bitnet_linear_upgate_gemm.argtypes = [P, P, P, P, I64, I64, P, P, P, I64, P, P, ctypes.c_size_t, P]
+        L.bitnet_linear_upgate_gemm.restype = I
         L.bitnet_bitlinear_gemv.argtypes = [P, I, P, F, P, P, I64, I64, I64, P, I, P]
         L.bitnet_bitlinear_gemv.restype = I
         L.bitnet_bitlinear_ffn_gemv.argtypes = [P, I, I64, I64, I64, P, F, P, P, P, P, P, F, P, P, P, P, I, P, P]
@@ -264,6 +268,36 @@ def bitnet_linear_gemm(W_packed, gamma, x_q, a_scale, x_rowsum=None, y=None, out
                                   _ptr(y), _dtype_code(y.dtype), _ptr(workspace), wsb, _stream(x_q.device))
     _check("bitnet_linear_gemm", st)
     return y
+
+
+def bitnet_linear_upgate_workspace_bytes(M: int, F: int, K: int) -> int:
+    """Workspace bytes of bitnet_linear_upgate_gemm on the current device."""
+    return int(lib().bitnet_linear_upgate_workspace_bytes(M, F, K))
+
+
+def bitnet_linear_upgate_gemm(W_up, gamma_up, W_gate, gamma_gate, x_q, a_scale, x_rowsum=None, h=None,
+                              workspace=None):
+    """FFN up and gate products with the squared-ReLU gate fused in the epilogue:
+    h = bf16(relu(g)^2 * u), M x F.  workspace: zeroed uint8 device tensor of
+    bitnet_linear_upgate_workspace_bytes bytes, reused across calls (allocated
+    zeroed for this call when None).  Returns h."""
+    torch = _torch()
+    _need_cuda(W_up, gamma_up, W_gate, gamma_gate, x_q, a_scale, x_rowsum, h, workspace)
+    F = W_up.shape[0]
+    K = W_up.shape[1] * 4
+    M = x_q.shape[0]
+    if tuple(W_gate.shape) != tuple(W_up.shape) or x_q.shape[1] != K:
+        raise ValueError("W_up, W_gate (F x K/4) and x_q (M x K) disagree")
+    if h is None:
+        h = torch.empty((M, F), dtype=torch.bfloat16, device=x_q.device)
+    if workspace is None:
+        workspace = torch.zeros(bitnet_linear_upgate_workspace_bytes(M, F, K), dtype=torch.uint8,
+                                device=x_q.device)
+    st = lib().bitnet_linear_upgate_gemm(_ptr(W_up), _ptr(gamma_up), _ptr(W_gate), _ptr(gamma_gate), F, K,
+                                         _ptr(x_q), _ptr(a_scale), _ptr(x_rowsum), M, _ptr(h), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(x_q.device))
+    _check("bitnet_linear_upgate_gemm", st)
+    return h
 
 
 def bitnet_bitlinear_gemv(x, W_packed, gamma, rms_gain=None, rms_eps: float = 1e-5, y=None, out_dtype=None):

@@ -36,6 +36,19 @@
 //     shallower ring freed by the MMA commits.  The unpacked A operand has T
 //     tensor-memory slots of 64 columns, freed by the MMA commits.
 //
+//   * Token tiles: the tiles are (row tile, token tile) pairs, row tiles
+//     fastest, so consecutive units share their activation tile in L2.
+//
+//   * GATE (the FFN's up and gate projections in one product, inferownia.pl,
+//     "BitNet b1.58: era 1-bitowych LLM-ów", "Zrób to sam": squared ReLU in
+//     the FFN; kripta.biz 2B4T news: ReLU^2 in the FFN layers): a tile is 64
+//     features, its rows 0..63 the up rows and 64..127 the gate rows of those
+//     features (two 64-row weight boxes per stage), so the epilogue holds u
+//     and g of every feature: the gate quarters dequantise g into shared
+//     memory and the up quarters write h = bf16(RN32(RN32(r*r)*u)), r = g if
+//     g > 0 else +0, straight into the down projection's input; u and g never
+//     reach memory.
+//
 // Warp roles (480 threads):
 //   warp 0, lane 0     weight producer (TMA, one 128-row x 64-byte box per stage);
 //   warp 1, lane 0     activation producer (TMA, two BN x 128-byte boxes per stage);
@@ -60,7 +73,7 @@ constexpr int kSkFirstEpi = kSkFirstUnpack + kSkUnpackWarps;
 constexpr int kSkEpiWarps = 4;
 constexpr int kSkThreads = (kSkFirstEpi + kSkEpiWarps) * 32;
 
-template <int BN>
+template <int BN, bool GATE = false>
 struct SkCfg {
   static constexpr int kWStage = kGemmBM * (kGemmBK / 4);  // packed codes of 128 rows x 256 K: 8 KB
   static constexpr int kXSub = BN * 128;                   // one 128-byte-wide activation box
@@ -74,7 +87,9 @@ struct SkCfg {
   static constexpr int kBarOff = kXOff + SX * kXStage;
   static constexpr int kNumBars = 2 * SW + 2 * SX + 2 * T + 6;
   static constexpr int kScaleOff = kBarOff + ((kNumBars * 8 + 8 + 127) / 128) * 128;
-  static constexpr int kNeeded = 1024 + kScaleOff + BN * 8;
+  static constexpr int kGateOff = kScaleOff + 2 * BN * 8;  // (GATE) g of a tile, fp32 [BN][64]
+  static constexpr int kRowsPerTile = GATE ? 64 : kGemmBM;  // output features per tile
+  static constexpr int kNeeded = 1024 + kGateOff + (GATE ? BN * 64 * 4 : 0);
   // The CTA holds all 512 TMEM columns: ask for enough shared memory that a
   // second CTA never fits on the SM, so none waits in tcgen05.alloc.
   static constexpr int kMinSmem = 233472 / 2;
@@ -114,13 +129,18 @@ BN_DEV bool sk_epi_sync(uint64_t* bar, int& phase) {
   return ok;
 }
 
-template <int BN, bool U8>
+// N: output features (rows of W; for GATE the rows of W_up and of W_gate).
+// tmap_w2 / gamma2_ptr: W_gate and its scale (GATE only).  y: M x N outputs
+// of y_dtype, or for GATE the bf16 h (M x N).
+template <int BN, bool U8, bool GATE = false>
 __global__ void __launch_bounds__(kSkThreads, 1)
     gemm_sk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                   const float* __restrict__ gamma_ptr, const float* __restrict__ a_scale,
+                   const __grid_constant__ CUtensorMap tmap_w2, const float* __restrict__ gamma_ptr,
+                   const float* __restrict__ gamma2_ptr, const float* __restrict__ a_scale,
                    const int32_t* __restrict__ rowsum, int M, int N, int K, void* __restrict__ y, int y_dtype,
                    unsigned int* __restrict__ flags, int* __restrict__ parts) {
-  using C = SkCfg<BN>;
+  using C = SkCfg<BN, GATE>;
+  constexpr int RPT = C::kRowsPerTile;
   constexpr int SW = C::SW, SX = C::SX, T = C::T;
   constexpr int NMMA = kGemmBK / 32;
   extern __shared__ uint8_t smem_raw[];
@@ -136,13 +156,15 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   uint64_t* done = acc_empty + 2;
   uint64_t* epi_bar = done + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi_bar + 1);
-  float* s_a = reinterpret_cast<float*>(smem + C::kScaleOff);
-  int* s_rs = reinterpret_cast<int*>(s_a + BN);
+  float* s_a = reinterpret_cast<float*>(smem + C::kScaleOff);  // [2][BN]: double-buffered per segment
+  int* s_rs = reinterpret_cast<int*>(s_a + 2 * BN);           // [2][BN]
+  float* gbuf = reinterpret_cast<float*>(smem + C::kGateOff);  // GATE: [BN][64]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_tiles = (N + kGemmBM - 1) / kGemmBM;
+  const int n_tiles = (N + RPT - 1) / RPT;
+  const int m_tiles = (M + BN - 1) / BN;
   const int nk = (K + kGemmBK - 1) / kGemmBK;
-  const long long U = static_cast<long long>(n_tiles) * nk;
+  const long long U = static_cast<long long>(n_tiles) * m_tiles * nk;
   const int G = static_cast<int>(gridDim.x), cta = static_cast<int>(blockIdx.x);
   const long long u0 = U * cta / G, u1 = U * (cta + 1) / G;
   const int total = static_cast<int>(u1 - u0);  // stages of this CTA
@@ -169,6 +191,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tmap_x);
     tma_prefetch_desc(&tmap_w);
+    if constexpr (GATE) tma_prefetch_desc(&tmap_w2);
   }
   if (warp == 2) {
     tmem_alloc(tmem_holder, 512);
@@ -193,9 +216,17 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           break;
         }
         const long long u = u0 + g;
-        const int t = static_cast<int>(u / nk), kb = static_cast<int>(u - static_cast<long long>(t) * nk);
+        const long long t = u / nk;
+        const int kb = static_cast<int>(u - t * nk);
+        const int row0 = static_cast<int>(t % n_tiles) * RPT;
         mbar_arrive_expect_tx(&w_full[s], C::kWStage);
-        tma_load_2d(smem + s * C::kWStage, &tmap_w, kb * (kGemmBK / 4), t * kGemmBM, &w_full[s]);
+        if constexpr (GATE) {
+          // up rows of the tile's 64 features, then their gate rows
+          tma_load_2d(smem + s * C::kWStage, &tmap_w, kb * (kGemmBK / 4), row0, &w_full[s]);
+          tma_load_2d(smem + s * C::kWStage + C::kWStage / 2, &tmap_w2, kb * (kGemmBK / 4), row0, &w_full[s]);
+        } else {
+          tma_load_2d(smem + s * C::kWStage, &tmap_w, kb * (kGemmBK / 4), row0, &w_full[s]);
+        }
       }
       if (!ok)  // let the copies in flight land before the shared memory goes away
         for (int h = g - SW > 0 ? g - SW : 0; h < g; ++h) mbar_wait(&w_full[h % SW], (h / SW) & 1);
@@ -213,11 +244,14 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           break;
         }
         const long long u = u0 + g;
-        const int kb = static_cast<int>(u % nk);
+        const long long t = u / nk;
+        const int kb = static_cast<int>(u - t * nk);
+        const int m0 = static_cast<int>(t / n_tiles) * BN;
         uint8_t* xs = smem + C::kXOff + s * C::kXStage;
         mbar_arrive_expect_tx(&x_full[s], C::kXStage);
 #pragma unroll
-        for (int i = 0; i < kGemmBK / 128; ++i) tma_load_2d(xs + i * C::kXSub, &tmap_x, kb * kGemmBK + 128 * i, 0, &x_full[s]);
+        for (int i = 0; i < kGemmBK / 128; ++i)
+          tma_load_2d(xs + i * C::kXSub, &tmap_x, kb * kGemmBK + 128 * i, m0, &x_full[s]);
       }
       if (!ok)
         for (int h = g - SX > 0 ? g - SX : 0; h < g; ++h) mbar_wait(&x_full[h % SX], (h / SX) & 1);
@@ -305,13 +339,9 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     const int et = (warp - kSkFirstEpi) * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * q) << 16);
     pdl_wait();  // a_scale, rowsum and the workspace follow the previous kernel
-    const float gamma = __ldg(gamma_ptr);
-    if (et < BN) {
-      s_a[et] = et < M ? __ldg(a_scale + et) : 0.0f;
-      s_rs[et] = (U8 && et < M) ? __ldg(rowsum + et) : 0;
-    }
+    // row r's scale: W_up's (or W's) for the first 64 rows of a gated tile, W_gate's for the others
+    const float gamma = (GATE && r >= 64) ? __ldg(gamma2_ptr) : __ldg(gamma_ptr);
     int ephase = 0;
-    sk_epi_sync(epi_bar, ephase);
     int seg = 0;
     for (long long u = u0; u < u1; ++seg) {
       const long long t = u / nk;
@@ -319,6 +349,14 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       const long long seg_end = (t + 1) * nk < u1 ? (t + 1) * nk : u1;
       const int kb_hi = static_cast<int>(seg_end - t * nk);
       u = seg_end;
+      const int m0 = static_cast<int>(t / n_tiles) * BN;
+      const int f0 = static_cast<int>(t % n_tiles) * RPT;
+      const int sb = (seg & 1) * BN;  // this segment's half of the scale buffers
+      if (et < BN) {  // requested before the accumulator wait, so the loads overlap it
+        const int m = m0 + et;
+        s_a[sb + et] = m < M ? __ldg(a_scale + m) : 0.0f;
+        s_rs[sb + et] = (U8 && m < M) ? __ldg(rowsum + m) : 0;
+      }
       const int b = seg & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[b], (seg >> 1) & 1))) break;
       tc_fence_after();
@@ -366,24 +404,50 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 #pragma unroll
           for (int j = 0; j < BN; ++j) v[j] += static_cast<uint32_t>(__ldcg(slot + j * kGemmBM + r));
         }
-        sk_epi_sync(epi_bar, ephase);
-        if (et == 0)
+        if (et == 0)  // every thread has read the partials once the next barrier completes
           for (int h = cta + 1; h <= last; ++h) flags[h] = 0u;  // all zero again for the next call
       }
-      // dequantise and store: thread = output feature n, columns = tokens
-      const int n = static_cast<int>(t) * kGemmBM + r;
-      if (n < N) {
+      sk_epi_sync(epi_bar, ephase);  // this segment's scales are in shared memory
+      if constexpr (GATE) {
+        // g of the tile's features through shared memory to the up quarters
+        const int f = f0 + (r & 63);
+        if (r >= 64) {
 #pragma unroll
-        for (int j = 0; j < BN; ++j) {
-          if (j < M) {
-            const int a = static_cast<int>(v[j]) - s_rs[j];
-            const int64_t o = static_cast<int64_t>(j) * N + n;
-            if (y_dtype == 2) {
-              static_cast<int32_t*>(y)[o] = a;
-            } else {
-              const float val = __fmul_rn(__fmul_rn(__int2float_rn(a), gamma), s_a[j]);
-              if (y_dtype == 0) static_cast<float*>(y)[o] = val;
-              else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(val);
+          for (int j = 0; j < BN; ++j) {
+            const int a = static_cast<int>(v[j]) - s_rs[sb + j];
+            gbuf[j * 64 + (r - 64)] = __fmul_rn(__fmul_rn(__int2float_rn(a), gamma), s_a[sb + j]);
+          }
+        }
+        sk_epi_sync(epi_bar, ephase);
+        if (r < 64 && f < N) {
+#pragma unroll
+          for (int j = 0; j < BN; ++j) {
+            if (m0 + j < M) {
+              const int a = static_cast<int>(v[j]) - s_rs[sb + j];
+              const float uu = __fmul_rn(__fmul_rn(__int2float_rn(a), gamma), s_a[sb + j]);
+              const float gg = gbuf[j * 64 + r];
+              const float rr = gg > 0.0f ? gg : 0.0f;
+              static_cast<__nv_bfloat16*>(y)[static_cast<int64_t>(m0 + j) * N + f] =
+                  __float2bfloat16_rn(__fmul_rn(__fmul_rn(rr, rr), uu));
+            }
+          }
+        }
+      } else {
+        // dequantise and store: thread = output feature n, columns = tokens
+        const int n = f0 + r;
+        if (n < N) {
+#pragma unroll
+          for (int j = 0; j < BN; ++j) {
+            if (m0 + j < M) {
+              const int a = static_cast<int>(v[j]) - s_rs[sb + j];
+              const int64_t o = static_cast<int64_t>(m0 + j) * N + n;
+              if (y_dtype == 2) {
+                static_cast<int32_t*>(y)[o] = a;
+              } else {
+                const float val = __fmul_rn(__fmul_rn(__int2float_rn(a), gamma), s_a[sb + j]);
+                if (y_dtype == 0) static_cast<float*>(y)[o] = val;
+                else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(val);
+              }
             }
           }
         }

@@ -147,34 +147,55 @@ size_t sk_workspace_bytes(int64_t M) {
   return sk_flag_bytes(G) + static_cast<size_t>(G) * sk_bn(M) * kGemmBM * 4;
 }
 
-template <int BN, bool U8>
-cudaError_t launch_sk(const CUtensorMap& mx, const CUtensorMap& mw, const float* gamma, const float* a,
-                      const int32_t* rs, int M, int N, int K, void* y, int yd, void* ws, cudaStream_t s) {
-  using C = SkCfg<BN>;
+template <int BN, bool U8, bool GATE>
+cudaError_t launch_sk(const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& mw2, const float* gamma,
+                      const float* gamma2, const float* a, const int32_t* rs, int M, int N, int K, void* y, int yd,
+                      void* ws, cudaStream_t s) {
+  using C = SkCfg<BN, GATE>;
   static std::atomic<bool> done[kMaxDevices] = {};
-  const cudaError_t e = set_smem(gemm_sk_kernel<BN, U8>, C::kSmemBytes, done);
+  auto kern = gemm_sk_kernel<BN, U8, GATE>;
+  const cudaError_t e = set_smem(kern, C::kSmemBytes, done);
   if (e != cudaSuccess) return e;
-  const int64_t units = static_cast<int64_t>((N + kGemmBM - 1) / kGemmBM) * ((K + kGemmBK - 1) / kGemmBK);
+  const int64_t units = static_cast<int64_t>((N + C::kRowsPerTile - 1) / C::kRowsPerTile) * ((M + BN - 1) / BN) *
+                        ((K + kGemmBK - 1) / kGemmBK);
   const int sms = sm_count();
   const int G = static_cast<int>(units < sms ? units : sms);
   unsigned int* flags = static_cast<unsigned int*>(ws);
   int* parts = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + sk_flag_bytes(sms));
-  return launch_pdl(gemm_sk_kernel<BN, U8>, dim3(G), dim3(kSkThreads), C::kSmemBytes, s, mx, mw, gamma, a, rs, M, N,
-                    K, y, yd, flags, parts);
+  return launch_pdl(kern, dim3(G), dim3(kSkThreads), C::kSmemBytes, s, mx, mw, mw2, gamma, gamma2, a, rs, M, N, K, y,
+                    yd, flags, parts);
+}
+
+// Tensor maps of a stream-K product: activations in 128-byte-wide boxes of BN
+// tokens (two per stage), packed codes in 64-byte-wide boxes of `rows` rows.
+template <int BN>
+bool sk_maps(const int8_t* xq, int M, int K, const uint8_t* Wp, int N, uint32_t rows, CUtensorMap* mx,
+             CUtensorMap* mw) {
+  return make_map_u8(mx, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(K), 128, BN,
+                     CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_map_u8(mw, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4),
+                     kGemmBK / 4, rows, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 template <int BN>
 cudaError_t launch_sk_bn(const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
                          const int32_t* rs, int M, void* y, int yd, void* ws, cudaStream_t s) {
   CUtensorMap mx, mw;
-  if (!make_map_u8(&mx, xq, static_cast<uint64_t>(K), static_cast<uint64_t>(M), static_cast<uint64_t>(K), 128, BN,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+  if (!sk_maps<BN>(xq, M, K, Wp, N, kGemmBM, &mx, &mw)) return cudaErrorInvalidValue;
+  if (rs != nullptr) return launch_sk<BN, true, false>(mx, mw, mw, gamma, gamma, a, rs, M, N, K, y, yd, ws, s);
+  return launch_sk<BN, false, false>(mx, mw, mw, gamma, gamma, a, rs, M, N, K, y, yd, ws, s);
+}
+
+// Up and gate projections with the squared-ReLU gate in the epilogue: h (bf16, M x F).
+template <int BN>
+cudaError_t launch_upgate_bn(const uint8_t* Wu, const float* gu, const uint8_t* Wg, const float* gg, int F, int K,
+                             const int8_t* xq, const float* a, const int32_t* rs, int M, void* h, void* ws,
+                             cudaStream_t s) {
+  CUtensorMap mx, mw, mw2, unused;
+  if (!sk_maps<BN>(xq, M, K, Wu, F, 64, &mx, &mw) || !sk_maps<BN>(xq, M, K, Wg, F, 64, &unused, &mw2))
     return cudaErrorInvalidValue;
-  if (!make_map_u8(&mw, Wp, static_cast<uint64_t>(K / 4), static_cast<uint64_t>(N), static_cast<uint64_t>(K / 4),
-                   kGemmBK / 4, kGemmBM, CU_TENSOR_MAP_SWIZZLE_64B))
-    return cudaErrorInvalidValue;
-  if (rs != nullptr) return launch_sk<BN, true>(mx, mw, gamma, a, rs, M, N, K, y, yd, ws, s);
-  return launch_sk<BN, false>(mx, mw, gamma, a, rs, M, N, K, y, yd, ws, s);
+  if (rs != nullptr) return launch_sk<BN, true, true>(mx, mw, mw2, gu, gg, a, rs, M, F, K, h, 1, ws, s);
+  return launch_sk<BN, false, true>(mx, mw, mw2, gu, gg, a, rs, M, F, K, h, 1, ws, s);
 }
 
 }  // namespace
@@ -182,6 +203,33 @@ cudaError_t launch_sk_bn(const uint8_t* Wp, const float* gamma, int N, int K, co
 BITNET_DEFINE_TAKE_ERROR(gemm)
 
 extern "C" {
+
+size_t bitnet_linear_upgate_workspace_bytes(int64_t M, int64_t F, int64_t K) {
+  if (M < 1 || M > INT32_MAX || F < 1 || F > INT32_MAX || !valid_k(K)) return 0;
+  return sk_workspace_bytes(M);
+}
+
+bitnet_status bitnet_linear_upgate_gemm(const uint8_t* W_up, const float* gamma_up, const uint8_t* W_gate,
+                                        const float* gamma_gate, int64_t F, int64_t K, const int8_t* x_q,
+                                        const float* a_scale, const int32_t* x_rowsum, int64_t M, void* h,
+                                        void* workspace, size_t workspace_bytes, void* stream) {
+  if (W_up == nullptr || gamma_up == nullptr || W_gate == nullptr || gamma_gate == nullptr || x_q == nullptr ||
+      a_scale == nullptr || h == nullptr || workspace == nullptr)
+    return BITNET_ERR_INVALID_ARG;
+  if (!aligned(W_up, 16) || !aligned(W_gate, 16) || !aligned(x_q, 16) || !aligned(h, 16) || !aligned(workspace, 16) ||
+      !aligned(gamma_up, 4) || !aligned(gamma_gate, 4) || !aligned(a_scale, 4) || !aligned(x_rowsum, 4))
+    return BITNET_ERR_INVALID_ARG;
+  if (!valid_k(K) || F < 1 || F > INT32_MAX || M < 1 || M > INT32_MAX || K > INT32_MAX)
+    return BITNET_ERR_UNSUPPORTED_SHAPE;
+  if (workspace_bytes < sk_workspace_bytes(M)) return BITNET_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int f = static_cast<int>(F), k = static_cast<int>(K), m = static_cast<int>(M);
+  cudaError_t e;
+  if (m <= 16) e = launch_upgate_bn<16>(W_up, gamma_up, W_gate, gamma_gate, f, k, x_q, a_scale, x_rowsum, m, h, workspace, s);
+  else if (m <= 32) e = launch_upgate_bn<32>(W_up, gamma_up, W_gate, gamma_gate, f, k, x_q, a_scale, x_rowsum, m, h, workspace, s);
+  else e = launch_upgate_bn<64>(W_up, gamma_up, W_gate, gamma_gate, f, k, x_q, a_scale, x_rowsum, m, h, workspace, s);
+  return from_cuda(e);
+}
 
 size_t bitnet_linear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   if (M < 1 || M > 64 || N < 1 || N > INT32_MAX || !valid_k(K)) return 0;

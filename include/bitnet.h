@@ -25,8 +25,8 @@
  *   - Errors are returned as bitnet_status; nothing is launched when an
  *     argument is rejected.  No C++ exception crosses this boundary.
  *   - The product entry points (bitnet_linear_gemv, bitnet_linear_gemm,
- *     bitnet_bitlinear_gemv, bitnet_bitlinear_ffn_gemv,
- *     bitnet_bitlinear_gemv_b3) are launched with programmatic dependent
+ *     bitnet_linear_upgate_gemm, bitnet_bitlinear_gemv,
+ *     bitnet_bitlinear_ffn_gemv, bitnet_bitlinear_gemv_b3) are launched with programmatic dependent
  *     launch: they start while the previous kernel on the stream finishes,
  *     and request their first packed-weight tiles BEFORE waiting for it
  *     (the weights of a layer never depend on the layer before).  So the
@@ -227,6 +227,43 @@ bitnet_status bitnet_linear_gemm(const uint8_t* W_packed, const float* gamma, in
                                  const int8_t* x_q, const float* a_scale, const int32_t* x_rowsum,
                                  int64_t M, void* y, int y_dtype, void* workspace, size_t workspace_bytes,
                                  void* stream);
+
+/*
+ * Bytes of workspace bitnet_linear_upgate_gemm uses on the CURRENT device
+ * (a flag per SM and one partial int32 tile of 128 rows x 16, 32 or 64
+ * tokens per SM); 0 for an invalid shape.
+ */
+size_t bitnet_linear_upgate_workspace_bytes(int64_t M, int64_t F, int64_t K);
+
+/*
+ * The feed-forward block's up and gate BitLinear products with the
+ * squared-ReLU gate in their epilogue (inferownia.pl, "BitNet b1.58: era
+ * 1-bitowych LLM-ów", section "Zrób to sam": squared ReLU in the FFN;
+ * kripta.biz 2B4T news: ReLU^2 in the FFN layers), for any M, on the
+ * tensor cores (the stream-K product of bitnet_linear_gemm: a 128-row tile
+ * holds the up and the gate rows of 64 features, so one epilogue sees both):
+ *
+ *   u[m][f] = RN32(RN32(float(acc_up[m][f])   * gamma_up)   * a_scale[m])
+ *   g[m][f] = RN32(RN32(float(acc_gate[m][f]) * gamma_gate) * a_scale[m])
+ *   r = g if g > 0 else +0;   h[m][f] = bf16(RN32(RN32(r * r) * u))
+ *
+ * (acc as in bitnet_linear_gemv).  u and g never reach memory; h is the
+ * down projection's bf16 input (quantise it with bitnet_quant_act, with the
+ * sub-layer norm's gain, then bitnet_linear_gemm).
+ *
+ * W_up, W_gate     [in]  F x K/4 packed bytes each (bitnet_pack_weights).
+ * gamma_up/gate    [in]  their fp32 scales (device).
+ * x_q, a_scale, x_rowsum [in]  the quantised block input, as bitnet_linear_gemm.
+ * h                [out] M x F bf16.
+ * workspace        [in,out] at least bitnet_linear_upgate_workspace_bytes(M, F,
+ *                  K) bytes, 16-byte aligned, zeroed before its first use;
+ *                  same rules as bitnet_linear_gemm's workspace (required).
+ * Asynchronous.
+ */
+bitnet_status bitnet_linear_upgate_gemm(const uint8_t* W_up, const float* gamma_up, const uint8_t* W_gate,
+                                        const float* gamma_gate, int64_t F, int64_t K, const int8_t* x_q,
+                                        const float* a_scale, const int32_t* x_rowsum, int64_t M, void* h,
+                                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Fused decode BitLinear: bitnet_quant_act followed by bitnet_linear_gemv in

@@ -128,6 +128,26 @@ def test_gemm_workspace_bytes(L):
     assert per_sm_16 >= 16 * 128 * 4
 
 
+def test_upgate_rejects_bad_arguments(L):
+    need = bl.bitnet_linear_upgate_workspace_bytes(64, 128, 256)
+    assert need == bl.bitnet_linear_gemm_workspace_bytes(64, 128, 256) and need > 0
+    assert bl.bitnet_linear_upgate_workspace_bytes(2048, 128, 256) == need      # token tiles of 64 at any M
+    assert bl.bitnet_linear_upgate_workspace_bytes(4, 128, 100) == 0
+
+    def call(Wu=FAKE, gu=FAKE, Wg=FAKE, gg=FAKE, F=128, K=256, xq=FAKE, a=FAKE, rs=None, M=4, h=FAKE, ws=FAKE,
+             wsb=1 << 24):
+        return L.bitnet_linear_upgate_gemm(Wu, gu, Wg, gg, F, K, xq, a, rs, M, h, ws, wsb, None)
+
+    for kw in ({"Wu": None}, {"gg": None}, {"xq": None}, {"h": None}, {"ws": None}):
+        assert call(**kw) == bl.BITNET_ERR_INVALID_ARG, kw
+    for kw in ({"Wg": MIS}, {"h": MIS}, {"ws": MIS}, {"gu": FAKE + 2}, {"rs": FAKE + 1}):
+        assert call(**kw) == bl.BITNET_ERR_INVALID_ARG, kw
+    assert call(wsb=16) == bl.BITNET_ERR_INVALID_ARG
+    assert call(K=96) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(F=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(M=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+
+
 def test_fused_rejects_bad_arguments(L):
     def call(x=FAKE, dt=bl.BITNET_BF16, g=None, eps=1e-5, W=FAKE, gam=FAKE, N=8, K=64, M=1, y=FAKE,
              yd=bl.BITNET_BF16):

@@ -504,3 +504,49 @@ def test_gemm_stream_k_in_a_cuda_graph(dev, orc):
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     assert int(ws[:4 * sms].view(torch.int32).abs().sum()) == 0
     assert bl.bitnet_get_device_status() == bl.BITNET_OK
+
+
+# --------------------------------------------------------------------------- FFN up|gate with the squared-ReLU gate
+
+UPGATE_CASES = [(64, 6912, 2560, False), (5, 200, 320, True), (16, 21504, 5376, False), (33, 777, 1344, True),
+                (2048, 6912, 2560, False)]
+
+
+@pytest.mark.parametrize("M,F,K,signed", UPGATE_CASES)
+def test_upgate_gemm_matches_oracle_ffn_gate(dev, orc, M, F, K, signed):
+    """h = bf16(relu(g)^2 u) from one tensor-core product of the up and gate
+    weights, against the oracle's BitLinears and squared-ReLU gate (bit-exact;
+    sampled at M = 2048)."""
+    import torch
+    W_up = synth.weights(F, K, 0.02, 3, 31)
+    W_gate = synth.weights(F, K, 0.02, 3, 32)
+    x = synth.activations(M, K, 3, 33, "normal", 0.01, 20.0, "bf16")
+    g_in = synth.gain(K, 3, 34, "bf16")
+    pu, gu = orc.pack_weights(W_up, EPS_W)
+    pg, gg = orc.pack_weights(W_gate, EPS_W)
+    xq_r, a_r, _ = orc.quant_act(x, g_in, EPS_RMS)
+    Pu, Gu = bl.bitnet_pack_weights(_t(W_up, dev), EPS_W)
+    Pg, Gg = bl.bitnet_pack_weights(_t(W_gate, dev), EPS_W)
+    xq, a, rs = bl.bitnet_quant_act(_x_dev(x, "bf16", dev), _x_dev(g_in, "bf16", dev), EPS_RMS, want_rowsum=True)
+    assert np.array_equal(xq.cpu().numpy(), xq_r)
+    ws = torch.zeros(bl.bitnet_linear_upgate_workspace_bytes(M, F, K), dtype=torch.uint8, device=dev)
+    h = bl.bitnet_linear_upgate_gemm(Pu, Gu, Pg, Gg, xq, a, None if signed else rs, workspace=ws)
+    hb = h.view(torch.int16).cpu().numpy().view(np.uint16)
+    if M * F <= 64 * 21504:
+        _, u = orc.bitlinear(pu, gu, K, xq_r, a_r)
+        _, g = orc.bitlinear(pg, gg, K, xq_r, a_r)
+        np.testing.assert_array_equal(hb, orc.f32_to_bf16(orc.relu2_gate(u, g)))
+    else:
+        rng = np.random.default_rng(0)
+        ms, ns = rng.integers(0, M, 4000), rng.integers(0, F, 4000)
+        _, u = orc.bitlinear_sampled(pu, gu, K, xq_r, a_r, ms, ns)
+        _, g = orc.bitlinear_sampled(pg, gg, K, xq_r, a_r, ms, ns)
+        np.testing.assert_array_equal(hb[ms, ns], orc.f32_to_bf16(orc.relu2_gate(u, g)))
+    # the same h from the two separate products and the oracle's gate on their outputs
+    u_d = bl.bitnet_linear_gemm(Pu, Gu, xq, a, rs, out_dtype=torch.float32)
+    g_d = bl.bitnet_linear_gemm(Pg, Gg, xq, a, rs, out_dtype=torch.float32)
+    ref = orc.f32_to_bf16(orc.relu2_gate(u_d.cpu().numpy(), g_d.cpu().numpy()))
+    np.testing.assert_array_equal(hb, ref)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    assert int(ws[:4 * sms].view(torch.int32).abs().sum()) == 0
+    assert bl.bitnet_get_device_status() == bl.BITNET_OK
