@@ -385,25 +385,27 @@ def run_reference(args, lins, rank: int):
 # ----------------------------------------------------------------------------- GPU arm
 
 class Workload:
-    """Device state of one workload: packed weights (rotated copies), inputs,
-    output buffers, and the launches of one step."""
+    """Device state of one workload: packed weights and, per linear, its input,
+    quantised input and output buffers, all in `copies` rotated copies (one
+    rotation over three times the 126 MB L2), and the launches of one step."""
 
-    def __init__(self, torch, bl, dev, lins, packs, rotate: bool):
+    def __init__(self, torch, bl, dev, lins, packs, rotate: bool = True):
         self.torch, self.bl, self.dev, self.lins = torch, bl, dev, lins
-        wbytes = sum(l.N * l.K // 4 for l in lins)
-        self.copies = max(2, min(MAX_COPIES, math.ceil(3 * L2_BYTES / wbytes))) if rotate else 1
+        per_step = sum(linear_bytes(l)["quant"] + linear_bytes(l)["product"] for l in lins)
+        self.copies = max(2, min(MAX_COPIES, math.ceil(3 * L2_BYTES / per_step))) if rotate else 1
         self.packs = [packs.get(torch, bl, dev, l, self.copies) for l in lins]
         self.xs, self.gains, self.bufs = [], [], []
         for lin in lins:
-            self.xs.append(self._act(lin.make_x(0), lin.x_dtype))
+            x0 = self._act(lin.make_x(0), lin.x_dtype)
+            self.xs.append([x0] + [x0.clone() for _ in range(self.copies - 1)])
             g = lin.make_gain(0)
             self.gains.append(None if g is None else self._act(g, lin.x_dtype))
             ydt = torch.bfloat16 if lin.y_dtype == "bf16" else torch.float32
-            self.bufs.append({
+            self.bufs.append([{
                 "xq": torch.empty((lin.M, lin.K), dtype=torch.int8, device=dev),
                 "a": torch.empty(lin.M, dtype=torch.float32, device=dev),
                 "rs": torch.empty(lin.M, dtype=torch.int32, device=dev),
-                "y": torch.empty((lin.M, lin.N), dtype=ydt, device=dev)})
+                "y": torch.empty((lin.M, lin.N), dtype=ydt, device=dev)} for _ in range(self.copies)])
         # one GEMM workspace for the whole step (its calls run one after another on one stream)
         wsb = max([bl.bitnet_linear_gemm_workspace_bytes(l.M, l.N, l.K) for l in lins if l.M > 8] or [0])
         self.ws = torch.zeros(wsb, dtype=torch.uint8, device=dev) if wsb else None
@@ -414,18 +416,28 @@ class Workload:
                                "gemm_sk_kernel (tcgen05 stream-K, bitnet_linear_gemm)" if all(l.M <= 64 for l in lins)
                                else "gemm_kernel (tcgen05, bitnet_linear_gemm)")
 
+    @property
+    def footprint_mb(self) -> float:
+        return self.copies * sum(linear_bytes(l)["quant"] + linear_bytes(l)["product"] for l in self.lins) / 1e6
+
     def _act(self, a, dtype):
         torch = self.torch
         if dtype == "bf16":
             return torch.from_numpy(synth.f32_to_bf16_bits(a).view(np.int16).copy()).to(self.dev).view(torch.bfloat16)
         return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(self.dev)
 
-    def quant(self, i, _c):
-        b = self.bufs[i]
-        self.bl.bitnet_quant_act(self.xs[i], self.gains[i], EPS_RMS, b["xq"], b["a"], b["rs"])
+    def x(self, i, c):
+        return self.xs[i][c % self.copies]
+
+    def buf(self, i, c):
+        return self.bufs[i][c % self.copies]
+
+    def quant(self, i, c):
+        b = self.buf(i, c)
+        self.bl.bitnet_quant_act(self.x(i, c), self.gains[i], EPS_RMS, b["xq"], b["a"], b["rs"])
 
     def product(self, i, c):
-        lin, b = self.lins[i], self.bufs[i]
+        lin, b = self.lins[i], self.buf(i, c)
         if lin.M <= 8:
             self.bl.bitnet_linear_gemv(self.packs[i][0][c % self.copies], self.packs[i][1], b["xq"], b["a"],
                                        b["rs"], y=b["y"])
@@ -434,8 +446,8 @@ class Workload:
                                        b["rs"], y=b["y"], workspace=self.ws)
 
     def fused_linear(self, i, c):
-        self.bl.bitnet_bitlinear_gemv(self.xs[i], self.packs[i][0][c % self.copies], self.packs[i][1],
-                                      self.gains[i], EPS_RMS, y=self.bufs[i]["y"])
+        self.bl.bitnet_bitlinear_gemv(self.x(i, c), self.packs[i][0][c % self.copies], self.packs[i][1],
+                                      self.gains[i], EPS_RMS, y=self.buf(i, c)["y"])
 
     def linear(self, i, c):
         if self.fused:
@@ -526,25 +538,32 @@ def measure_rotating(torch, bl, dev, stream, wl, peaks, peak_src, group, steps=G
     per = []
     for i, lin in enumerate(lins):
         prod = wl.fused_linear if wl.fused else wl.product
-        pms = per_launch_ms(torch, dev, stream, wl, prod, i, group=group)
-        qms = None if wl.fused else per_launch_ms(torch, dev, stream, wl, wl.quant, i, group=group)
+        pms = per_launch_ms(torch, dev, stream, wl, prod, i, steps=steps, replays=max(2, replays // 2), group=group)
+        qms = None if wl.fused else per_launch_ms(torch, dev, stream, wl, wl.quant, i, steps=steps,
+                                                  replays=max(2, replays // 2), group=group)
+        qb = linear_bytes(lin)["quant"]
         per.append({"linear": lin.name, "M": lin.M, "K": lin.K, "N": lin.N, "product_us": pms * 1e3,
-                    "quant_us": None if qms is None else qms * 1e3})
+                    "product_tops": lin.ops / (pms / 1e3) / 1e12,
+                    "quant_us": None if qms is None else qms * 1e3,
+                    "quant_gbs": None if qms is None else qb / (qms / 1e3) / 1e9,
+                    "quant_frac": None if qms is None else qb / (qms / 1e3) / 1e9 / float(peaks["hbm_gbs"])})
     kbytes = sum(linear_bytes(l)["fused" if wl.fused else "product"] for l in lins)
     ksec = sum(p["product_us"] for p in per) * 1e-6
     rl = roofline(wl.product_kernel, kbytes, step_ops(lins), ksec, peaks, peak_src,
                   "each linear's product kernel alone, back to back in CUDA graphs over the rotating weight copies, "
                   "CUDA events on the launching stream; bytes and time summed over the linears", launches=len(lins))
-    return {"ms_per_step": ms, "per_linear": per, "roofline": rl, "weight_copies": wl.copies,
+    return {"ms_per_step": ms, "per_linear": per, "roofline": rl, "copies": wl.copies,
             "device_status": bl.bitnet_get_device_status(),
-            "timing": f"CUDA graphs of {steps} steps over {wl.copies} rotating weight copies, {replays} replays "
-                      "after one untimed replay, CUDA events"}
+            "timing": f"CUDA graphs of {steps} steps back to back over {wl.copies} rotated copies of every buffer "
+                      f"({wl.footprint_mb:.0f} MB per rotation > 3 x 126 MB L2), {replays} replays after one untimed "
+                      "replay, CUDA events"}
 
 
 def measure_flushed(torch, bl, dev, stream, wl, peaks, peak_src, group, reps=10) -> dict:
-    """A prefill-sized configuration: each step with the L2 flushed (256 MB
-    write) before it; CUDA events around every kernel; medians of reps steps
-    after 3 untimed ones."""
+    """Single cold steps: each step with the L2 flushed (256 MB write) before
+    it; CUDA events around every kernel; medians of reps steps after 3
+    untimed ones.  (The write-back of the flush's dirty lines lands on the
+    first kernel, so this is a pessimistic figure.)"""
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     lins = wl.lins
     qt = [[] for _ in lins]
@@ -672,8 +691,8 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
     # ------------------------------------------------------------------ end to end through the public API
     h2d = sum(linear_bytes(l)["x_in"] for l in lins)
     d2h = sum(linear_bytes(l)["y_out"] for l in lins)
-    xs_host = [x.cpu().pin_memory() for x in wl.xs]
-    ys_host = [torch.empty_like(b["y"], device="cpu").pin_memory() for b in wl.bufs]
+    xs_host = [wl.x(i, 0).cpu().pin_memory() for i in range(len(lins))]
+    ys_host = [torch.empty_like(wl.buf(i, 0)["y"], device="cpu").pin_memory() for i in range(len(lins))]
     k_e2e = min(max(K, 200), 2000)
 
     def e2e_loop(n, copies=True, calls=True):
@@ -686,11 +705,11 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
             for c in range(n):
                 for i in range(len(lins)):
                     if copies:
-                        wl.xs[i].copy_(xs_host[i], non_blocking=True)
+                        wl.x(i, c).copy_(xs_host[i], non_blocking=True)
                     if calls:
                         wl.linear(i, c)
                     if copies:
-                        ys_host[i].copy_(wl.bufs[i]["y"], non_blocking=True)
+                        ys_host[i].copy_(wl.buf(i, c)["y"], non_blocking=True)
             b.record(stream)
             torch.cuda.synchronize(dev)
             host_ms = (time.perf_counter() - t0) * 1e3
@@ -747,8 +766,8 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
                        "step": ("per linear: one bitnet_bitlinear_gemv kernel (RMSNorm/absmax int8 quantisation of "
                                 "the input fused with the ternary GEMV and dequant)") if wl.fused else
                                "per linear: bitnet_quant_act + ternary product with dequant",
-                       "l2": f"{wl.copies} rotating packed-weight copies per linear "
-                             f"({wl.copies * sum(l.N * l.K // 4 for l in lins) / 1e6:.0f} MB > 126 MB L2)",
+                       "l2": f"{wl.copies} rotated copies of every buffer ({wl.footprint_mb:.0f} MB per rotation "
+                             "> 3 x 126 MB L2): inputs larger than L2, no flush",
                        "timing": f"CUDA graphs of {G} steps, programmatic dependent launch between kernels; every "
                                  "graph of the timed region replayed during the warm-up",
                        "parallelism": "replicas" if ws > 1 else "single"},
@@ -776,12 +795,17 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
 
 def bench_config(torch, bl, dev, stream, name, packs, peaks, peak_src, group, with_cpu, cpu_seconds) -> dict:
     """One configuration of the benchmark set: its step time, value in its unit,
-    the roofline of its product kernel and the CPU oracle beside it."""
+    the roofline of its product kernel and the CPU oracle beside it.  Steps run
+    back to back over rotated copies of every buffer; large batches also get
+    single cold steps after an L2 flush ("cold")."""
     lins = synth.WORKLOADS[name]
     unit = config_unit(lins, peaks)
     big = any(l.M >= 256 for l in lins)
-    wl = Workload(torch, bl, dev, lins, packs, rotate=not big)
-    m = (measure_flushed if big else measure_rotating)(torch, bl, dev, stream, wl, peaks, peak_src, group)
+    wl = Workload(torch, bl, dev, lins, packs)
+    m = measure_rotating(torch, bl, dev, stream, wl, peaks, peak_src, group, steps=16 if big else GRAPH_STEPS,
+                         replays=5 if big else 20)
+    if big:
+        m["cold"] = measure_flushed(torch, bl, dev, stream, wl, peaks, peak_src, group)
     sec = m["ms_per_step"] / 1e3
     value = step_ops(lins) / sec / 1e12 if unit == "TOPS" else step_bytes(lins) / sec / 1e9
     out = {"workload": name, "linears": [[l.M, l.K, l.N] for l in lins], "value": value, "unit": unit,
@@ -805,12 +829,10 @@ def bench_b3(torch, bl, dev, stream, wl, peaks, group, two_bit_step_ms):
         P, G = bl.bitnet_pack_weights_b3(W, EPS_W)
         del W
         packs.append(([P] + [P.clone() for _ in range(wl.copies - 1)], G))
-    ys = [torch.empty_like(b["y"]) for b in wl.bufs]
-
     def step(c):
         for i in range(len(lins)):
-            bl.bitnet_bitlinear_gemv_b3(wl.xs[i], packs[i][0][c % wl.copies], packs[i][1], wl.gains[i], EPS_RMS,
-                                        y=ys[i])
+            bl.bitnet_bitlinear_gemv_b3(wl.x(i, c), packs[i][0][c % wl.copies], packs[i][1], wl.gains[i], EPS_RMS,
+                                        y=wl.buf(i, c)["y"])
 
     g = capture(torch, stream, step, GRAPH_STEPS)
     with torch.cuda.stream(stream):
