@@ -216,7 +216,11 @@ size_t bitnet_linear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *           rest is scratch that every call overwrites before reading).  Two calls that may run at the same time (on two
  *           streams) must not share a workspace.  If a call reports
  *           BITNET_ERR_TIMEOUT through bitnet_get_device_status, zero the
- *           workspace again before reusing it.  Without a workspace (NULL,
+ *           workspace again before reusing it.  The stream-K launch
+ *           has one CTA per SM and its CTAs wait on one another (bounded
+ *           waits), so it needs all the device's SMs to be available to it at
+ *           once: where the process gets only part of the GPU (an MPS limit
+ *           on active SMs), pass no workspace.  Without a workspace (NULL,
  *           with workspace_bytes ignored) or for M > 64, the product runs on
  *           persistent tiles, split over thread-block clusters when there
  *           are few tiles; the results are identical.
