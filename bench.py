@@ -406,15 +406,27 @@ class Workload:
                 "a": torch.empty(lin.M, dtype=torch.float32, device=dev),
                 "rs": torch.empty(lin.M, dtype=torch.int32, device=dev),
                 "y": torch.empty((lin.M, lin.N), dtype=ydt, device=dev)} for _ in range(self.copies)])
-        # one GEMM workspace for the whole step (its calls run one after another on one stream)
-        wsb = max([bl.bitnet_linear_gemm_workspace_bytes(l.M, l.N, l.K) for l in lins if l.M > 8] or [0])
+        # the path of a step: one fused kernel per linear for decode-sized batches, else quantisation + product
+        kmax = lambda l: 32768 if l.x_dtype == "bf16" else 16384
+        if all(l.M <= 8 and l.M * l.K <= 21504 for l in lins):
+            self.path = "gemv_fused"
+        elif all(l.M <= 64 and l.K <= kmax(l) for l in lins):
+            self.path = "gemm_fused"
+        else:
+            self.path = "quant_gemv" if all(l.M <= 8 for l in lins) else "quant_gemm"
+        self.fused = self.path.endswith("_fused")
+        # one workspace for the whole step (its calls run one after another on one stream)
+        wsb = max([bl.bitnet_linear_gemm_workspace_bytes(l.M, l.N, l.K) for l in lins if l.M > 8] +
+                  [bl.bitnet_bitlinear_gemm_workspace_bytes(l.M, l.N, l.K) for l in lins
+                   if self.path == "gemm_fused"] or [0])
         self.ws = torch.zeros(wsb, dtype=torch.uint8, device=dev) if wsb else None
-        self.fused = all(l.M <= 8 and l.M * l.K <= 21504 for l in lins)
         self.kernels_per_step = (1 if self.fused else 2) * len(lins)
-        self.product_kernel = ("gemv_kernel (fused quantisation + GEMV, bitnet_bitlinear_gemv)" if self.fused else
-                               "gemv_kernel (bitnet_linear_gemv)" if all(l.M <= 8 for l in lins) else
-                               "gemm_sk_kernel (tcgen05 stream-K, bitnet_linear_gemm)" if all(l.M <= 64 for l in lins)
-                               else "gemm_kernel (tcgen05, bitnet_linear_gemm)")
+        self.product_kernel = {
+            "gemv_fused": "gemv_kernel (fused quantisation + GEMV, bitnet_bitlinear_gemv)",
+            "gemm_fused": "gemm_sk_kernel (fused quantisation + tcgen05 stream-K, bitnet_bitlinear_gemm)",
+            "quant_gemv": "gemv_kernel (bitnet_linear_gemv)",
+            "quant_gemm": ("gemm_sk_kernel (tcgen05 stream-K, bitnet_linear_gemm)" if all(l.M <= 64 for l in lins)
+                           else "gemm_kernel (tcgen05, bitnet_linear_gemm)")}[self.path]
 
     @property
     def footprint_mb(self) -> float:
@@ -446,8 +458,12 @@ class Workload:
                                        b["rs"], y=b["y"], workspace=self.ws)
 
     def fused_linear(self, i, c):
-        self.bl.bitnet_bitlinear_gemv(self.x(i, c), self.packs[i][0][c % self.copies], self.packs[i][1],
-                                      self.gains[i], EPS_RMS, y=self.buf(i, c)["y"])
+        if self.path == "gemv_fused":
+            self.bl.bitnet_bitlinear_gemv(self.x(i, c), self.packs[i][0][c % self.copies], self.packs[i][1],
+                                          self.gains[i], EPS_RMS, y=self.buf(i, c)["y"])
+        else:
+            self.bl.bitnet_bitlinear_gemm(self.x(i, c), self.packs[i][0][c % self.copies], self.packs[i][1],
+                                          self.gains[i], EPS_RMS, y=self.buf(i, c)["y"], workspace=self.ws)
 
     def linear(self, i, c):
         if self.fused:
@@ -552,7 +568,18 @@ def measure_rotating(torch, bl, dev, stream, wl, peaks, peak_src, group, steps=G
     rl = roofline(wl.product_kernel, kbytes, step_ops(lins), ksec, peaks, peak_src,
                   "each linear's product kernel alone, back to back in CUDA graphs over the rotating weight copies, "
                   "CUDA events on the launching stream; bytes and time summed over the linears", launches=len(lins))
-    return {"ms_per_step": ms, "per_linear": per, "roofline": rl, "copies": wl.copies,
+    unfused = None
+    if wl.fused:
+        # the same steps as two kernels per linear (quantisation, then the product)
+        gu = capture(torch, stream, wl.step_unfused, steps)
+        with torch.cuda.stream(stream):
+            gu.replay()
+        torch.cuda.synchronize(dev)
+        ums = replay_ms(torch, dev, stream, gu, replays, group) / (steps * replays)
+        del gu
+        unfused = {"ms_per_step": ums, "kernels_per_step": 2 * len(lins),
+                   "what": "bitnet_quant_act + the product per linear (two kernels)"}
+    return {"ms_per_step": ms, "per_linear": per, "roofline": rl, "copies": wl.copies, "unfused_step": unfused,
             "device_status": bl.bitnet_get_device_status(),
             "timing": f"CUDA graphs of {steps} steps back to back over {wl.copies} rotated copies of every buffer "
                       f"({wl.footprint_mb:.0f} MB per rotation > 3 x 126 MB L2), {replays} replays after one untimed "
@@ -676,17 +703,9 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
     if wl.fused and lins[0].K == 5376 and lins[0].N == 21504:
         rl["traffic"] = profiled_traffic(os.path.join(PROFILES, "gemv_decode_m1_27b_ffn.md"),
                                          kernel_source_hash(["gemv.cuh", "quant.cuh", "ptx.cuh"]))
-    unfused = None
-    if wl.fused:
-        gu = capture(torch, stream, wl.step_unfused, GRAPH_STEPS)
-        with torch.cuda.stream(stream):
-            gu.replay()
-        torch.cuda.synchronize(dev)
-        ms = replay_ms(torch, dev, stream, gu, 10, group) / (10 * GRAPH_STEPS)
-        del gu
-        unfused = {"value": ws * sbytes / (ms / 1e3) / 1e9, "unit": "GB/s", "ms_per_step": ms,
-                   "kernels_per_step": 2 * len(lins),
-                   "what": "bitnet_quant_act + bitnet_linear_gemv per linear (two kernels)"}
+    unfused = head.get("unfused_step")
+    if unfused is not None:
+        unfused = dict(unfused, value=ws * sbytes / (unfused["ms_per_step"] / 1e3) / 1e9, unit="GB/s")
 
     # ------------------------------------------------------------------ end to end through the public API
     h2d = sum(linear_bytes(l)["x_in"] for l in lins)
@@ -746,7 +765,7 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
         ffn_block = {n: bench_ffn_block(torch, bl, dev, stream, peaks, peak_src, group, n)
                      for n in ("ffn_block_m1_27b", "ffn_block_m1_2p5b")}
     decode_b3 = None
-    if not args.no_b3 and wl.fused and all(l.M * ((l.K + 79) // 80 * 80) <= 24000 for l in lins):
+    if not args.no_b3 and wl.path == "gemv_fused" and all(l.M * ((l.K + 79) // 80 * 80) <= 24000 for l in lins):
         decode_b3 = bench_b3(torch, bl, dev, stream, wl, peaks, group, el_ms / K)
     ste = None
     if not args.no_ste:
@@ -763,9 +782,11 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
             "warmup_steps_run": warm_steps, "ms_per_step": el_ms / K, "step_percentiles": step_stats,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
             "config": {"workload": args.workload, "linears": [[l.M, l.K, l.N] for l in lins],
-                       "step": ("per linear: one bitnet_bitlinear_gemv kernel (RMSNorm/absmax int8 quantisation of "
-                                "the input fused with the ternary GEMV and dequant)") if wl.fused else
-                               "per linear: bitnet_quant_act + ternary product with dequant",
+                       "step": {"gemv_fused": "per linear: one bitnet_bitlinear_gemv kernel (RMSNorm/absmax int8 "
+                                              "quantisation of the input fused with the ternary GEMV and dequant)",
+                                "gemm_fused": "per linear: one bitnet_bitlinear_gemm kernel (quantisation fused with "
+                                              "the stream-K tensor-core product and dequant)"}.get(
+                                    wl.path, "per linear: bitnet_quant_act + ternary product with dequant"),
                        "l2": f"{wl.copies} rotated copies of every buffer ({wl.footprint_mb:.0f} MB per rotation "
                              "> 3 x 126 MB L2): inputs larger than L2, no flush",
                        "timing": f"CUDA graphs of {G} steps, programmatic dependent launch between kernels; every "
@@ -810,8 +831,7 @@ def bench_config(torch, bl, dev, stream, name, packs, peaks, peak_src, group, wi
     value = step_ops(lins) / sec / 1e12 if unit == "TOPS" else step_bytes(lins) / sec / 1e9
     out = {"workload": name, "linears": [[l.M, l.K, l.N] for l in lins], "value": value, "unit": unit,
            "us_per_step": m["ms_per_step"] * 1e3, "kernels_per_step": wl.kernels_per_step,
-           "path": "fused decode GEMV" if wl.fused else ("quant + GEMV" if all(l.M <= 8 for l in lins)
-                                                         else "quant + tcgen05 GEMM"), **m}
+           "path": wl.path, **m}
     del wl
     torch.cuda.empty_cache()
     if with_cpu:

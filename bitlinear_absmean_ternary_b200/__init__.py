@@ -60,6 +60,10 @@ def lib() -> ctypes.CDLL:
         L.bitnet_linear_gemm.restype = I
         L.bitnet_linear_gemm_workspace_bytes.argtypes = [I64, I64, I64]
         L.bitnet_linear_gemm_workspace_bytes.restype = ctypes.c_size_t
+        L.bitnet_bitlinear_gemm_workspace_bytes.argtypes = [I64, I64, I64]
+        L.bitnet_bitlinear_gemm_workspace_bytes.restype = ctypes.c_size_t
+        L.bitnet_bitlinear_gemm.argtypes = [P, I, P, F, P, P, I64, I64, I64, P, I, P, ctypes.c_size_t, P]
+        L.bitnet_bitlinear_gemm.restype = I
         L.bitnet_linear_upgate_workspace_bytes.argtypes = [I64, I64, I64]
         L.bitnet_linear_upgate_workspace_bytes.restype = ctypes.c_size_t
         L.bitnet_linear_upgate_gemm.argtypes = [P, P, P, P, I64, I64, P, P, P, I64, P, P, ctypes.c_size_t, P]
@@ -317,6 +321,36 @@ def bitnet_bitlinear_gemv(x, W_packed, gamma, rms_gain=None, rms_eps: float = 1e
     return y
 
 
+def bitnet_bitlinear_gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    """Workspace bytes of bitnet_bitlinear_gemm on the current device (0 outside M = 1..64)."""
+    return int(lib().bitnet_bitlinear_gemm_workspace_bytes(M, N, K))
+
+
+def bitnet_bitlinear_gemm(x, W_packed, gamma, rms_gain=None, rms_eps: float = 1e-5, y=None, out_dtype=None,
+                          workspace=None):
+    """Fused BitLinear for 1 <= M <= 64 tokens: quantisation (with RMSNorm when
+    rms_gain is given) and the stream-K tensor-core product in one launch.
+    workspace: zeroed uint8 device tensor of bitnet_bitlinear_gemm_workspace_bytes
+    bytes, reused across calls on one stream (allocated zeroed for this call when
+    None).  Returns y (M x N)."""
+    torch = _torch()
+    _need_cuda(x, rms_gain, W_packed, gamma, y, workspace)
+    M, K = x.shape
+    N = W_packed.shape[0]
+    if W_packed.shape[1] * 4 != K:
+        raise ValueError("x and W_packed disagree on K")
+    if y is None:
+        y = torch.empty((M, N), dtype=out_dtype or torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.zeros(max(1, bitnet_bitlinear_gemm_workspace_bytes(M, N, K)), dtype=torch.uint8,
+                                device=x.device)
+    st = lib().bitnet_bitlinear_gemm(_ptr(x), _dtype_code(x.dtype), _ptr(rms_gain), rms_eps, _ptr(W_packed),
+                                     _ptr(gamma), N, K, M, _ptr(y), _dtype_code(y.dtype), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(x.device))
+    _check("bitnet_bitlinear_gemm", st)
+    return y
+
+
 def bitnet_bitlinear_ffn_gemv(x, W_up, gamma_up, W_gate, gamma_gate, W_down, gamma_down, rms_gain_in=None,
                               rms_eps_in: float = 1e-5, rms_gain_sub=None, rms_eps_sub: float = 1e-5, h=None, y=None,
                               out_dtype=None, sync=None):
@@ -443,10 +477,13 @@ def bitnet_get_device_status(device=None) -> int:
 def bitlinear(x, W_packed, gamma, rms_gain=None, rms_eps: float = 1e-5, out_dtype=None):
     """One BitLinear forward: quantise x (fused RMSNorm when rms_gain is given),
     then the ternary product with dequant.  Uses the fused decode kernel for
-    M <= 8 when the quantised rows fit its shared memory."""
+    M <= 8 when the quantised rows fit its shared memory, the fused stream-K
+    kernel for M <= 64, else the quantisation and the tensor-core product."""
     M, K = x.shape
     if M <= 8 and M * K <= 21504:
         return bitnet_bitlinear_gemv(x, W_packed, gamma, rms_gain, rms_eps, out_dtype=out_dtype)
+    if M <= 64 and K <= (32768 if x.dtype == _torch().bfloat16 else 16384):
+        return bitnet_bitlinear_gemm(x, W_packed, gamma, rms_gain, rms_eps, out_dtype=out_dtype)
     x_q, a, rs = bitnet_quant_act(x, rms_gain, rms_eps, want_rowsum=True)
     if x.shape[0] <= 8:
         return bitnet_linear_gemv(W_packed, gamma, x_q, a, rs, out_dtype=out_dtype)

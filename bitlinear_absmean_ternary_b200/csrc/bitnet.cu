@@ -146,8 +146,9 @@ bitnet_status bitnet_pack_weights_noalloc(const float* W, int64_t N, int64_t K, 
 bitnet_status bitnet_get_device_status(void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return BITNET_ERR_CUDA;
-  cudaError_t (*const takers[])(unsigned int*) = {take_error_gemv, take_error_gemm, take_error_ffn,
-                                                  take_error_b3,   take_error_ste,  take_error_quant};
+  cudaError_t (*const takers[])(unsigned int*) = {take_error_gemv, take_error_gemm, take_error_gemm_fused,
+                                                  take_error_ffn,  take_error_b3,   take_error_ste,
+                                                  take_error_quant};
   bool timed_out = false;
   for (auto take : takers) {
     unsigned int v = 0;

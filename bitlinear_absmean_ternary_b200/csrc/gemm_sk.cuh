@@ -39,6 +39,16 @@
 //   * Token tiles: the tiles are (row tile, token tile) pairs, row tiles
 //     fastest, so consecutive units share their activation tile in L2.
 //
+//   * XT (fused quantisation, bitnet_bitlinear_gemm, M <= 64: the four
+//     BitLinear steps of the comrad404.com review, "Метод", in one launch):
+//     the unpack warps (256 threads: the fixed 256-lane order of the RMSNorm
+//     sum) of CTA c quantise the token rows c, c+G, ... into the workspace
+//     (x_q, scales, row sums), while every CTA's weight producer already
+//     streams.  A sense-reversal grid barrier in the workspace (arrival
+//     count, generation) then releases the activation producers and the
+//     epilogues of all CTAs: every CTA of the launch is resident at once (one
+//     per SM), and every wait is bounded.
+//
 //   * GATE (the FFN's up and gate projections in one product, inferownia.pl,
 //     "BitNet b1.58: era 1-bitowych LLM-ów", "Zrób to sam": squared ReLU in
 //     the FFN; kripta.biz 2B4T news: ReLU^2 in the FFN layers): a tile is 64
@@ -62,8 +72,11 @@
 
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "gemm.cuh"
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace bitnet {
 
@@ -85,7 +98,7 @@ struct SkCfg {
   static constexpr int T = (512 - kAcol) / kAslot;         // A slots in TMEM
   static constexpr int kXOff = SW * kWStage;
   static constexpr int kBarOff = kXOff + SX * kXStage;
-  static constexpr int kNumBars = 2 * SW + 2 * SX + 2 * T + 6;
+  static constexpr int kNumBars = 2 * SW + 2 * SX + 2 * T + 7;
   static constexpr int kScaleOff = kBarOff + ((kNumBars * 8 + 8 + 127) / 128) * 128;
   static constexpr int kGateOff = kScaleOff + 2 * BN * 8;  // (GATE) g of a tile, fp32 [BN][64]
   static constexpr int kRowsPerTile = GATE ? 64 : kGemmBM;  // output features per tile
@@ -129,16 +142,56 @@ BN_DEV bool sk_epi_sync(uint64_t* bar, int& phase) {
   return ok;
 }
 
+// In-kernel quantisation of the token rows (XT != void): the unquantised
+// rows, the optional RMSNorm gain, where the quantised rows, scales and row
+// sums go (the workspace), and the grid barrier's words (arrivals,
+// generation; both start at zero, and the barrier leaves the arrival count
+// at zero).
+template <typename XT>
+struct SkQuant {
+  const XT* x;
+  const XT* gain;
+  float eps;
+  int8_t* xq;
+  float* a;
+  int32_t* rs;
+  unsigned int* bar;
+};
+template <typename XT>
+using sk_qx_t = std::conditional_t<std::is_void_v<XT>, float, XT>;
+
+BN_DEV unsigned int atom_add_acq_rel_gpu_u32(unsigned int* p, unsigned int v) {
+  unsigned int old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Waits (bounded) until the grid barrier's generation differs from gen0.
+BN_DEV bool sk_wait_generation(const unsigned int* gen, unsigned int gen0) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1; ld_acquire_gpu_u32(gen) == gen0; ++i) {
+    if ((i & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+      flag_timeout();
+      return false;
+    }
+  }
+  return true;
+}
+
 // N: output features (rows of W; for GATE the rows of W_up and of W_gate).
 // tmap_w2 / gamma2_ptr: W_gate and its scale (GATE only).  y: M x N outputs
 // of y_dtype, or for GATE the bf16 h (M x N).
-template <int BN, bool U8, bool GATE = false>
+// XT, MAXC: fused quantisation of x of type XT (void: x_q, a_scale and
+// rowsum are given), MAXC 8-element chunks per unpack thread.
+template <int BN, bool U8, bool GATE = false, typename XT = void, int MAXC = 1>
 __global__ void __launch_bounds__(kSkThreads, 1)
     gemm_sk_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                    const __grid_constant__ CUtensorMap tmap_w2, const float* __restrict__ gamma_ptr,
                    const float* __restrict__ gamma2_ptr, const float* __restrict__ a_scale,
                    const int32_t* __restrict__ rowsum, int M, int N, int K, void* __restrict__ y, int y_dtype,
-                   unsigned int* __restrict__ flags, int* __restrict__ parts) {
+                   unsigned int* __restrict__ flags, int* __restrict__ parts, const SkQuant<sk_qx_t<XT>> qa) {
+  constexpr bool FQ = !std::is_void_v<XT>;
+  static_assert(!FQ || (U8 && !GATE), "the fused quantisation computes the row sums; no gate");
   using C = SkCfg<BN, GATE>;
   constexpr int RPT = C::kRowsPerTile;
   constexpr int SW = C::SW, SX = C::SX, T = C::T;
@@ -155,7 +208,9 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* done = acc_empty + 2;
   uint64_t* epi_bar = done + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(epi_bar + 1);
+  uint64_t* qdone = epi_bar + 1;  // FQ: the generation the grid barrier starts from is in s_gen0
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qdone + 1);
+  uint32_t* s_gen0 = tmem_holder + 1;
   float* s_a = reinterpret_cast<float*>(smem + C::kScaleOff);  // [2][BN]: double-buffered per segment
   int* s_rs = reinterpret_cast<int*>(s_a + 2 * BN);           // [2][BN]
   float* gbuf = reinterpret_cast<float*>(smem + C::kGateOff);  // GATE: [BN][64]
@@ -188,6 +243,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     }
     mbar_init(done, 1);
     mbar_init(epi_bar, kSkEpiWarps);
+    mbar_init(qdone, 1);
     fence_barrier_init();
     tma_prefetch_desc(&tmap_x);
     tma_prefetch_desc(&tmap_w);
@@ -236,8 +292,13 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       // ------------------------------------------------------------ activation producer
       pdl_wait();  // x_q comes from the previous kernel
       bool ok = true;
+      if constexpr (FQ) {
+        // x_q comes from this launch: wait for every CTA's quantisation
+        ok = mbar_wait(qdone, 0) && sk_wait_generation(qa.bar + 1, *s_gen0);
+        asm volatile("fence.proxy.async.global;" ::: "memory");  // generic writes -> TMA reads
+      }
       int g = 0;
-      for (; g < total; ++g) {
+      for (; ok && g < total; ++g) {
         const int s = g % SX;
         if (g >= SX && !mbar_wait(&x_empty[s], ((g / SX) & 1) ^ 1)) {
           ok = false;
@@ -295,6 +356,39 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     }
   } else if (warp < kSkFirstEpi) {
     // ------------------------------------------------------------ unpack
+    if constexpr (FQ) {
+      // first the quantisation of the token rows cta, cta + G, ... (256 threads: the
+      // unpack warps are threads 96 .. 351), then one arrival on the grid barrier
+      __shared__ QuantScratch qsc;
+      constexpr int kT0 = kSkFirstUnpack * 32;
+      const int ut = static_cast<int>(threadIdx.x) - kT0;
+      pdl_wait();
+      unsigned int gen0 = 0;
+      if (ut == 0) {
+        gen0 = *reinterpret_cast<volatile unsigned int*>(qa.bar + 1);
+        *s_gen0 = gen0;
+        mbar_arrive(qdone);
+      }
+      for (int m = cta; m < M; m += G) {
+        float amax;
+        int sum;
+        quant_row_cta<sk_qx_t<XT>, MAXC, false, 256, kT0>(qa.x + static_cast<int64_t>(m) * K, K, qa.gain, qa.eps,
+                                                          qa.xq + static_cast<int64_t>(m) * K, qsc, amax, sum);
+        if (ut == 0) {
+          qa.a[m] = amax == 0.0f ? 0.0f : __fdiv_rn(amax, 127.0f);
+          qa.rs[m] = sum;
+        }
+      }
+      __threadfence();
+      sync_threads<256>();
+      if (ut == 0) {
+        const unsigned int old = atom_add_acq_rel_gpu_u32(qa.bar, 1u);
+        if (old == static_cast<unsigned int>(G) - 1u) {
+          qa.bar[0] = 0u;  // the last arrival: count back to zero, then the new generation
+          st_release_gpu_u32(qa.bar + 1, gen0 + 1u);
+        }
+      }
+    }
     const int q = warp & 3;
     const int par = (warp - kSkFirstUnpack) >> 2;  // this warp takes stages with g % 2 == par
     const int r = 32 * q + lane;
@@ -342,6 +436,13 @@ __global__ void __launch_bounds__(kSkThreads, 1)
     // row r's scale: W_up's (or W's) for the first 64 rows of a gated tile, W_gate's for the others
     const float gamma = (GATE && r >= 64) ? __ldg(gamma2_ptr) : __ldg(gamma_ptr);
     int ephase = 0;
+    if constexpr (FQ) {
+      // the scales and row sums come from this launch's quantisation (every CTA's)
+      if (et == 0) {
+        if (mbar_wait(qdone, 0)) sk_wait_generation(qa.bar + 1, *s_gen0);
+      }
+      sk_epi_sync(epi_bar, ephase);
+    }
     int seg = 0;
     for (long long u = u0; u < u1; ++seg) {
       const long long t = u / nk;
@@ -354,8 +455,8 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       const int sb = (seg & 1) * BN;  // this segment's half of the scale buffers
       if (et < BN) {  // requested before the accumulator wait, so the loads overlap it
         const int m = m0 + et;
-        s_a[sb + et] = m < M ? __ldg(a_scale + m) : 0.0f;
-        s_rs[sb + et] = (U8 && m < M) ? __ldg(rowsum + m) : 0;
+        s_a[sb + et] = m < M ? __ldcg(a_scale + m) : 0.0f;
+        s_rs[sb + et] = (U8 && m < M) ? __ldcg(rowsum + m) : 0;
       }
       const int b = seg & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[b], (seg >> 1) & 1))) break;

@@ -141,6 +141,7 @@ constexpr int kGemvB3XMaxBytes = 24000;
 // bounded waits: each reads its word into *v and clears it when set.
 cudaError_t take_error_gemv(unsigned int* v);
 cudaError_t take_error_gemm(unsigned int* v);
+cudaError_t take_error_gemm_fused(unsigned int* v);
 cudaError_t take_error_ffn(unsigned int* v);
 cudaError_t take_error_b3(unsigned int* v);
 cudaError_t take_error_ste(unsigned int* v);

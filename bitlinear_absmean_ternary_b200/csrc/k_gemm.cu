@@ -163,7 +163,7 @@ cudaError_t launch_sk(const CUtensorMap& mx, const CUtensorMap& mw, const CUtens
   unsigned int* flags = static_cast<unsigned int*>(ws);
   int* parts = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + sk_flag_bytes(sms));
   return launch_pdl(kern, dim3(G), dim3(kSkThreads), C::kSmemBytes, s, mx, mw, mw2, gamma, gamma2, a, rs, M, N, K, y,
-                    yd, flags, parts);
+                    yd, flags, parts, SkQuant<float>{});
 }
 
 // Tensor maps of a stream-K product: activations in 128-byte-wide boxes of BN

@@ -112,12 +112,13 @@ BN_DEV void sync_threads() {
 // warp obtains the norm itself, with the oracle's order of additions.
 // Consecutive calls may reuse the scratch: every write to a scratch array
 // comes after a barrier that all readers of its previous contents passed.
-// NT: the threads taking part are the first NT of the CTA (synchronised by
-// named barrier 1), or all of them when NT == 0.
-template <typename T, int MAXC, bool COHERENT = false, int NT = 0>
+// NT: the threads taking part are the NT threads from T0 on (T0 a multiple of
+// 32; synchronised by named barrier 1), or all of the CTA's when NT == 0.
+template <typename T, int MAXC, bool COHERENT = false, int NT = 0, int T0 = 0>
 BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict__ gain, float rms_eps,
                           int8_t* xq_row, QuantScratch& sc, float& amax_out, int& sum_out) {
-  const int t = threadIdx.x;
+  static_assert(T0 % 32 == 0 && (T0 == 0 || NT != 0), "a thread offset needs a fixed thread count");
+  const int t = static_cast<int>(threadIdx.x) - T0;
   const int lane = t & 31, warp = t >> 5;
   const int nthreads = NT == 0 ? static_cast<int>(blockDim.x) : NT;
   const int nwarps = nthreads >> 5;

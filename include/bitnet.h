@@ -25,7 +25,7 @@
  *   - Errors are returned as bitnet_status; nothing is launched when an
  *     argument is rejected.  No C++ exception crosses this boundary.
  *   - The product entry points (bitnet_linear_gemv, bitnet_linear_gemm,
- *     bitnet_linear_upgate_gemm, bitnet_bitlinear_gemv,
+ *     bitnet_linear_upgate_gemm, bitnet_bitlinear_gemv, bitnet_bitlinear_gemm,
  *     bitnet_bitlinear_ffn_gemv, bitnet_bitlinear_gemv_b3) are launched with programmatic dependent
  *     launch: they start while the previous kernel on the stream finishes,
  *     and request their first packed-weight tiles BEFORE waiting for it
@@ -231,6 +231,39 @@ bitnet_status bitnet_linear_gemm(const uint8_t* W_packed, const float* gamma, in
                                  const int8_t* x_q, const float* a_scale, const int32_t* x_rowsum,
                                  int64_t M, void* y, int y_dtype, void* workspace, size_t workspace_bytes,
                                  void* stream);
+
+/*
+ * Bytes of workspace bitnet_bitlinear_gemm uses on the CURRENT device: the
+ * stream-K flags and partial tiles of bitnet_linear_gemm, 256 bytes of grid
+ * barrier, and the quantised rows, scales and row sums; 0 for M outside
+ * 1..64 or an invalid K.
+ */
+size_t bitnet_bitlinear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * Fused BitLinear for decode-sized batches (1 <= M <= 64 tokens):
+ * bitnet_quant_act followed by bitnet_linear_gemm's stream-K product in one
+ * kernel launch (the four BitLinear steps of the comrad404.com review,
+ * section "Метод", in one pass).  The first CTAs quantise one token row each
+ * (same arithmetic and summation order as bitnet_quant_act) into the
+ * workspace while every CTA already streams its share of the packed weights;
+ * a grid barrier in the workspace then releases the product.  The results
+ * are identical to the two calls.
+ *
+ * x, x_dtype, rms_gain, rms_eps   as bitnet_quant_act (K <= 32768 bf16, 16384 f32).
+ * W_packed, gamma, N, K, y, y_dtype   as bitnet_linear_gemm.
+ * workspace [in,out] at least bitnet_bitlinear_gemm_workspace_bytes(M, N, K)
+ *           bytes, 16-byte aligned, zeroed before its first use; the calls
+ *           leave its flags and barrier words zero-based again.  Same rules
+ *           as bitnet_linear_gemm's workspace: not shared by calls that may
+ *           overlap, zeroed again after a BITNET_ERR_TIMEOUT, and the launch
+ *           needs every SM of the device at once (its CTAs wait on one
+ *           another, with bounded waits).
+ * Asynchronous.
+ */
+bitnet_status bitnet_bitlinear_gemm(const void* x, int x_dtype, const void* rms_gain, float rms_eps,
+                                    const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, int64_t M,
+                                    void* y, int y_dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Bytes of workspace bitnet_linear_upgate_gemm uses on the CURRENT device

@@ -148,6 +148,30 @@ def test_upgate_rejects_bad_arguments(L):
     assert call(M=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
 
 
+def test_fused_gemm_rejects_bad_arguments(L):
+    need = bl.bitnet_bitlinear_gemm_workspace_bytes(16, 256, 512)
+    assert need > bl.bitnet_linear_gemm_workspace_bytes(16, 256, 512)   # + barrier, scales, x_q
+    assert bl.bitnet_bitlinear_gemm_workspace_bytes(65, 256, 512) == 0
+    assert bl.bitnet_bitlinear_gemm_workspace_bytes(4, 256, 100) == 0
+
+    def call(x=FAKE, dt=bl.BITNET_BF16, g=None, eps=1e-5, W=FAKE, gam=FAKE, N=256, K=512, M=16, y=FAKE,
+             yd=bl.BITNET_BF16, ws=FAKE, wsb=1 << 30):
+        return L.bitnet_bitlinear_gemm(x, dt, g, eps, W, gam, N, K, M, y, yd, ws, wsb, None)
+
+    for kw in ({"x": None}, {"W": None}, {"gam": None}, {"y": None}, {"ws": None}):
+        assert call(**kw) == bl.BITNET_ERR_INVALID_ARG, kw
+    for kw in ({"x": MIS}, {"W": MIS}, {"ws": MIS}, {"g": MIS}, {"gam": FAKE + 2}):
+        assert call(**kw) == bl.BITNET_ERR_INVALID_ARG, kw
+    assert call(dt=bl.BITNET_I32) == bl.BITNET_ERR_INVALID_ARG
+    assert call(yd=7) == bl.BITNET_ERR_INVALID_ARG
+    assert call(g=FAKE, eps=0.0) == bl.BITNET_ERR_INVALID_ARG
+    assert call(wsb=need - 16) == bl.BITNET_ERR_INVALID_ARG
+    assert call(M=65) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(M=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(K=96) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(dt=bl.BITNET_F32, K=16384 + 64) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+
+
 def test_fused_rejects_bad_arguments(L):
     def call(x=FAKE, dt=bl.BITNET_BF16, g=None, eps=1e-5, W=FAKE, gam=FAKE, N=8, K=64, M=1, y=FAKE,
              yd=bl.BITNET_BF16):

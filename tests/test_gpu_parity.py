@@ -550,3 +550,98 @@ def test_upgate_gemm_matches_oracle_ffn_gate(dev, orc, M, F, K, signed):
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     assert int(ws[:4 * sms].view(torch.int32).abs().sum()) == 0
     assert bl.bitnet_get_device_status() == bl.BITNET_OK
+
+
+# --------------------------------------------------------------------------- fused quantisation + stream-K (M <= 64)
+
+FQ_CASES = [
+    # M, N, K, x dtype, norm, y dtype
+    (64, 3840, 2560, "bf16", True, "bf16"),      # the 2.5B block's Q|K|V at M = 64
+    (64, 2560, 6912, "bf16", True, "f32"),       # its down projection
+    (16, 21504, 5376, "bf16", False, "bf16"),    # 27B up at M = 16
+    (16, 5376, 21504, "bf16", False, "i32"),     # 27B down at M = 16 (16 chunks per thread)
+    (5, 300, 320, "f32", True, "f32"),
+    (33, 777, 1344, "f32", False, "bf16"),
+    (1, 128, 64, "bf16", True, "f32"),           # one unit: a grid of one CTA quantises every row
+    (9, 129, 8192, "f32", True, "i32"),
+]
+
+
+@pytest.mark.parametrize("M,N,K,dt,norm,yt", FQ_CASES)
+def test_fused_bitlinear_gemm_parity(dev, orc, M, N, K, dt, norm, yt):
+    """Quantisation inside the stream-K product (one launch, grid barrier in the
+    workspace) against the oracle and against the two-call path."""
+    import torch
+    W = synth.weights(N, K, 0.02, M + N, 1)
+    x = synth.activations(M, K, M + K, 2, "normal", 0.01, 20.0, dt)
+    x[0, :3] = 0.0
+    if M > 2:
+        x[2] = 0.0                                   # an all-zero token
+    g = synth.gain(K, 1, 3, dt) if norm else None
+    P, G = bl.bitnet_pack_weights(_t(W, dev), EPS_W)
+    p_ref, g_ref = orc.pack_weights(W, EPS_W)
+    xq_r, a_r, _ = orc.quant_act(x, g, EPS_RMS)
+    out = {"bf16": torch.bfloat16, "f32": torch.float32, "i32": torch.int32}[yt]
+    xd = _x_dev(x, dt, dev)
+    gd = None if g is None else _x_dev(g, dt, dev)
+    ws = torch.zeros(bl.bitnet_bitlinear_gemm_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
+    y = bl.bitnet_bitlinear_gemm(xd, P, G, gd, EPS_RMS, out_dtype=out, workspace=ws)
+    if M * N * K <= 64 * 3840 * 2560:
+        acc_r, y_r = orc.bitlinear(p_ref, g_ref, K, xq_r, a_r)
+        got = y.cpu().numpy()
+    else:
+        rng = np.random.default_rng(1)
+        ms, ns = rng.integers(0, M, 4000), rng.integers(0, N, 4000)
+        acc_r, y_r = orc.bitlinear_sampled(p_ref, g_ref, K, xq_r, a_r, ms, ns)
+        got = y.cpu().numpy()[ms, ns] if yt != "bf16" else None
+    if yt == "i32":
+        np.testing.assert_array_equal(got, acc_r)
+    elif yt == "f32":
+        assert ulp_diff_f32(got, y_r).max() == 0
+    else:
+        yb = y.view(torch.int16).cpu().numpy().view(np.uint16)
+        if M * N * K > 64 * 3840 * 2560:
+            yb = yb[ms, ns]
+        assert ulp_diff_bf16(yb, orc.f32_to_bf16(y_r)).max() == 0
+    # identical to the two-call path, and again with the same workspace (barrier words reused)
+    xq, a, rs = bl.bitnet_quant_act(xd, gd, EPS_RMS, want_rowsum=True)
+    y2 = bl.bitnet_linear_gemm(P, G, xq, a, rs, out_dtype=out)
+    assert torch.equal(y, y2)
+    y3 = bl.bitnet_bitlinear_gemm(xd, P, G, gd, EPS_RMS, out_dtype=out, workspace=ws)
+    assert torch.equal(y, y3)
+    assert bl.bitnet_get_device_status() == bl.BITNET_OK
+
+
+def test_fused_bitlinear_gemm_shares_a_workspace_across_shapes_and_graph_replays(dev, orc):
+    """One workspace for launches of different grid sizes (the barrier's arrival
+    count returns to zero after each), captured in a CUDA graph and replayed."""
+    import torch
+    shapes = [(16, 21504, 5376), (3, 128, 64), (64, 2560, 2560), (16, 21504, 5376)]
+    ws_bytes = max(bl.bitnet_bitlinear_gemm_workspace_bytes(*s) for s in shapes)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    cases = []
+    for i, (M, N, K) in enumerate(shapes):
+        W = synth.weights(N, K, 0.02, i, 7)
+        x = synth.activations(M, K, i, 8, "normal", 0.0, 1.0, "bf16")
+        g = synth.gain(K, i, 9, "bf16")
+        P, G = bl.bitnet_pack_weights(_t(W, dev), EPS_W)
+        xd, gd = _x_dev(x, "bf16", dev), _x_dev(g, "bf16", dev)
+        xq, a, rs = bl.bitnet_quant_act(xd, gd, EPS_RMS, want_rowsum=True)
+        ref = bl.bitnet_linear_gemm(P, G, xq, a, rs, out_dtype=torch.int32)
+        cases.append((xd, gd, P, G, ref, torch.empty_like(ref)))
+    for xd, gd, P, G, ref, y in cases:
+        bl.bitnet_bitlinear_gemm(xd, P, G, gd, EPS_RMS, y=y, workspace=ws)
+        assert torch.equal(y, ref)
+    s = torch.cuda.Stream(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        for xd, gd, P, G, ref, y in cases:
+            bl.bitnet_bitlinear_gemm(xd, P, G, gd, EPS_RMS, y=y, workspace=ws)
+    for _ in range(3):
+        for *_, y in cases:
+            y.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        for xd, gd, P, G, ref, y in cases:
+            assert torch.equal(y, ref)
+    assert bl.bitnet_get_device_status() == bl.BITNET_OK
