@@ -107,7 +107,7 @@ struct SkCfg {
   // second CTA never fits on the SM, so none waits in tcgen05.alloc.
   static constexpr int kMinSmem = 233472 / 2;
   static constexpr int kSmemBytes = kNeeded > kMinSmem ? kNeeded : kMinSmem;
-  // workspace: G flags (rounded to 256 bytes), then G partial tiles int32 [BN][128]
+  // workspace: G flags (rounded to 256 bytes), then G partial tiles int4 [BN/4][128] (int32 [BN][128])
   static constexpr int kPartInts = BN * kGemmBM;
   static_assert(kWStage % 1024 == 0 && kXStage % 1024 == 0, "stages stay 1024-byte aligned");
   static_assert(kAcol + T * kAslot <= 512 && T >= 2, "TMEM budget");
@@ -475,9 +475,12 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       if (lane == 0) mbar_arrive(&acc_empty[b]);  // the accumulator may be reused
       if (kb_lo > 0) {
         // helper: this CTA's partial of a tile finished by an earlier CTA
-        int* slot = parts + static_cast<size_t>(cta) * C::kPartInts;
+        // partial tile layout int4 [BN/4][128]: thread r moves 16 bytes per access, a warp 512 contiguous bytes
+        int4* slot = reinterpret_cast<int4*>(parts + static_cast<size_t>(cta) * C::kPartInts);
 #pragma unroll
-        for (int j = 0; j < BN; ++j) slot[j * kGemmBM + r] = static_cast<int>(v[j]);
+        for (int j4 = 0; j4 < BN / 4; ++j4)
+          slot[j4 * kGemmBM + r] = make_int4(static_cast<int>(v[4 * j4]), static_cast<int>(v[4 * j4 + 1]),
+                                             static_cast<int>(v[4 * j4 + 2]), static_cast<int>(v[4 * j4 + 3]));
         __threadfence();
         if (sk_epi_sync(epi_bar, ephase) && et == 0) st_release_gpu_u32(&flags[cta], 1u);
         continue;
@@ -501,9 +504,15 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         sk_epi_sync(epi_bar, ephase);
         __threadfence();
         for (int h = cta + 1; h <= last; ++h) {
-          const int* slot = parts + static_cast<size_t>(h) * C::kPartInts;
+          const int4* slot = reinterpret_cast<const int4*>(parts + static_cast<size_t>(h) * C::kPartInts);
 #pragma unroll
-          for (int j = 0; j < BN; ++j) v[j] += static_cast<uint32_t>(__ldcg(slot + j * kGemmBM + r));
+          for (int j4 = 0; j4 < BN / 4; ++j4) {
+            const int4 p = __ldcg(slot + j4 * kGemmBM + r);
+            v[4 * j4] += static_cast<uint32_t>(p.x);
+            v[4 * j4 + 1] += static_cast<uint32_t>(p.y);
+            v[4 * j4 + 2] += static_cast<uint32_t>(p.z);
+            v[4 * j4 + 3] += static_cast<uint32_t>(p.w);
+          }
         }
         if (et == 0)  // every thread has read the partials once the next barrier completes
           for (int h = cta + 1; h <= last; ++h) flags[h] = 0u;  // all zero again for the next call
