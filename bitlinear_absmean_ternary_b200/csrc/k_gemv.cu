@@ -109,7 +109,11 @@ cudaError_t launch_fused_t(const void* x, const void* gain, float eps, const uin
 template <int MT, typename T>
 cudaError_t launch_fused_c(const void* x, const void* gain, float eps, const uint8_t* Wp, const float* gamma, int N,
                            int K, void* y, int yd, cudaStream_t s) {
-  const int per_thread = (K / 8 + kQuantThreads - 1) / kQuantThreads;
+  // 8-element chunks per thread of the quantisation prologue: the fixed-order
+  // RMSNorm sum is defined on 256 threads; without a norm all 512 take part
+  // (fewer registers, so the next launch's CTA can share the SM)
+  const int nthr = gain != nullptr ? kQuantThreads : kGemvThreads;
+  const int per_thread = (K / 8 + nthr - 1) / nthr;
   if (per_thread <= 1) return launch_fused_t<MT, T, 1>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
   if (per_thread <= 2) return launch_fused_t<MT, T, 2>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
   if (per_thread <= 4) return launch_fused_t<MT, T, 4>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
