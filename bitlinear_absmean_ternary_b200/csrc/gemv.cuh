@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint8_t* __res
                                                             const int32_t* __restrict__ rowsum,
                                                             const T* __restrict__ xin, const T* __restrict__ gain,
                                                             float rms_eps, void* __restrict__ y, int y_dtype,
-                                                            int kchunk, int nslots) {
+                                                            int kchunk, int nslots, int l2_prefetch) {
   static_assert(!FUSED || (XS && U8), "the fused kernel keeps x_q in shared memory and uses its row sums");
   extern __shared__ __align__(1024) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -152,8 +152,22 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const uint8_t* __res
     }
   };
   const int my_items = items > warp ? (items - warp + kGemvWarps - 1) / kGemvWarps : 0;
-  if (lane == 0)
+  if (lane == 0) {
     for (int k = 0; k < nslots && k < my_items; ++k) issue(k);
+    if (l2_prefetch) {
+      // The CTA's rows are contiguous in memory: request all of them into L2 now, one slice
+      // per warp.  Under programmatic dependent launch this runs while the previous kernel
+      // still works, so the weights stream from HBM across the kernel boundary and the ring
+      // refills after the dependency wait hit L2.
+      const int64_t share = static_cast<int64_t>(nrows) * row_bytes;
+      const int64_t slice = (share / kGemvWarps + 15) / 16 * 16;
+      const int64_t lo = slice * warp, hi = lo + slice < share ? lo + slice : share;
+      for (int64_t o = lo; o < hi; o += 65536) {
+        const int64_t n = hi - o < 65536 ? hi - o : 65536;
+        bulk_prefetch_l2(Wp + row_lo * row_bytes + o, static_cast<uint32_t>(n));
+      }
+    }
+  }
 
   // Everything below reads the outputs of the previous kernel.
   pdl_launch_dependents();

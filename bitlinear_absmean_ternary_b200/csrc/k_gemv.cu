@@ -30,7 +30,7 @@ using namespace bitnet_host;
 constexpr int kGemvSmemMax = 232448 - 2048;  // 227 KB less the fused kernel's static scratch
 
 struct GemvPlan {
-  int grid, kchunk, nslots, smem;
+  int grid, kchunk, nslots, smem, l2_prefetch;
 };
 
 GemvPlan gemv_plan(int mt, int N, int K, bool xs) {
@@ -39,6 +39,7 @@ GemvPlan gemv_plan(int mt, int N, int K, bool xs) {
   p.grid = static_cast<int>(groups < sm_count() ? groups : sm_count());
   const int64_t rows = (N + p.grid - 1) / p.grid;
   const int64_t share = rows * (K / 4);
+  p.l2_prefetch = share > BITNET_GEMV_SMALL_SHARE ? 1 : 0;
   if (share <= BITNET_GEMV_SMALL_SHARE) {
     p.kchunk = gemv_kchunk(K);
     p.nslots = kGemvSlots;
@@ -62,7 +63,7 @@ cudaError_t launch_gemv_x(const uint8_t* Wp, const float* gamma, int N, int K, c
   if (p.smem > kGemvSmemMax) return cudaErrorInvalidValue;
   return launch_pdl(gemv_kernel<MT, U8, XS>, dim3(p.grid), dim3(kGemvThreads), p.smem, s, Wp, gamma, N, K, xq, a, rs,
                     static_cast<const float*>(nullptr), static_cast<const float*>(nullptr), 0.0f, y, yd, p.kchunk,
-                    p.nslots);
+                    p.nslots, p.l2_prefetch);
 }
 
 template <int MT, bool U8>
@@ -103,7 +104,7 @@ cudaError_t launch_fused_t(const void* x, const void* gain, float eps, const uin
   return launch_pdl(kern, dim3(p.grid), dim3(kGemvThreads), p.smem, s, Wp, gamma, N, K,
                     static_cast<const int8_t*>(nullptr), static_cast<const float*>(nullptr),
                     static_cast<const int32_t*>(nullptr), static_cast<const T*>(x), static_cast<const T*>(gain), eps, y,
-                    yd, p.kchunk, p.nslots);
+                    yd, p.kchunk, p.nslots, p.l2_prefetch);
 }
 
 template <int MT, typename T>

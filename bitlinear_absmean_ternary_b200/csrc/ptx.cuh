@@ -91,6 +91,12 @@ BN_DEV void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* 
       : "memory");
 }
 
+// Prefetch `bytes` of global memory into L2 (no destination, no completion
+// to wait for).  src 16-byte aligned; bytes a multiple of 16.
+BN_DEV void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 BN_DEV uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
