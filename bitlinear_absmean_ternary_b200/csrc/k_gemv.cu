@@ -2,6 +2,7 @@
 // fused decode BitLinear bitnet_bitlinear_gemv (gemv.cuh).
 #include "host_common.h"
 #include "gemv.cuh"
+#include "gemv1.cuh"
 
 namespace {
 
@@ -53,6 +54,97 @@ GemvPlan gemv_plan(int mt, int N, int K, bool xs) {
   return p;
 }
 
+// Launch plan of gemv1_kernel (one token): S column segments per row (the
+// fewest that leave each lane at most kGemv1MaxPairs word pairs), NP pairs
+// per lane, slots of R whole rows (a multiple of the 16/S rows the warps take
+// at once, about BITNET_GEMV1_SLOT_TARGET bytes), a ring of about
+// BITNET_GEMV1_RING_TARGET bytes, and the rest of a large share prefetched
+// into L2.  The kernel's shared memory stays under half an SM's (two CTAs
+// per SM, so that a launch overlaps the previous one).  Returns false when K
+// is beyond the register budget (K > 16 * 16 * 64 * kGemv1MaxPairs); those
+// shapes take gemv_kernel.
+#ifndef BITNET_GEMV1_SLOT_TARGET
+#define BITNET_GEMV1_SLOT_TARGET (48 * 1024)
+#endif
+#ifndef BITNET_GEMV1_RING_TARGET
+#define BITNET_GEMV1_RING_TARGET (88 * 1024)
+#endif
+#ifndef BITNET_GEMV1_RING_TARGET1
+#define BITNET_GEMV1_RING_TARGET1 (176 * 1024)
+#endif
+#ifndef BITNET_GEMV1_WARPS
+#define BITNET_GEMV1_WARPS 16
+#endif
+constexpr int kGemv1SmemMax = 232448 / 2 - 2048 - 1024;  // two CTAs per SM, each with static scratch
+constexpr int kGemv1SmemMax1 = 232448 - 2048;            // one CTA per SM
+
+struct Gemv1Plan {
+  int grid, warps, S, NP, R, nslots, rows_max, smem, l2_prefetch;
+};
+
+int gemv1_segw(int Bw, int S) { return ((Bw + S - 1) / S + 1) & ~1; }
+
+bool gemv1_plan(int N, int K, bool xs, Gemv1Plan& p) {
+  const int B = K / 4, Bw = B / 4;
+  p.warps = BITNET_GEMV1_WARPS;
+  const int smem_max = p.warps == 16 ? kGemv1SmemMax : kGemv1SmemMax1;
+  p.S = 1;
+  while (p.S < kGemvWarps && gemv1_segw(Bw, p.S) > 64 * kGemv1MaxPairs) p.S *= 2;
+  const int segw = gemv1_segw(Bw, p.S);
+  if (segw > 64 * kGemv1MaxPairs) return false;
+  p.NP = (segw + 63) / 64;
+  p.grid = N < sm_count() ? N : sm_count();
+  p.rows_max = (N + p.grid - 1) / p.grid;
+  const int RG = p.warps / p.S;
+  const int per = BITNET_GEMV1_SLOT_TARGET / (RG * B);
+  p.R = RG * (per > 1 ? per : 1);
+  if (p.R > p.rows_max) p.R = p.rows_max;
+  const int slot_bytes = p.R * B;
+  const int slots_per_cta = (p.rows_max + p.R - 1) / p.R;
+  p.nslots = (p.warps == 16 ? BITNET_GEMV1_RING_TARGET : BITNET_GEMV1_RING_TARGET1) / slot_bytes;
+  if (p.nslots < 2) p.nslots = 2;
+  if (p.nslots > kGemv1MaxSlots) p.nslots = kGemv1MaxSlots;
+  if (p.nslots > slots_per_cta) p.nslots = slots_per_cta;
+  while (p.nslots > 1 && gemv1_smem_bytes(K, xs, slot_bytes, p.nslots, p.rows_max, p.S) > smem_max) --p.nslots;
+  p.smem = gemv1_smem_bytes(K, xs, slot_bytes, p.nslots, p.rows_max, p.S);
+  if (p.smem > smem_max) return false;
+  p.l2_prefetch = static_cast<int64_t>(p.rows_max) * B > static_cast<int64_t>(p.nslots) * slot_bytes ? 1 : 0;
+  return true;
+}
+
+template <bool U8, int NP, int NWARPS, bool FUSED, typename T, int MAXC>
+cudaError_t launch_gemv1_w(const Gemv1Plan& p, const uint8_t* Wp, const float* gamma, int N, int K,
+                            const int8_t* xq, const float* a, const int32_t* rs, const T* x, const T* gain,
+                            float eps, void* y, int yd, cudaStream_t s) {
+  static std::atomic<bool> done[kMaxDevices] = {};
+  auto kern = gemv1_kernel<U8, NP, NWARPS, FUSED, T, MAXC>;
+  const cudaError_t e = set_smem(kern, NWARPS == 16 ? kGemv1SmemMax : kGemv1SmemMax1, done);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3(p.grid), dim3(NWARPS * 32), p.smem, s, Wp, gamma, N, K, xq, a, rs, x, gain, eps, y,
+                    yd, p.S, p.R, p.nslots, p.rows_max, p.l2_prefetch);
+}
+
+template <bool U8, int NP, bool FUSED, typename T, int MAXC>
+cudaError_t launch_gemv1_np(const Gemv1Plan& p, const uint8_t* Wp, const float* gamma, int N, int K,
+                            const int8_t* xq, const float* a, const int32_t* rs, const T* x, const T* gain,
+                            float eps, void* y, int yd, cudaStream_t s) {
+  static_assert(BITNET_GEMV1_WARPS == 16 || BITNET_GEMV1_WARPS == 32, "16 or 32 warps");
+  return launch_gemv1_w<U8, NP, BITNET_GEMV1_WARPS, FUSED, T, MAXC>(p, Wp, gamma, N, K, xq, a, rs, x, gain, eps, y,
+                                                                    yd, s);
+}
+
+template <bool U8, bool FUSED, typename T = float, int MAXC = 1>
+cudaError_t launch_gemv1(const Gemv1Plan& p, const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq,
+                         const float* a, const int32_t* rs, const T* x, const T* gain, float eps, void* y, int yd,
+                         cudaStream_t s) {
+  switch (p.NP) {
+    case 1: return launch_gemv1_np<U8, 1, FUSED, T, MAXC>(p, Wp, gamma, N, K, xq, a, rs, x, gain, eps, y, yd, s);
+    case 2: return launch_gemv1_np<U8, 2, FUSED, T, MAXC>(p, Wp, gamma, N, K, xq, a, rs, x, gain, eps, y, yd, s);
+    case 3: return launch_gemv1_np<U8, 3, FUSED, T, MAXC>(p, Wp, gamma, N, K, xq, a, rs, x, gain, eps, y, yd, s);
+    default: return launch_gemv1_np<U8, 4, FUSED, T, MAXC>(p, Wp, gamma, N, K, xq, a, rs, x, gain, eps, y, yd, s);
+  }
+}
+
 template <int MT, bool U8, bool XS>
 cudaError_t launch_gemv_x(const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
                           const int32_t* rs, void* y, int yd, cudaStream_t s) {
@@ -69,6 +161,12 @@ cudaError_t launch_gemv_x(const uint8_t* Wp, const float* gamma, int N, int K, c
 template <int MT, bool U8>
 cudaError_t launch_gemv_t(const uint8_t* Wp, const float* gamma, int N, int K, const int8_t* xq, const float* a,
                           const int32_t* rs, void* y, int yd, cudaStream_t s) {
+  if constexpr (MT == 1) {
+    Gemv1Plan p;
+    if (gemv1_plan(N, K, false, p))
+      return launch_gemv1<U8, false>(p, Wp, gamma, N, K, xq, a, rs, static_cast<const float*>(nullptr),
+                                     static_cast<const float*>(nullptr), 0.0f, y, yd, s);
+  }
   if (static_cast<int64_t>(MT) * K <= kGemvXMaxBytes)
     return launch_gemv_x<MT, U8, true>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
   return launch_gemv_x<MT, U8, false>(Wp, gamma, N, K, xq, a, rs, y, yd, s);
@@ -95,6 +193,14 @@ cudaError_t launch_gemv_u(int M, const uint8_t* Wp, const float* gamma, int N, i
 template <int MT, typename T, int MAXC>
 cudaError_t launch_fused_t(const void* x, const void* gain, float eps, const uint8_t* Wp, const float* gamma, int N,
                            int K, void* y, int yd, cudaStream_t s) {
+  if constexpr (MT == 1) {
+    Gemv1Plan p;
+    if (gemv1_plan(N, K, true, p))
+      return launch_gemv1<true, true, T, MAXC>(p, Wp, gamma, N, K, static_cast<const int8_t*>(nullptr),
+                                               static_cast<const float*>(nullptr),
+                                               static_cast<const int32_t*>(nullptr), static_cast<const T*>(x),
+                                               static_cast<const T*>(gain), eps, y, yd, s);
+  }
   static std::atomic<bool> done[kMaxDevices] = {};
   auto kern = gemv_kernel<MT, true, true, true, T, MAXC>;
   const cudaError_t e = set_smem(kern, kGemvSmemMax, done);
