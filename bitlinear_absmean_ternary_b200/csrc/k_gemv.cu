@@ -60,9 +60,10 @@ GemvPlan gemv_plan(int mt, int N, int K, bool xs) {
 // at once, about BITNET_GEMV1_SLOT_TARGET bytes), a ring of about
 // BITNET_GEMV1_RING_TARGET bytes, and the rest of a large share prefetched
 // into L2.  The kernel's shared memory stays under half an SM's (two CTAs
-// per SM, so that a launch overlaps the previous one).  Returns false when K
-// is beyond the register budget (K > 16 * 16 * 64 * kGemv1MaxPairs); those
-// shapes take gemv_kernel.
+// per SM, so that a launch overlaps the previous one).  Returns false for a
+// share of at most BITNET_GEMV_SMALL_SHARE bytes per CTA and when K is beyond
+// the register budget (K > 16 * 16 * 64 * kGemv1MaxPairs); those shapes take
+// gemv_kernel.
 #ifndef BITNET_GEMV1_SLOT_TARGET
 #define BITNET_GEMV1_SLOT_TARGET (48 * 1024)
 #endif
@@ -95,6 +96,9 @@ bool gemv1_plan(int N, int K, bool xs, Gemv1Plan& p) {
   p.NP = (segw + 63) / 64;
   p.grid = N < sm_count() ? N : sm_count();
   p.rows_max = (N + p.grid - 1) / p.grid;
+  // a small share (a few rows per SM) is latency-bound: the item kernel, whose
+  // 16 warps each start on their own first item at once, serves it better
+  if (static_cast<int64_t>(p.rows_max) * B <= BITNET_GEMV_SMALL_SHARE) return false;
   const int RG = p.warps / p.S;
   const int per = BITNET_GEMV1_SLOT_TARGET / (RG * B);
   p.R = RG * (per > 1 ? per : 1);

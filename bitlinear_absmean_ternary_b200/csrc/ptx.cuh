@@ -44,15 +44,6 @@ BN_DEV void fence_barrier_init() {
 // async-proxy (bulk copy / TMA) accesses of the same memory.
 BN_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-// Shared-memory atomic add with acquire-release semantics at CTA scope:
-// the caller's earlier accesses are ordered before it, and it sees those of
-// every thread whose add it follows.  Returns the old value.
-BN_DEV unsigned int atom_add_acq_rel_cta_shared(unsigned int* p, unsigned int v) {
-  unsigned int old;
-  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(smem_addr(p)), "r"(v) : "memory");
-  return old;
-}
-
 BN_DEV void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }

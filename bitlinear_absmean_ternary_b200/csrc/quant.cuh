@@ -11,6 +11,8 @@
 
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "ptx.cuh"
 
 namespace bitnet {
@@ -207,20 +209,26 @@ BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict_
       amax = __uint_as_float(mb << 16);
     }
   }
+  // The branch on the gain is taken once, outside the element loops.
+  auto amax_chunks = [&](auto has_gain) {
+    constexpr bool HG = decltype(has_gain)::value;
 #pragma unroll
-  for (int i = 0; i < MAXC && !(sizeof(T) == 2 && gain == nullptr); ++i) {
-    const int c = t + nt * i;
-    if (c < nchunks) {
-      Chunk8<T> g;
-      if (gain != nullptr) g = gain_chunk(i, c);
+    for (int i = 0; i < MAXC; ++i) {
+      const int c = t + nt * i;
+      if (c < nchunks) {
+        Chunk8<T> g;
+        if constexpr (HG) g = gain_chunk(i, c);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float v = ch[i].get(e);
-        const float h = gain != nullptr ? __fmul_rn(__fmul_rn(v, r), g.get(e)) : v;
-        amax = fmaxf(amax, fabsf(h));
+        for (int e = 0; e < 8; ++e) {
+          const float v = ch[i].get(e);
+          const float h = HG ? __fmul_rn(__fmul_rn(v, r), g.get(e)) : v;
+          amax = fmaxf(amax, fabsf(h));
+        }
       }
     }
-  }
+  };
+  if (gain != nullptr) amax_chunks(std::true_type{});
+  else if (sizeof(T) != 2) amax_chunks(std::false_type{});
 #pragma unroll
   for (int s = 16; s >= 1; s >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, s));
   if (lane == 0) sc.amx[warp] = amax;
@@ -231,29 +239,34 @@ BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict_
 
   int sum = 0;
   const float s = amax == 0.0f ? 0.0f : __fdiv_rn(127.0f, amax);
+  auto quantise_chunks = [&](auto has_gain) {
+    constexpr bool HG = decltype(has_gain)::value;
 #pragma unroll
-  for (int i = 0; i < MAXC; ++i) {
-    const int c = t + nt * i;
-    if (c < nchunks) {
-      uint32_t lo = 0, hi = 0;
-      if (amax != 0.0f) {
-        Chunk8<T> g;
-        if (gain != nullptr) g = gain_chunk(i, c);
-        uint32_t q[8];
+    for (int i = 0; i < MAXC; ++i) {
+      const int c = t + nt * i;
+      if (c < nchunks) {
+        uint32_t lo = 0, hi = 0;
+        if (amax != 0.0f) {
+          Chunk8<T> g;
+          if constexpr (HG) g = gain_chunk(i, c);
+          uint32_t q[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float v = ch[i].get(e);
-          const float h = gain != nullptr ? __fmul_rn(__fmul_rn(v, r), g.get(e)) : v;
-          q[e] = f32_to_s8_rne_bits(__fmul_rn(h, s));
+          for (int e = 0; e < 8; ++e) {
+            const float v = ch[i].get(e);
+            const float h = HG ? __fmul_rn(__fmul_rn(v, r), g.get(e)) : v;
+            q[e] = f32_to_s8_rne_bits(__fmul_rn(h, s));
+          }
+          lo = pack4_s8(q[0], q[1], q[2], q[3]);
+          hi = pack4_s8(q[4], q[5], q[6], q[7]);
+          sum = __dp4a(static_cast<int>(lo), 0x01010101, sum);
+          sum = __dp4a(static_cast<int>(hi), 0x01010101, sum);
         }
-        lo = pack4_s8(q[0], q[1], q[2], q[3]);
-        hi = pack4_s8(q[4], q[5], q[6], q[7]);
-        sum = __dp4a(static_cast<int>(lo), 0x01010101, sum);
-        sum = __dp4a(static_cast<int>(hi), 0x01010101, sum);
+        *reinterpret_cast<uint2*>(xq_row + 8 * c) = make_uint2(lo, hi);
       }
-      *reinterpret_cast<uint2*>(xq_row + 8 * c) = make_uint2(lo, hi);
     }
-  }
+  };
+  if (gain != nullptr) quantise_chunks(std::true_type{});
+  else quantise_chunks(std::false_type{});
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   if (lane == 0) sc.ired[warp] = sum;

@@ -248,7 +248,10 @@ def _check_linear(dev, orc, fn, M, N, K, seed=0, zero_row=None, zero_tok=None, s
 GEMV_CASES = [(1, 256, 256), (4, 256, 256), (8, 6912, 2560), (1, 2560, 6912), (3, 129, 192), (5, 1, 64),
               (2, 37, 4160), (7, 300, 640), (1, 1000, 21504), (6, 77, 8192),
               # 27B-class shapes: the deep-ring launch plan (long chunks, several slots per warp)
-              (1, 21504, 5376), (3, 21504, 5376), (2, 5376, 21504), (1, 5373, 21504)]
+              (1, 21504, 5376), (3, 21504, 5376), (2, 5376, 21504), (1, 5373, 21504),
+              # one token, large shares (whole-row slots): ragged rows and slots, 2/8/16 column
+              # segments per row, and the first K past the register budget (the item kernel again)
+              (1, 10007, 8192), (1, 3001, 32768), (1, 600, 65536), (1, 700, 65600)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMV_CASES)
@@ -299,6 +302,7 @@ FUSED_CASES = [
     (1, 21504, 5376, "bf16", False, "bf16"),   # 27B up: deep-ring plan, one token (masked fields)
     (2, 5376, 10752, "bf16", True, "f32"),     # deep-ring plan with two tokens
     (1, 21501, 5376, "bf16", True, "i32"),     # ragged last group of the last CTA
+    (1, 9000, 12288, "f32", True, "bf16"),     # one token, whole-row slots, f32 input with the norm
 ]
 
 
