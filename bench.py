@@ -119,6 +119,12 @@ def linear_bytes(lin) -> dict:
     return {"quant": quant, "product": prod, "fused": xin + w + 4 + yb, "x_in": xin, "y_out": yb, "w": w}
 
 
+def sk_units(lin) -> int:
+    """(128-row tile, 256-K step) units of the stream-K product of a linear with M <= 64 tokens."""
+    bn = 16 if lin.M <= 16 else (32 if lin.M <= 32 else 64)
+    return -(-lin.N // 128) * -(-lin.M // bn) * -(-lin.K // 256)
+
+
 def step_bytes(lins) -> int:
     """Algorithmic bytes of one step (quantisation + product of every linear);
     the same count for the fused and the two-kernel path."""
@@ -420,10 +426,20 @@ class Workload:
                   [bl.bitnet_bitlinear_gemm_workspace_bytes(l.M, l.N, l.K) for l in lins
                    if self.path == "gemm_fused"] or [0])
         self.ws = torch.zeros(wsb, dtype=torch.uint8, device=dev) if wsb else None
-        self.kernels_per_step = (1 if self.fused else 2) * len(lins)
+        # bitnet_bitlinear_gemm: the quantisation, then the stream-K product from 12 (row tile, K step)
+        # units of work per SM, else the tile product -- the library's rule, restated here only to name
+        # the product kernel
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        self.sk = [self.path == "gemm_fused" and sk_units(l) >= 12 * sms for l in lins]
+        self.kernels_per_step = (1 if self.path == "gemv_fused" else 2) * len(lins)
         self.product_kernel = {
             "gemv_fused": "gemv_kernel (fused quantisation + GEMV, bitnet_bitlinear_gemv)",
-            "gemm_fused": "gemm_sk_kernel (fused quantisation + tcgen05 stream-K, bitnet_bitlinear_gemm)",
+            "gemm_fused": ("gemm_sk_kernel (tcgen05 stream-K, after the quantisation, in bitnet_bitlinear_gemm)"
+                           if all(self.sk) else
+                           "gemm_kernel (tcgen05 tiles, after the quantisation, in bitnet_bitlinear_gemm)"
+                           if not any(self.sk) else
+                           "gemm_sk_kernel / gemm_kernel (tcgen05 stream-K or tiles per linear, after the "
+                           "quantisation, in bitnet_bitlinear_gemm)"),
             "quant_gemv": "gemv_kernel (bitnet_linear_gemv)",
             "quant_gemm": ("gemm_sk_kernel (tcgen05 stream-K, bitnet_linear_gemm)" if all(l.M <= 64 for l in lins)
                            else "gemm_kernel (tcgen05, bitnet_linear_gemm)")}[self.path]
@@ -702,7 +718,7 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
     rl = head["roofline"]
     if wl.fused and lins[0].K == 5376 and lins[0].N == 21504:
         rl["traffic"] = profiled_traffic(os.path.join(PROFILES, "gemv_decode_m1_27b_ffn.md"),
-                                         kernel_source_hash(["gemv.cuh", "quant.cuh", "ptx.cuh"]))
+                                         kernel_source_hash(["gemv1.cuh", "gemv.cuh", "quant.cuh", "ptx.cuh"]))
     unfused = head.get("unfused_step")
     if unfused is not None:
         unfused = dict(unfused, value=ws * sbytes / (unfused["ms_per_step"] / 1e3) / 1e9, unit="GB/s")
@@ -784,8 +800,9 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
             "config": {"workload": args.workload, "linears": [[l.M, l.K, l.N] for l in lins],
                        "step": {"gemv_fused": "per linear: one bitnet_bitlinear_gemv kernel (RMSNorm/absmax int8 "
                                               "quantisation of the input fused with the ternary GEMV and dequant)",
-                                "gemm_fused": "per linear: one bitnet_bitlinear_gemm kernel (quantisation fused with "
-                                              "the stream-K tensor-core product and dequant)"}.get(
+                                "gemm_fused": ("per linear: one bitnet_bitlinear_gemm call = the quantisation kernel "
+                                               "+ the tcgen05 product with dequant (stream-K from 12 units of work "
+                                               f"per SM, else tiles; stream-K per linear: {wl.sk})")}.get(
                                     wl.path, "per linear: bitnet_quant_act + ternary product with dequant"),
                        "l2": f"{wl.copies} rotated copies of every buffer ({wl.footprint_mb:.0f} MB per rotation "
                              "> 3 x 126 MB L2): inputs larger than L2, no flush",

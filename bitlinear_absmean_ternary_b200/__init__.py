@@ -58,12 +58,16 @@ def lib() -> ctypes.CDLL:
         L.bitnet_linear_gemv.restype = I
         L.bitnet_linear_gemm.argtypes = [P, P, I64, I64, P, P, P, I64, P, I, P, ctypes.c_size_t, P]
         L.bitnet_linear_gemm.restype = I
+        L.bitnet_linear_gemm_stream_k.argtypes = [P, P, I64, I64, P, P, P, I64, P, I, P, ctypes.c_size_t, P]
+        L.bitnet_linear_gemm_stream_k.restype = I
         L.bitnet_linear_gemm_workspace_bytes.argtypes = [I64, I64, I64]
         L.bitnet_linear_gemm_workspace_bytes.restype = ctypes.c_size_t
         L.bitnet_bitlinear_gemm_workspace_bytes.argtypes = [I64, I64, I64]
         L.bitnet_bitlinear_gemm_workspace_bytes.restype = ctypes.c_size_t
         L.bitnet_bitlinear_gemm.argtypes = [P, I, P, F, P, P, I64, I64, I64, P, I, P, ctypes.c_size_t, P]
         L.bitnet_bitlinear_gemm.restype = I
+        L.bitnet_bitlinear_gemm_stream_k.argtypes = [P, I, P, F, P, P, I64, I64, I64, P, I, P, ctypes.c_size_t, P]
+        L.bitnet_bitlinear_gemm_stream_k.restype = I
         L.bitnet_linear_upgate_workspace_bytes.argtypes = [I64, I64, I64]
         L.bitnet_linear_upgate_workspace_bytes.restype = ctypes.c_size_t
         L.bitnet_linear_upgate_gemm.argtypes = [P, P, P, P, I64, I64, P, P, P, I64, P, P, ctypes.c_size_t, P]
@@ -251,16 +255,18 @@ def bitnet_linear_gemm_workspace_bytes(M: int, N: int, K: int) -> int:
 
 
 def bitnet_linear_gemm(W_packed, gamma, x_q, a_scale, x_rowsum=None, y=None, out_dtype=None, workspace=None,
-                       stream_k: bool = True):
+                       stream_k=None):
     """W1.58A8 product for any M (tcgen05 tensor cores).  Returns y (M x N).
 
     workspace: a zeroed uint8 device tensor of bitnet_linear_gemm_workspace_bytes
     bytes, reused across calls on one stream (the calls leave it zeroed), or None
-    to allocate a zeroed one for this call when M <= 64.  stream_k=False passes
-    no workspace (the persistent-tile path; same results)."""
+    to allocate a zeroed one for this call when M <= 64.  stream_k: None lets the
+    library choose (stream-K from 12 units of work per SM when a workspace is
+    given), True forces stream-K (bitnet_linear_gemm_stream_k), False passes no
+    workspace (the persistent-tile path).  The results are the same."""
     torch = _torch()
     M, N, K, y = _linear_args(W_packed, gamma, x_q, a_scale, x_rowsum, y, out_dtype)
-    if not stream_k:
+    if stream_k is False:
         workspace = None
     elif workspace is None:
         nbytes = bitnet_linear_gemm_workspace_bytes(M, N, K)
@@ -268,10 +274,17 @@ def bitnet_linear_gemm(W_packed, gamma, x_q, a_scale, x_rowsum=None, y=None, out
             workspace = torch.zeros(nbytes, dtype=torch.uint8, device=x_q.device)
     _need_cuda(workspace)
     wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib().bitnet_linear_gemm(_ptr(W_packed), _ptr(gamma), N, K, _ptr(x_q), _ptr(a_scale), _ptr(x_rowsum), M,
-                                  _ptr(y), _dtype_code(y.dtype), _ptr(workspace), wsb, _stream(x_q.device))
-    _check("bitnet_linear_gemm", st)
+    fn = lib().bitnet_linear_gemm_stream_k if stream_k else lib().bitnet_linear_gemm
+    st = fn(_ptr(W_packed), _ptr(gamma), N, K, _ptr(x_q), _ptr(a_scale), _ptr(x_rowsum), M, _ptr(y),
+            _dtype_code(y.dtype), _ptr(workspace), wsb, _stream(x_q.device))
+    _check("bitnet_linear_gemm_stream_k" if stream_k else "bitnet_linear_gemm", st)
     return y
+
+
+def bitnet_linear_gemm_stream_k(W_packed, gamma, x_q, a_scale, x_rowsum=None, y=None, out_dtype=None,
+                                workspace=None):
+    """bitnet_linear_gemm with the stream-K product forced (M <= 64)."""
+    return bitnet_linear_gemm(W_packed, gamma, x_q, a_scale, x_rowsum, y, out_dtype, workspace, stream_k=True)
 
 
 def bitnet_linear_upgate_workspace_bytes(M: int, F: int, K: int) -> int:
@@ -327,12 +340,13 @@ def bitnet_bitlinear_gemm_workspace_bytes(M: int, N: int, K: int) -> int:
 
 
 def bitnet_bitlinear_gemm(x, W_packed, gamma, rms_gain=None, rms_eps: float = 1e-5, y=None, out_dtype=None,
-                          workspace=None):
-    """Fused BitLinear for 1 <= M <= 64 tokens: quantisation (with RMSNorm when
-    rms_gain is given) and the stream-K tensor-core product in one launch.
-    workspace: zeroed uint8 device tensor of bitnet_bitlinear_gemm_workspace_bytes
-    bytes, reused across calls on one stream (allocated zeroed for this call when
-    None).  Returns y (M x N)."""
+                          workspace=None, stream_k=None):
+    """BitLinear for 1 <= M <= 64 tokens: quantisation (with RMSNorm when
+    rms_gain is given) into the workspace, then the tensor-core product
+    (stream-K or tiles), two launches; stream_k=True takes the one-launch kernel
+    (quantisation inside the stream-K product).  workspace: zeroed uint8 device
+    tensor of bitnet_bitlinear_gemm_workspace_bytes bytes, reused across calls on
+    one stream (allocated zeroed for this call when None).  Returns y (M x N)."""
     torch = _torch()
     _need_cuda(x, rms_gain, W_packed, gamma, y, workspace)
     M, K = x.shape
@@ -344,11 +358,17 @@ def bitnet_bitlinear_gemm(x, W_packed, gamma, rms_gain=None, rms_eps: float = 1e
     if workspace is None:
         workspace = torch.zeros(max(1, bitnet_bitlinear_gemm_workspace_bytes(M, N, K)), dtype=torch.uint8,
                                 device=x.device)
-    st = lib().bitnet_bitlinear_gemm(_ptr(x), _dtype_code(x.dtype), _ptr(rms_gain), rms_eps, _ptr(W_packed),
-                                     _ptr(gamma), N, K, M, _ptr(y), _dtype_code(y.dtype), _ptr(workspace),
-                                     workspace.numel() * workspace.element_size(), _stream(x.device))
-    _check("bitnet_bitlinear_gemm", st)
+    fn = lib().bitnet_bitlinear_gemm_stream_k if stream_k else lib().bitnet_bitlinear_gemm
+    st = fn(_ptr(x), _dtype_code(x.dtype), _ptr(rms_gain), rms_eps, _ptr(W_packed), _ptr(gamma), N, K, M, _ptr(y),
+            _dtype_code(y.dtype), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(x.device))
+    _check("bitnet_bitlinear_gemm_stream_k" if stream_k else "bitnet_bitlinear_gemm", st)
     return y
+
+
+def bitnet_bitlinear_gemm_stream_k(x, W_packed, gamma, rms_gain=None, rms_eps: float = 1e-5, y=None,
+                                   out_dtype=None, workspace=None):
+    """bitnet_bitlinear_gemm as one launch (quantisation inside the stream-K product)."""
+    return bitnet_bitlinear_gemm(x, W_packed, gamma, rms_gain, rms_eps, y, out_dtype, workspace, stream_k=True)
 
 
 def bitnet_bitlinear_ffn_gemv(x, W_up, gamma_up, W_gate, gamma_gate, W_down, gamma_down, rms_gain_in=None,

@@ -21,11 +21,14 @@
 //     (the tile is the last segment of that CTA's range), and helpers, the
 //     later CTAs holding its other stages (for each helper the tile is its
 //     FIRST segment, so a CTA is the helper of at most one tile).  A helper
-//     stores its int32 partial tile into its own slot of the workspace and
+//     adds its int32 partial tile into the finisher's slot of the workspace
+//     with reductions at L2 (integer adds: exact and order-free, and the
+//     helpers' latencies overlap instead of adding up at the finisher) and
 //     raises its flag; the finisher, which reaches the tile last, waits for
-//     the flags of its helpers, adds their partials (integer adds: the result
-//     is bit-identical to an unsplit product), dequantises, stores y and
-//     lowers the flags again, so the workspace is all zero between calls.
+//     the flags of its helpers, reads the summed partials once (the result is
+//     bit-identical to an unsplit product), dequantises, stores y and zeroes
+//     its slot and the flags again, so the workspace is all zero between
+//     calls.
 //
 //   * Feed: the packed weights have a ring of their own (SW stages of 8 KB),
 //     freed as soon as the unpack warps have read a stage into registers, so
@@ -107,21 +110,47 @@ struct SkCfg {
   // second CTA never fits on the SM, so none waits in tcgen05.alloc.
   static constexpr int kMinSmem = 233472 / 2;
   static constexpr int kSmemBytes = kNeeded > kMinSmem ? kNeeded : kMinSmem;
-  // workspace: G flags (rounded to 256 bytes), then G partial tiles int4 [BN/4][128] (int32 [BN][128])
-  static constexpr int kPartInts = BN * kGemmBM;
+  // workspace: G flags (rounded to 256 bytes), then G accumulation slots of kSkSlotInts (this tile
+  // uses the first BN x 128 of its slot as int32 [BN][128]), zero between calls
   static_assert(kWStage % 1024 == 0 && kXStage % 1024 == 0, "stages stay 1024-byte aligned");
   static_assert(kAcol + T * kAslot <= 512 && T >= 2, "TMEM budget");
   static_assert(kNeeded <= 232448, "shared memory budget");
-  static_assert(BN == 16 || BN == 32 || BN == 64, "token tile");
+  static_assert(BN == 16 || BN == 32 || BN == 64, "token tile (at most the slot's 64)");
 };
 
 __host__ __device__ inline size_t sk_flag_bytes(int G) { return (static_cast<size_t>(G) * 4 + 255) / 256 * 256; }
+
+// Whether a product of M <= 64 tokens runs stream-K.  Every CTA pays a fixed
+// cost (the pipeline's fill, then partial tiles exchanged through L2 and the
+// finisher's wait), which a share of a few K steps does not repay: below
+// kSkMinUnitsPerCta (row tile, K step) units per SM the tile kernel, which
+// exchanges no partials, is faster (measured: the 2.5B-class block's
+// matrices, 1.4 to 7.3 units per SM, ran in 7.7 to 10.2 us on tiles against
+// 13 to 15.5 us stream-K; the 27B FFN's, 24 units per SM, in 19.3 to 21.6
+// us stream-K against 20.6 to 31 us on tiles).
+constexpr int kSkMinUnitsPerCta = 12;
+inline bool sk_preferred(int64_t M, int64_t N, int64_t K, int sms) {
+  if (M > 64) return false;
+  const int64_t bn = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+  const int64_t units = ((N + 127) / 128) * ((M + bn - 1) / bn) * ((K + 255) / 256);
+  return units >= static_cast<int64_t>(kSkMinUnitsPerCta) * sms;
+}
+
+// One accumulation slot per CTA, sized for the widest token tile whatever
+// the call's tile, so that calls of any token count can share a workspace
+// (each leaves its slots zero).
+constexpr int kSkSlotInts = 64 * kGemmBM;
+__host__ __device__ inline size_t sk_slot_bytes(int G) { return static_cast<size_t>(G) * kSkSlotInts * 4; }
 
 // CTA (of G) whose unit range [U*c/G, U*(c+1)/G) holds unit u.
 __device__ __forceinline__ int sk_cta_of(long long u, long long U, int G) {
   return static_cast<int>(((u + 1) * G - 1) / U);
 }
 
+// Integer add at L2, no result returned (the helpers' partial tiles).
+BN_DEV void red_add_gpu_u32(unsigned int* p, unsigned int v) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 BN_DEV void st_release_gpu_u32(unsigned int* p, unsigned int v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -474,13 +503,13 @@ __global__ void __launch_bounds__(kSkThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[b]);  // the accumulator may be reused
       if (kb_lo > 0) {
-        // helper: this CTA's partial of a tile finished by an earlier CTA
-        // partial tile layout int4 [BN/4][128]: thread r moves 16 bytes per access, a warp 512 contiguous bytes
-        int4* slot = reinterpret_cast<int4*>(parts + static_cast<size_t>(cta) * C::kPartInts);
+        // helper: this CTA's partial of a tile finished by an earlier CTA (the one holding the tile's
+        // first stage), added into that finisher's accumulation slot [BN][128] by integer reductions at
+        // L2 -- exact and order-free, and none of the helpers' latencies adds up at the finisher
+        unsigned int* acc = reinterpret_cast<unsigned int*>(parts) +
+                            static_cast<size_t>(sk_cta_of(t * nk, U, G)) * kSkSlotInts;
 #pragma unroll
-        for (int j4 = 0; j4 < BN / 4; ++j4)
-          slot[j4 * kGemmBM + r] = make_int4(static_cast<int>(v[4 * j4]), static_cast<int>(v[4 * j4 + 1]),
-                                             static_cast<int>(v[4 * j4 + 2]), static_cast<int>(v[4 * j4 + 3]));
+        for (int j = 0; j < BN; ++j) red_add_gpu_u32(acc + j * kGemmBM + r, v[j]);
         __threadfence();
         if (sk_epi_sync(epi_bar, ephase) && et == 0) st_release_gpu_u32(&flags[cta], 1u);
         continue;
@@ -503,15 +532,17 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         }
         sk_epi_sync(epi_bar, ephase);
         __threadfence();
-        for (int h = cta + 1; h <= last; ++h) {
-          const int4* slot = reinterpret_cast<const int4*>(parts + static_cast<size_t>(h) * C::kPartInts);
+        {
+          // the helpers' partials, already summed in this CTA's slot: one read, then the slot is
+          // zeroed again for the next call (a warp moves 128 contiguous bytes per access)
+          unsigned int* acc = reinterpret_cast<unsigned int*>(parts) + static_cast<size_t>(cta) * kSkSlotInts;
+          uint32_t pv[BN];
 #pragma unroll
-          for (int j4 = 0; j4 < BN / 4; ++j4) {
-            const int4 p = __ldcg(slot + j4 * kGemmBM + r);
-            v[4 * j4] += static_cast<uint32_t>(p.x);
-            v[4 * j4 + 1] += static_cast<uint32_t>(p.y);
-            v[4 * j4 + 2] += static_cast<uint32_t>(p.z);
-            v[4 * j4 + 3] += static_cast<uint32_t>(p.w);
+          for (int j = 0; j < BN; ++j) pv[j] = __ldcg(acc + j * kGemmBM + r);
+#pragma unroll
+          for (int j = 0; j < BN; ++j) {
+            v[j] += pv[j];
+            __stcg(acc + j * kGemmBM + r, 0u);
           }
         }
         if (et == 0)  // every thread has read the partials once the next barrier completes
@@ -543,22 +574,26 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           }
         }
       } else {
-        // dequantise and store: thread = output feature n, columns = tokens
+        // dequantise and store: thread = output feature n, columns = tokens (the output type and the
+        // token count decided once per segment, outside the store loop)
         const int n = f0 + r;
-        if (n < N) {
+        const int jn = M - m0 < BN ? M - m0 : BN;
+        auto store_all = [&](auto* out, auto conv) {
+          auto* p = out + static_cast<int64_t>(m0) * N + n;
 #pragma unroll
-          for (int j = 0; j < BN; ++j) {
-            if (m0 + j < M) {
-              const int a = static_cast<int>(v[j]) - s_rs[sb + j];
-              const int64_t o = static_cast<int64_t>(m0 + j) * N + n;
-              if (y_dtype == 2) {
-                static_cast<int32_t*>(y)[o] = a;
-              } else {
-                const float val = __fmul_rn(__fmul_rn(__int2float_rn(a), gamma), s_a[sb + j]);
-                if (y_dtype == 0) static_cast<float*>(y)[o] = val;
-                else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(val);
-              }
-            }
+          for (int j = 0; j < BN; ++j)
+            if (j < jn) p[static_cast<int64_t>(j) * N] = conv(static_cast<int>(v[j]) - s_rs[sb + j], j);
+        };
+        if (n < N) {
+          if (y_dtype == 2) {
+            store_all(static_cast<int32_t*>(y), [](int a, int) { return a; });
+          } else if (y_dtype == 0) {
+            store_all(static_cast<float*>(y),
+                      [&](int a, int j) { return __fmul_rn(__fmul_rn(__int2float_rn(a), gamma), s_a[sb + j]); });
+          } else {
+            store_all(static_cast<__nv_bfloat16*>(y), [&](int a, int j) {
+              return __float2bfloat16_rn(__fmul_rn(__fmul_rn(__int2float_rn(a), gamma), s_a[sb + j]));
+            });
           }
         }
       }

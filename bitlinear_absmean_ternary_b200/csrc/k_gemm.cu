@@ -137,14 +137,12 @@ cudaError_t launch_gemm_bn(const uint8_t* Wp, const float* gamma, int N, int K, 
   return launch_gemm_t<BN, S, false>(mx, mw, gamma, a, rs, M, N, K, y, yd, s);
 }
 
-// Token tile of the stream-K kernel for M <= 64 tokens.
-int sk_bn(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
-
 // Workspace of the stream-K kernel on the current device: a flag per CTA
-// (one CTA per SM at most) and a partial int32 tile [BN][128] per CTA.
-size_t sk_workspace_bytes(int64_t M) {
+// (one CTA per SM at most) and an accumulation slot per CTA, the same for
+// every token count M <= 64.
+size_t sk_workspace_bytes(int64_t) {
   const int G = sm_count();
-  return sk_flag_bytes(G) + static_cast<size_t>(G) * sk_bn(M) * kGemmBM * 4;
+  return sk_flag_bytes(G) + sk_slot_bytes(G);
 }
 
 template <int BN, bool U8, bool GATE>
@@ -236,14 +234,21 @@ size_t bitnet_linear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return sk_workspace_bytes(M);
 }
 
-bitnet_status bitnet_linear_gemm(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, const int8_t* x_q,
-                                 const float* a_scale, const int32_t* x_rowsum, int64_t M, void* y, int y_dtype,
-                                 void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The product with the stream-K kernel forced (force_sk), or chosen by sk_preferred.
+bitnet_status linear_gemm(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, const int8_t* x_q,
+                          const float* a_scale, const int32_t* x_rowsum, int64_t M, void* y, int y_dtype,
+                          void* workspace, size_t workspace_bytes, void* stream, bool force_sk) {
   const bitnet_status st = check_linear(W_packed, gamma, N, K, x_q, a_scale, x_rowsum, M, y, y_dtype);
   if (st != BITNET_OK) return st;
   if (!aligned(workspace, 16)) return BITNET_ERR_INVALID_ARG;
-  const bool stream_k = workspace != nullptr && M <= 64;
-  if (stream_k && workspace_bytes < sk_workspace_bytes(M)) return BITNET_ERR_INVALID_ARG;
+  if (force_sk && (workspace == nullptr || M > 64)) return workspace == nullptr ? BITNET_ERR_INVALID_ARG
+                                                                                 : BITNET_ERR_UNSUPPORTED_SHAPE;
+  if (workspace != nullptr && M <= 64 && workspace_bytes < sk_workspace_bytes(M)) return BITNET_ERR_INVALID_ARG;
+  const bool stream_k = force_sk || (workspace != nullptr && sk_preferred(M, N, K, sm_count()));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int n = static_cast<int>(N), k = static_cast<int>(K), m = static_cast<int>(M);
   cudaError_t e;
@@ -261,6 +266,25 @@ bitnet_status bitnet_linear_gemm(const uint8_t* W_packed, const float* gamma, in
     e = launch_gemm_bn<128, 4>(W_packed, gamma, n, k, x_q, a_scale, x_rowsum, m, y, y_dtype, s);
   }
   return from_cuda(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+bitnet_status bitnet_linear_gemm(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, const int8_t* x_q,
+                                 const float* a_scale, const int32_t* x_rowsum, int64_t M, void* y, int y_dtype,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  return linear_gemm(W_packed, gamma, N, K, x_q, a_scale, x_rowsum, M, y, y_dtype, workspace, workspace_bytes, stream,
+                     false);
+}
+
+bitnet_status bitnet_linear_gemm_stream_k(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K,
+                                          const int8_t* x_q, const float* a_scale, const int32_t* x_rowsum, int64_t M,
+                                          void* y, int y_dtype, void* workspace, size_t workspace_bytes,
+                                          void* stream) {
+  return linear_gemm(W_packed, gamma, N, K, x_q, a_scale, x_rowsum, M, y, y_dtype, workspace, workspace_bytes, stream,
+                     true);
 }
 
 }  // extern "C"

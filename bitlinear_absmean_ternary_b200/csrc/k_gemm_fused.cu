@@ -1,6 +1,12 @@
-// Host side of bitnet_bitlinear_gemm: the fused BitLinear for decode-sized
-// batches (M <= 64) -- quantisation of the token rows (with the optional
-// RMSNorm) and the stream-K tensor-core product in one launch (gemm_sk.cuh).
+// Host side of bitnet_bitlinear_gemm: the BitLinear for decode-sized batches
+// (M <= 64) -- quantisation of the token rows (with the optional RMSNorm)
+// into the workspace, then bitnet_linear_gemm's product (two launches) -- and
+// of bitnet_bitlinear_gemm_stream_k: the same in ONE launch, the quantisation
+// inside the stream-K product (gemm_sk.cuh).  Measured on B200, the one-launch
+// kernel was the slower of the two (27B FFN at M = 16: 23.6 and 26.7 us per
+// linear against 21.2 and 25.2 us; its grid barrier costs more than the kernel
+// boundary, which programmatic dependent launch overlaps with the product's
+// weight prefetch), so the entry point without a suffix takes two launches.
 #include "host_common.h"
 #include "gemm_sk.cuh"
 
@@ -8,8 +14,6 @@ namespace {
 
 using namespace bitnet;
 using namespace bitnet_host;
-
-int fq_bn(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 
 // Workspace layout: stream-K flags and partial tiles (as bitnet_linear_gemm),
 // the grid barrier's two words, the scales, the row sums, x_q.
@@ -21,7 +25,7 @@ FqLayout fq_layout(int64_t M, int64_t K) {
   const int G = sm_count();
   auto r256 = [](size_t b) { return (b + 255) / 256 * 256; };
   FqLayout L;
-  L.bar = sk_flag_bytes(G) + static_cast<size_t>(G) * fq_bn(M) * kGemmBM * 4;
+  L.bar = sk_flag_bytes(G) + sk_slot_bytes(G);
   L.a = L.bar + 256;
   L.rs = L.a + r256(static_cast<size_t>(M) * 4);
   L.xq = L.rs + r256(static_cast<size_t>(M) * 4);
@@ -92,9 +96,14 @@ size_t bitnet_bitlinear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return fq_layout(M, K).total;
 }
 
-bitnet_status bitnet_bitlinear_gemm(const void* x, int x_dtype, const void* rms_gain, float rms_eps,
-                                    const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, int64_t M,
-                                    void* y, int y_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The fused BitLinear with the one-launch stream-K kernel forced (force_sk), or chosen by sk_preferred.
+bitnet_status bitlinear_gemm(const void* x, int x_dtype, const void* rms_gain, float rms_eps,
+                             const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, int64_t M, void* y,
+                             int y_dtype, void* workspace, size_t workspace_bytes, void* stream, bool force_sk) {
   if (x == nullptr || W_packed == nullptr || gamma == nullptr || y == nullptr || workspace == nullptr)
     return BITNET_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(rms_gain, 16) || !aligned(W_packed, 16) || !aligned(y, 16) ||
@@ -109,11 +118,41 @@ bitnet_status bitnet_bitlinear_gemm(const void* x, int x_dtype, const void* rms_
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int n = static_cast<int>(N), k = static_cast<int>(K), m = static_cast<int>(M);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (!force_sk) {
+    // the quantisation into the workspace, then bitnet_linear_gemm's product with the rest of the
+    // workspace (stream-K or tiles): two launches, chained by programmatic dependent launch
+    const FqLayout L = fq_layout(M, K);
+    int8_t* xq = reinterpret_cast<int8_t*>(ws + L.xq);
+    float* a = reinterpret_cast<float*>(ws + L.a);
+    int32_t* rs = reinterpret_cast<int32_t*>(ws + L.rs);
+    const bitnet_status st = bitnet_quant_act(x, x_dtype, M, K, rms_gain, rms_eps, xq, a, rs, stream);
+    if (st != BITNET_OK) return st;
+    return bitnet_linear_gemm(W_packed, gamma, N, K, xq, a, rs, M, y, y_dtype, ws, L.bar, stream);
+  }
   const cudaError_t e =
       x_dtype == BITNET_BF16
           ? launch_fq<__nv_bfloat16>(x, rms_gain, rms_eps, W_packed, gamma, n, k, m, y, y_dtype, ws, s)
           : launch_fq<float>(x, rms_gain, rms_eps, W_packed, gamma, n, k, m, y, y_dtype, ws, s);
   return from_cuda(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+bitnet_status bitnet_bitlinear_gemm(const void* x, int x_dtype, const void* rms_gain, float rms_eps,
+                                    const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, int64_t M,
+                                    void* y, int y_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  return bitlinear_gemm(x, x_dtype, rms_gain, rms_eps, W_packed, gamma, N, K, M, y, y_dtype, workspace,
+                        workspace_bytes, stream, false);
+}
+
+bitnet_status bitnet_bitlinear_gemm_stream_k(const void* x, int x_dtype, const void* rms_gain, float rms_eps,
+                                             const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K,
+                                             int64_t M, void* y, int y_dtype, void* workspace,
+                                             size_t workspace_bytes, void* stream) {
+  return bitlinear_gemm(x, x_dtype, rms_gain, rms_eps, W_packed, gamma, N, K, M, y, y_dtype, workspace,
+                        workspace_bytes, stream, true);
 }
 
 }  // extern "C"

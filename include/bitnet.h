@@ -206,14 +206,16 @@ size_t bitnet_linear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *
  * workspace [in,out] device memory of at least
  *           bitnet_linear_gemm_workspace_bytes(M, N, K) bytes, 16-byte
- *           aligned, or NULL.  With M <= 64 and a workspace, the product
- *           runs "stream-K": every SM takes an equal share of the (row tile,
- *           K step) work and partial tiles cut between SMs are added
- *           exactly in int32 through the workspace, so decode-sized batches
- *           stream the packed weights at HBM rate.  Zero the workspace before
- *           its first use (e.g. cudaMemset): its first bytes are flags that
- *           must start at zero, and every call leaves them zero again (the
- *           rest is scratch that every call overwrites before reading).  Two calls that may run at the same time (on two
+ *           aligned, or NULL.  With M <= 64, a workspace, and at least 12
+ *           (128-row tile, 256-K step) units of work per SM, the product
+ *           runs "stream-K": every SM takes an equal share of the units and
+ *           partial tiles cut between SMs are added exactly in int32 through
+ *           the workspace, so decode-sized batches stream the packed weights
+ *           on every SM (smaller products run on tiles: their fixed cost is
+ *           lower).  Zero the workspace
+ *           before its first use (e.g. cudaMemset): it holds flags and
+ *           partial-tile accumulators that must start at zero, and every
+ *           call leaves them zero again.  Two calls that may run at the same time (on two
  *           streams) must not share a workspace.  If a call reports
  *           BITNET_ERR_TIMEOUT through bitnet_get_device_status, zero the
  *           workspace again before reusing it.  The stream-K launch
@@ -233,6 +235,18 @@ bitnet_status bitnet_linear_gemm(const uint8_t* W_packed, const float* gamma, in
                                  void* stream);
 
 /*
+ * bitnet_linear_gemm with the stream-K product forced for any size (the
+ * automatic choice takes it only from 12 units of work per SM).  Same
+ * arguments, results and errors; the workspace is required
+ * (BITNET_ERR_INVALID_ARG without one) and M must be at most 64
+ * (BITNET_ERR_UNSUPPORTED_SHAPE otherwise).
+ */
+bitnet_status bitnet_linear_gemm_stream_k(const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K,
+                                          const int8_t* x_q, const float* a_scale, const int32_t* x_rowsum, int64_t M,
+                                          void* y, int y_dtype, void* workspace, size_t workspace_bytes,
+                                          void* stream);
+
+/*
  * Bytes of workspace bitnet_bitlinear_gemm uses on the CURRENT device: the
  * stream-K flags and partial tiles of bitnet_linear_gemm, 256 bytes of grid
  * barrier, and the quantised rows, scales and row sums; 0 for M outside
@@ -241,14 +255,18 @@ bitnet_status bitnet_linear_gemm(const uint8_t* W_packed, const float* gamma, in
 size_t bitnet_bitlinear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 /*
- * Fused BitLinear for decode-sized batches (1 <= M <= 64 tokens):
- * bitnet_quant_act followed by bitnet_linear_gemm's stream-K product in one
- * kernel launch (the four BitLinear steps of the comrad404.com review,
- * section "Метод", in one pass).  The first CTAs quantise one token row each
+ * BitLinear for decode-sized batches (1 <= M <= 64 tokens): bitnet_quant_act
+ * into the workspace, then bitnet_linear_gemm's product with the rest of the
+ * workspace (stream-K, or tiles for a small product), as two launches chained
+ * by programmatic dependent launch (the four BitLinear steps of the
+ * comrad404.com review, section "Метод").  bitnet_bitlinear_gemm_stream_k
+ * does the same in ONE launch: the first CTAs quantise one token row each
  * (same arithmetic and summation order as bitnet_quant_act) into the
- * workspace while every CTA already streams its share of the packed weights;
- * a grid barrier in the workspace then releases the product.  The results
- * are identical to the two calls.
+ * workspace while every CTA already streams its share of the packed weights,
+ * and a grid barrier in the workspace then releases the stream-K product;
+ * measured on B200 that launch is the slower one (its grid barrier costs more
+ * than the kernel boundary it removes).  The results are identical either way
+ * and to the two public calls.
  *
  * x, x_dtype, rms_gain, rms_eps   as bitnet_quant_act (K <= 32768 bf16, 16384 f32).
  * W_packed, gamma, N, K, y, y_dtype   as bitnet_linear_gemm.
@@ -264,6 +282,15 @@ size_t bitnet_bitlinear_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 bitnet_status bitnet_bitlinear_gemm(const void* x, int x_dtype, const void* rms_gain, float rms_eps,
                                     const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, int64_t M,
                                     void* y, int y_dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * bitnet_bitlinear_gemm as ONE launch (quantisation inside the stream-K
+ * product, see above), at any size.  Same arguments, results and errors.
+ */
+bitnet_status bitnet_bitlinear_gemm_stream_k(const void* x, int x_dtype, const void* rms_gain, float rms_eps,
+                                             const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K,
+                                             int64_t M, void* y, int y_dtype, void* workspace,
+                                             size_t workspace_bytes, void* stream);
 
 /*
  * Bytes of workspace bitnet_linear_upgate_gemm uses on the CURRENT device

@@ -115,17 +115,15 @@ def test_linear_rejects_bad_arguments(L, name):
 
 
 def test_gemm_workspace_bytes(L):
-    # one flag per SM (rounded to 256 bytes) and one int32 tile of 128 rows x BN tokens per SM
+    # one flag per SM (rounded to 256 bytes) and one int32 slot of 128 rows x 64 tokens per SM, the same
+    # for every M <= 64 (calls of different token counts share one workspace)
     sms = [bl.bitnet_linear_gemm_workspace_bytes(m, 256, 256) for m in (1, 16, 17, 32, 33, 64)]
-    assert sms[0] == sms[1] and sms[2] == sms[3] and sms[4] == sms[5]
+    assert len(set(sms)) == 1
     assert sms[0] > 0 and sms[0] % 256 == 0
-    per_sm_16 = sms[0]
-    # BN = 16, 32, 64: the partial tiles double with BN, the flags do not
-    assert sms[2] - sms[0] == sms[4] - sms[2] - (sms[2] - sms[0])
     assert bl.bitnet_linear_gemm_workspace_bytes(65, 256, 256) == 0
     assert bl.bitnet_linear_gemm_workspace_bytes(0, 256, 256) == 0
     assert bl.bitnet_linear_gemm_workspace_bytes(8, 256, 100) == 0
-    assert per_sm_16 >= 16 * 128 * 4
+    assert sms[0] >= 64 * 128 * 4
 
 
 def test_upgate_rejects_bad_arguments(L):

@@ -131,6 +131,9 @@ QUANT_CASES = [
     (600, 6144, "normal", 0.01, 20.0, "bf16", True),     # 24 chunks per lane, the most a warp holds
     (513, 6080, "normal", 0.0, 1.0, "bf16", False),      # 760 chunks: lanes own 23 or 24
     (600, 6912, "normal", 0.01, 20.0, "bf16", True),     # K above 6144: a CTA per row again
+    (520, 6208, "normal", 0.0, 1.0, "bf16", True),       # the first K past the warp kernel's registers
+    (600, 21504, "normal", 0.005, 30.0, "bf16", True),   # the 27B down projection's input
+    (513, 32768, "student_t4", 0.0, 1.0, "bf16", False),  # the longest bf16 row
     (777, 64, "normal", 0.0, 1.0, "bf16", True),         # 8 chunks: 24 lanes own none
     (640, 1344, "student_t4", 0.0, 1.0, "bf16", False),
     (2048, 5376, "normal", 0.005, 30.0, "bf16", True),
@@ -177,10 +180,11 @@ def test_quant_edge_tokens(dev, orc):
 
 def test_quant_edge_tokens_many_rows(dev, orc):
     """The same edge rows among 640 bf16 tokens, where one warp quantises each
-    row: zero, one-hot, exact ties after scaling, huge, tiny and a row whose
-    maximum sits in its last chunk (held by lane 31 for K = 2560 and 6144)."""
+    row (a CTA per row for K = 21504): zero, one-hot, exact ties after
+    scaling, huge, tiny and a row whose maximum sits in its last chunk (held
+    by lane 31 for K = 2560 and 6144)."""
     import torch
-    for K in (128, 2560, 6144):
+    for K in (128, 2560, 6144, 21504):
         x = synth.activations(640, K, 5, 2, "normal", 0.0, 1.0, "bf16")
         x[0] = 0.0
         x[1] = 0.0
@@ -441,9 +445,10 @@ SK_CASES = [(1, 128, 64), (16, 21504, 5376), (16, 5376, 21504), (64, 3840, 2560)
 
 @pytest.mark.parametrize("M,N,K", SK_CASES)
 def test_gemm_stream_k_matches_tiles_and_oracle(dev, orc, M, N, K):
-    """Stream-K (equal work per SM, partial tiles added through the workspace)
-    against the persistent-tile path and the oracle, with one workspace reused
-    by every call (the calls must leave its flags zero)."""
+    """Stream-K (equal work per SM, partial tiles added through the workspace;
+    forced at every size) against the persistent-tile path, the automatic
+    choice and the oracle, with one workspace reused by every call (the calls
+    must leave its flags and accumulation slots zero)."""
     import torch
     rng = np.random.default_rng(M + N + K)
     q = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
@@ -459,9 +464,10 @@ def test_gemm_stream_k_matches_tiles_and_oracle(dev, orc, M, N, K):
     acc_r, y_r = orc.bitlinear_sampled(packed, gamma, K, xq, a, ms, ns)
     for rowsum in (RS, None):
         for out in (torch.int32, torch.float32, torch.bfloat16):
-            y_sk = bl.bitnet_linear_gemm(P, G, XQ, A, rowsum, out_dtype=out, workspace=ws)
+            y_sk = bl.bitnet_linear_gemm_stream_k(P, G, XQ, A, rowsum, out_dtype=out, workspace=ws)
             y_t = bl.bitnet_linear_gemm(P, G, XQ, A, rowsum, out_dtype=out, stream_k=False)
-            assert torch.equal(y_sk, y_t)
+            y_auto = bl.bitnet_linear_gemm(P, G, XQ, A, rowsum, out_dtype=out, workspace=ws)
+            assert torch.equal(y_sk, y_t) and torch.equal(y_sk, y_auto)
             if out == torch.int32:
                 np.testing.assert_array_equal(y_sk.cpu().numpy()[ms, ns], acc_r)
             elif out == torch.float32:
@@ -472,6 +478,7 @@ def test_gemm_stream_k_matches_tiles_and_oracle(dev, orc, M, N, K):
     torch.cuda.synchronize()
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     assert int(ws[:4 * sms].view(torch.int32).abs().sum()) == 0, "flags left raised"
+    assert int(ws.view(torch.int32).abs().sum()) == 0, "accumulation slots left non-zero"
     assert bl.bitnet_get_device_status() == bl.BITNET_OK
 
 
@@ -492,12 +499,12 @@ def test_gemm_stream_k_in_a_cuda_graph(dev, orc):
     ws = torch.zeros(bl.bitnet_linear_gemm_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
     ys = [torch.empty((M, N), dtype=torch.int32, device=dev) for _ in range(3)]
     s = torch.cuda.Stream(dev)
-    bl.bitnet_linear_gemm(P, G, XQ, A, RS, y=ys[0], workspace=ws)  # first call outside the capture
+    bl.bitnet_linear_gemm_stream_k(P, G, XQ, A, RS, y=ys[0], workspace=ws)  # first call outside the capture
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
         for y in ys:
-            bl.bitnet_linear_gemm(P, G, XQ, A, RS, y=y, workspace=ws)
+            bl.bitnet_linear_gemm_stream_k(P, G, XQ, A, RS, y=y, workspace=ws)
     for _ in range(3):
         for y in ys:
             y.zero_()
@@ -589,7 +596,7 @@ def test_fused_bitlinear_gemm_parity(dev, orc, M, N, K, dt, norm, yt):
     xd = _x_dev(x, dt, dev)
     gd = None if g is None else _x_dev(g, dt, dev)
     ws = torch.zeros(bl.bitnet_bitlinear_gemm_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
-    y = bl.bitnet_bitlinear_gemm(xd, P, G, gd, EPS_RMS, out_dtype=out, workspace=ws)
+    y = bl.bitnet_bitlinear_gemm_stream_k(xd, P, G, gd, EPS_RMS, out_dtype=out, workspace=ws)
     if M * N * K <= 64 * 3840 * 2560:
         acc_r, y_r = orc.bitlinear(p_ref, g_ref, K, xq_r, a_r)
         got = y.cpu().numpy() if yt != "bf16" else None
@@ -611,7 +618,7 @@ def test_fused_bitlinear_gemm_parity(dev, orc, M, N, K, dt, norm, yt):
     xq, a, rs = bl.bitnet_quant_act(xd, gd, EPS_RMS, want_rowsum=True)
     y2 = bl.bitnet_linear_gemm(P, G, xq, a, rs, out_dtype=out)
     assert torch.equal(y, y2)
-    y3 = bl.bitnet_bitlinear_gemm(xd, P, G, gd, EPS_RMS, out_dtype=out, workspace=ws)
+    y3 = bl.bitnet_bitlinear_gemm(xd, P, G, gd, EPS_RMS, out_dtype=out, workspace=ws)  # the automatic choice
     assert torch.equal(y, y3)
     assert bl.bitnet_get_device_status() == bl.BITNET_OK
 
@@ -634,13 +641,13 @@ def test_fused_bitlinear_gemm_shares_a_workspace_across_shapes_and_graph_replays
         ref = bl.bitnet_linear_gemm(P, G, xq, a, rs, out_dtype=torch.int32)
         cases.append((xd, gd, P, G, ref, torch.empty_like(ref)))
     for xd, gd, P, G, ref, y in cases:
-        bl.bitnet_bitlinear_gemm(xd, P, G, gd, EPS_RMS, y=y, workspace=ws)
+        bl.bitnet_bitlinear_gemm_stream_k(xd, P, G, gd, EPS_RMS, y=y, workspace=ws)
         assert torch.equal(y, ref)
     s = torch.cuda.Stream(dev)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=s):
         for xd, gd, P, G, ref, y in cases:
-            bl.bitnet_bitlinear_gemm(xd, P, G, gd, EPS_RMS, y=y, workspace=ws)
+            bl.bitnet_bitlinear_gemm_stream_k(xd, P, G, gd, EPS_RMS, y=y, workspace=ws)
     for _ in range(3):
         for *_, y in cases:
             y.zero_()
