@@ -7,7 +7,9 @@ One step = one pass of the whole hot path over one batch: for every linear
 of the workload, the RMSNorm/absmax int8 quantisation of its input and the
 W1.58A8 product with dequant epilogue.  Decode shapes (M <= 8) run it as one
 kernel per linear (bitnet_bitlinear_gemv, quantisation fused into the GEMV);
-larger batches run bitnet_quant_act + the tcgen05 GEMM.  Weight packing
+batches of up to 64 tokens run bitnet_bitlinear_gemm (the quantisation, then
+the stream-K or tile tcgen05 product); larger batches bitnet_quant_act + the
+tcgen05 GEMM.  Weight packing
 (absmean ternarisation) is the offline step: it runs once before timing and
 is reported separately under "stages".
 
@@ -117,6 +119,13 @@ def linear_bytes(lin) -> dict:
     w = lin.N * lin.K // 4
     prod = w + lin.M * lin.K + 8 * lin.M + 4 + yb
     return {"quant": quant, "product": prod, "fused": xin + w + 4 + yb, "x_in": xin, "y_out": yb, "w": w}
+
+
+def gemv1_used(lin, sms: int = 148) -> bool:
+    """Whether the decode GEMV of a linear runs the one-token whole-row-slot kernel: one token, more than 64 KB
+    of packed weights per SM, K within its register budget -- the library's rule, restated to name the kernel."""
+    rows = -(-lin.N // min(lin.N, sms))
+    return lin.M == 1 and rows * (lin.K // 4) > 64 * 1024 and lin.K <= 65536
 
 
 def sk_units(lin) -> int:
@@ -433,7 +442,9 @@ class Workload:
         self.sk = [self.path == "gemm_fused" and sk_units(l) >= 12 * sms for l in lins]
         self.kernels_per_step = (1 if self.path == "gemv_fused" else 2) * len(lins)
         self.product_kernel = {
-            "gemv_fused": "gemv_kernel (fused quantisation + GEMV, bitnet_bitlinear_gemv)",
+            "gemv_fused": ("gemv1_kernel (one token, whole-row slots; fused quantisation + GEMV, "
+                           "bitnet_bitlinear_gemv)" if all(gemv1_used(l) for l in lins) else
+                           "gemv_kernel (fused quantisation + GEMV, bitnet_bitlinear_gemv)"),
             "gemm_fused": ("gemm_sk_kernel (tcgen05 stream-K, after the quantisation, in bitnet_bitlinear_gemm)"
                            if all(self.sk) else
                            "gemm_kernel (tcgen05 tiles, after the quantisation, in bitnet_bitlinear_gemm)"
