@@ -127,9 +127,15 @@ def _check(fn: str, status: int) -> None:
 
 # ----------------------------------------------------------------- marshalling
 
+_torch_mod = None
+
+
 def _torch():
-    import torch
-    return torch
+    global _torch_mod
+    if _torch_mod is None:
+        import torch
+        _torch_mod = torch
+    return _torch_mod
 
 
 def _ptr(t) -> Optional[int]:
@@ -137,7 +143,11 @@ def _ptr(t) -> Optional[int]:
 
 
 def _stream(device) -> int:
+    """The current CUDA stream of `device` as a raw handle (the stream a torch user is launching on)."""
     torch = _torch()
+    raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+    if raw is not None and device.index is not None:
+        return raw(device.index)  # no Stream object built per call
     return torch.cuda.current_stream(device).cuda_stream
 
 

@@ -112,7 +112,11 @@ bool gemv1_plan(int N, int K, bool xs, Gemv1Plan& p) {
   while (p.nslots > 1 && gemv1_smem_bytes(K, xs, slot_bytes, p.nslots, p.rows_max, p.S) > smem_max) --p.nslots;
   p.smem = gemv1_smem_bytes(K, xs, slot_bytes, p.nslots, p.rows_max, p.S);
   if (p.smem > smem_max) return false;
-  p.l2_prefetch = static_cast<int64_t>(p.rows_max) * B > static_cast<int64_t>(p.nslots) * slot_bytes ? 1 : 0;
+#ifndef BITNET_GEMV1_L2_PREFETCH
+#define BITNET_GEMV1_L2_PREFETCH 1
+#endif
+  p.l2_prefetch = BITNET_GEMV1_L2_PREFETCH &&
+                  static_cast<int64_t>(p.rows_max) * B > static_cast<int64_t>(p.nslots) * slot_bytes;
   return true;
 }
 
