@@ -146,8 +146,9 @@ def _stream(device) -> int:
     """The current CUDA stream of `device` as a raw handle (the stream a torch user is launching on)."""
     torch = _torch()
     raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
-    if raw is not None and device.index is not None:
-        return raw(device.index)  # no Stream object built per call
+    idx = device if isinstance(device, int) else getattr(device, "index", None)
+    if raw is not None and idx is not None:
+        return raw(idx)  # no Stream object built per call
     return torch.cuda.current_stream(device).cuda_stream
 
 

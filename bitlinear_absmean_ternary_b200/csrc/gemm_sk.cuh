@@ -196,9 +196,12 @@ BN_DEV unsigned int atom_add_acq_rel_gpu_u32(unsigned int* p, unsigned int v) {
 }
 
 // Waits (bounded) until the grid barrier's generation differs from gen0.
+// Polls back off briefly (__nanosleep), so that the hundreds of waiting
+// threads leave the word's L2 line to the arrivals.
 BN_DEV bool sk_wait_generation(const unsigned int* gen, unsigned int gen0) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1; ld_acquire_gpu_u32(gen) == gen0; ++i) {
+    __nanosleep(64);
     if ((i & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
       flag_timeout();
       return false;
@@ -522,6 +525,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           const uint64_t t0 = global_timer_ns();
           for (int h = cta + 1; h <= last && ok; ++h) {
             for (uint32_t i = 1; ld_acquire_gpu_u32(&flags[h]) == 0u; ++i) {
+              __nanosleep(64);
               if ((i & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
                 flag_timeout();
                 ok = false;
