@@ -53,31 +53,43 @@ constexpr int kGemv1MaxSlots = 8;     // ring slots (at most)
 constexpr int kGemv1BarBytes = 256;   // full and empty barriers, refill elections, issue counts
 
 // Dynamic shared memory of gemv1_kernel: ring, barrier block, the row sums
-// per column segment (S x rows_max) and (FUSED) x_q.
-__host__ __device__ constexpr int gemv1_acc_bytes(int rows_max, int S) { return ((S * rows_max * 4 + 15) / 16) * 16; }
-__host__ __device__ constexpr int gemv1_smem_bytes(int K, bool xs, int slot_bytes, int nslots, int rows_max, int S) {
-  return nslots * slot_bytes + kGemv1BarBytes + gemv1_acc_bytes(rows_max, S) + (xs ? K : 0);
+// per column segment (S x rows_max, twice with GATE) and (FUSED) x_q.
+__host__ __device__ constexpr int gemv1_acc_bytes(int rows_max, int S, bool gate = false) {
+  return (((gate ? 2 : 1) * S * rows_max * 4 + 15) / 16) * 16;
+}
+__host__ __device__ constexpr int gemv1_smem_bytes(int K, bool xs, int slot_bytes, int nslots, int rows_max, int S,
+                                                  bool gate = false) {
+  return nslots * slot_bytes + kGemv1BarBytes + gemv1_acc_bytes(rows_max, S, gate) + (xs ? K : 0);
 }
 
 // NWARPS: 16 (two CTAs per SM, so that consecutive launches overlap) or 32
 // (one CTA per SM with a deeper ring).
+// GATE: the FFN's up and gate projections at once (Wp = W_up, Wp2 = W_gate,
+// the same N x K shape): a slot holds R rows of W_up then the same R rows of
+// W_gate, a pass takes up row r and gate row r against the same x_q
+// registers, and the epilogue writes h = bf16(RN32(RN32(r*r)*u)), r = g if
+// g > 0 else +0 (u, g dequantised as the plain product's fp32 output) to y
+// (bf16, M = 1 x N) -- the squared-ReLU gate of the FFN (inferownia.pl,
+// "BitNet b1.58: era 1-bitowych LLM-ów", "Zrób to sam"; kripta.biz 2B4T news).
 // NP: word pairs per lane (segments of at most 64 * NP words).  S: column
 // segments per row (a power of two <= 16; a segment is ceil(K/16 / S)
 // words rounded up to even); R: rows per slot; nslots: ring depth; rows_max
 // = ceil(N / gridDim.x); l2_prefetch: request the part of the CTA's range
 // beyond the ring into L2 up front.
-template <bool U8, int NP, int NWARPS, bool FUSED = false, typename T = float, int MAXC = 1>
+template <bool U8, int NP, int NWARPS, bool FUSED = false, typename T = float, int MAXC = 1, bool GATE = false>
 __global__ void __launch_bounds__(NWARPS * 32, 1024 / (NWARPS * 32))
-    gemv1_kernel(const uint8_t* __restrict__ Wp, const float* __restrict__ gamma_ptr, int N, int K,
+    gemv1_kernel(const uint8_t* __restrict__ Wp, const float* __restrict__ gamma_ptr,
+                 const uint8_t* __restrict__ Wp2, const float* __restrict__ gamma2_ptr, int N, int K,
                  const int8_t* __restrict__ xq, const float* __restrict__ a_scale,
                  const int32_t* __restrict__ rowsum, const T* __restrict__ xin, const T* __restrict__ gain,
                  float rms_eps, void* __restrict__ y, int y_dtype, int S, int R, int nslots, int rows_max,
                  int l2_prefetch) {
   static_assert(!FUSED || U8, "the fused kernel computes the row sum of x_q");
+  static_assert(!GATE || U8, "the gated kernel takes the row sum of x_q");
   extern __shared__ __align__(1024) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int B = K >> 2;  // bytes per packed row
-  const int slot_bytes = R * B;
+  const int slot_bytes = (GATE ? 2 : 1) * R * B;  // GATE: R up rows, then the same R gate rows
   uint8_t* ring = smem;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + nslots * slot_bytes);
   uint64_t* empty = full + kGemv1MaxSlots;
@@ -85,13 +97,14 @@ __global__ void __launch_bounds__(NWARPS * 32, 1024 / (NWARPS * 32))
   unsigned int* issued = elect + kGemv1MaxSlots;
   int* failed = reinterpret_cast<int*>(issued + kGemv1MaxSlots);
   int* accs = reinterpret_cast<int*>(smem + nslots * slot_bytes + kGemv1BarBytes);
-  uint8_t* xs = smem + nslots * slot_bytes + kGemv1BarBytes + gemv1_acc_bytes(rows_max, S);
+  uint8_t* xs = smem + nslots * slot_bytes + kGemv1BarBytes + gemv1_acc_bytes(rows_max, S, GATE);
 
   const int64_t row_lo = static_cast<int64_t>(N) * blockIdx.x / gridDim.x;
   const int64_t row_hi = static_cast<int64_t>(N) * (blockIdx.x + 1) / gridDim.x;
   const int nrows = static_cast<int>(row_hi - row_lo);
   const int nsl = (nrows + R - 1) / R;  // slots of this CTA
   const uint8_t* wbase = Wp + row_lo * B;
+  const uint8_t* wbase2 = GATE ? Wp2 + row_lo * B : nullptr;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < nslots; ++s) {
@@ -113,15 +126,17 @@ __global__ void __launch_bounds__(NWARPS * 32, 1024 / (NWARPS * 32))
     const int nr = nrows - r0 < R ? nrows - r0 : R;
     const uint32_t bytes = static_cast<uint32_t>(nr) * static_cast<uint32_t>(B);
     issued[s] += 1u;
-    mbar_arrive_expect_tx(&full[s], bytes);
+    mbar_arrive_expect_tx(&full[s], GATE ? 2 * bytes : bytes);
     bulk_copy_g2s(ring + s * slot_bytes, wbase + static_cast<int64_t>(r0) * B, bytes, &full[s], policy);
+    if constexpr (GATE)
+      bulk_copy_g2s(ring + s * slot_bytes + R * B, wbase2 + static_cast<int64_t>(r0) * B, bytes, &full[s], policy);
   };
   if (threadIdx.x == 0)
     for (int j = 0; j < nslots && j < nsl; ++j) issue(j);
   if (l2_prefetch && lane == 0) {
     // the part of the range beyond the ring, one slice per warp
     const int64_t share = static_cast<int64_t>(nrows) * B;
-    const int64_t ring_part = static_cast<int64_t>(nslots) * slot_bytes;
+    const int64_t ring_part = static_cast<int64_t>(nslots) * R * B;
     const int64_t from = ring_part < share ? ring_part : share;
     const int64_t slice = ((share - from) / NWARPS + 15) / 16 * 16;
     const int64_t lo = from + slice * warp;
@@ -129,6 +144,7 @@ __global__ void __launch_bounds__(NWARPS * 32, 1024 / (NWARPS * 32))
     for (int64_t o = lo; o < hi; o += 65536) {
       const int64_t n = hi - o < 65536 ? hi - o : 65536;
       bulk_prefetch_l2(wbase + o, static_cast<uint32_t>(n));
+      if constexpr (GATE) bulk_prefetch_l2(wbase2 + o, static_cast<uint32_t>(n));
     }
   }
 
@@ -215,11 +231,12 @@ __global__ void __launch_bounds__(NWARPS * 32, 1024 / (NWARPS * 32))
       break;
     }
     const uint32_t sbase = smem_addr(ring + s * slot_bytes);
-    // two rows at a time (r and r + RG): twice the independent loads and chains
-    for (int r = grp; r < nr; r += 2 * RG) {
-      const bool two = r + RG < nr;
+    // two rows at a time: r and r + RG, or (GATE) up row r and gate row r -- twice the
+    // independent loads and chains
+    for (int r = grp; r < nr; r += (GATE ? 1 : 2) * RG) {
+      const bool two = GATE || r + RG < nr;
       const uint32_t rb0 = sbase + r * B;
-      const uint32_t rb1 = two ? rb0 + RG * B : rb0;
+      const uint32_t rb1 = GATE ? rb0 + R * B : (two ? rb0 + RG * B : rb0);
       uint2 w0[NP], w1[NP];
 #pragma unroll
       for (int p = 0; p < NP; ++p) {
@@ -230,7 +247,8 @@ __global__ void __launch_bounds__(NWARPS * 32, 1024 / (NWARPS * 32))
       const int v1 = __reduce_add_sync(0xffffffffu, row_dot(w1));
       if (lane == 0) {
         part[seg * rows_max + r0 + r] = v0;
-        if (two) part[seg * rows_max + r0 + r + RG] = v1;
+        if constexpr (GATE) part[(S + seg) * rows_max + r0 + r] = v1;  // the gate rows' sums after the up rows'
+        else if (two) part[seg * rows_max + r0 + r + RG] = v1;
       }
     }
     __syncwarp();
@@ -256,16 +274,31 @@ __global__ void __launch_bounds__(NWARPS * 32, 1024 / (NWARPS * 32))
         if (issued[s] > 0) mbar_wait(&full[s], (issued[s] - 1u) & 1u);
     return;
   }
-  for (int i = threadIdx.x; i < nrows; i += NWARPS * 32) {
-    int a = -rsum;
-    for (int g = 0; g < S; ++g) a += part[g * rows_max + i];
-    const int64_t o = row_lo + i;
-    if (y_dtype == 2) {
-      static_cast<int32_t*>(y)[o] = a;
-    } else {
-      const float v = __fmul_rn(__fmul_rn(__int2float_rn(a), gamma), asc);
-      if (y_dtype == 0) static_cast<float*>(y)[o] = v;
-      else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
+  if constexpr (GATE) {
+    const float gamma2 = __ldg(gamma2_ptr);
+    for (int i = threadIdx.x; i < nrows; i += NWARPS * 32) {
+      int au = -rsum, ag = -rsum;
+      for (int g = 0; g < S; ++g) {
+        au += part[g * rows_max + i];
+        ag += part[(S + g) * rows_max + i];
+      }
+      const float u = __fmul_rn(__fmul_rn(__int2float_rn(au), gamma), asc);
+      const float g = __fmul_rn(__fmul_rn(__int2float_rn(ag), gamma2), asc);
+      const float r = g > 0.0f ? g : 0.0f;
+      static_cast<__nv_bfloat16*>(y)[row_lo + i] = __float2bfloat16_rn(__fmul_rn(__fmul_rn(r, r), u));
+    }
+  } else {
+    for (int i = threadIdx.x; i < nrows; i += NWARPS * 32) {
+      int a = -rsum;
+      for (int g = 0; g < S; ++g) a += part[g * rows_max + i];
+      const int64_t o = row_lo + i;
+      if (y_dtype == 2) {
+        static_cast<int32_t*>(y)[o] = a;
+      } else {
+        const float v = __fmul_rn(__fmul_rn(__int2float_rn(a), gamma), asc);
+        if (y_dtype == 0) static_cast<float*>(y)[o] = v;
+        else static_cast<__nv_bfloat16*>(y)[o] = __float2bfloat16_rn(v);
+      }
     }
   }
 }

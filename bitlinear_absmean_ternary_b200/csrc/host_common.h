@@ -8,6 +8,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
 #include <atomic>
@@ -136,6 +137,13 @@ inline bitnet_status check_linear(const uint8_t* Wp, const float* gamma, int64_t
 // Largest M * Kp (token rows x padded K) the base-3 decode kernel keeps in
 // shared memory; the base-3 pack refuses K beyond it.
 constexpr int kGemvB3XMaxBytes = 24000;
+
+// The decode FFN's up and gate products for one token with the squared-ReLU
+// gate in the epilogue (k_gemv.cu): *used = false, nothing launched, where
+// that kernel's plan does not apply.
+cudaError_t launch_ffn_upgate_gemv1(const __nv_bfloat16* x, const __nv_bfloat16* gain, float eps, const uint8_t* Wu,
+                                    const float* gu, const uint8_t* Wg, const float* gg, int F, int D,
+                                    __nv_bfloat16* h, cudaStream_t s, bool* used);
 
 // Device error words, one per translation unit that launches kernels with
 // bounded waits: each reads its word into *v and clears it when set.

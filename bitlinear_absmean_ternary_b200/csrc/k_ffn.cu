@@ -90,6 +90,20 @@ bitnet_status bitnet_bitlinear_ffn_gemv(const void* x, int x_dtype, int64_t M, i
   if (!valid_k(D) || !valid_k(F) || D > kFfnMaxK || F > kFfnMaxK || M < 1 || M > 8)
     return BITNET_ERR_UNSUPPORTED_SHAPE;
   const int m = static_cast<int>(M), d = static_cast<int>(D), f = static_cast<int>(F);
+  if (m == 1) {
+    // one token with large weight shares: the gated one-token GEMV (x -> h), then the fused
+    // one-token GEMV on h (h -> y) -- two launches whose weights stream in whole-row slots, which on
+    // the 27B FFN beat the one-launch kernel below (its per-warp rings issue many small copies)
+    bool used = false;
+    const cudaError_t e = launch_ffn_upgate_gemv1(static_cast<const __nv_bfloat16*>(x),
+                                                  static_cast<const __nv_bfloat16*>(rms_gain_in), rms_eps_in, W_up,
+                                                  gamma_up, W_gate, gamma_gate, f, d, static_cast<__nv_bfloat16*>(h),
+                                                  static_cast<cudaStream_t>(stream), &used);
+    if (e != cudaSuccess) return from_cuda(e);
+    if (used)
+      return bitnet_bitlinear_gemv(h, BITNET_BF16, rms_gain_sub, rms_eps_sub, W_down, gamma_down, D, F, 1, y, y_dtype,
+                                   stream);
+  }
   const int G = sm_count();
   const int slots = ffn_slots(m, d, f, G);
   if (slots == 0) return BITNET_ERR_UNSUPPORTED_SHAPE;

@@ -85,7 +85,7 @@ struct Gemv1Plan {
 
 int gemv1_segw(int Bw, int S) { return ((Bw + S - 1) / S + 1) & ~1; }
 
-bool gemv1_plan(int N, int K, bool xs, Gemv1Plan& p) {
+bool gemv1_plan(int N, int K, bool xs, Gemv1Plan& p, bool gate = false) {
   const int B = K / 4, Bw = B / 4;
   p.warps = BITNET_GEMV1_WARPS;
   const int smem_max = p.warps == 16 ? kGemv1SmemMax : kGemv1SmemMax1;
@@ -100,36 +100,38 @@ bool gemv1_plan(int N, int K, bool xs, Gemv1Plan& p) {
   // 16 warps each start on their own first item at once, serves it better
   if (static_cast<int64_t>(p.rows_max) * B <= BITNET_GEMV_SMALL_SHARE) return false;
   const int RG = p.warps / p.S;
-  const int per = BITNET_GEMV1_SLOT_TARGET / (RG * B);
+  const int mats = gate ? 2 : 1;  // GATE: a slot holds the rows of both matrices
+  const int per = BITNET_GEMV1_SLOT_TARGET / (mats * RG * B);
   p.R = RG * (per > 1 ? per : 1);
   if (p.R > p.rows_max) p.R = p.rows_max;
-  const int slot_bytes = p.R * B;
+  const int slot_bytes = mats * p.R * B;
   const int slots_per_cta = (p.rows_max + p.R - 1) / p.R;
   p.nslots = (p.warps == 16 ? BITNET_GEMV1_RING_TARGET : BITNET_GEMV1_RING_TARGET1) / slot_bytes;
   if (p.nslots < 2) p.nslots = 2;
   if (p.nslots > kGemv1MaxSlots) p.nslots = kGemv1MaxSlots;
   if (p.nslots > slots_per_cta) p.nslots = slots_per_cta;
-  while (p.nslots > 1 && gemv1_smem_bytes(K, xs, slot_bytes, p.nslots, p.rows_max, p.S) > smem_max) --p.nslots;
-  p.smem = gemv1_smem_bytes(K, xs, slot_bytes, p.nslots, p.rows_max, p.S);
+  while (p.nslots > 1 && gemv1_smem_bytes(K, xs, slot_bytes, p.nslots, p.rows_max, p.S, gate) > smem_max) --p.nslots;
+  p.smem = gemv1_smem_bytes(K, xs, slot_bytes, p.nslots, p.rows_max, p.S, gate);
   if (p.smem > smem_max) return false;
 #ifndef BITNET_GEMV1_L2_PREFETCH
 #define BITNET_GEMV1_L2_PREFETCH 1
 #endif
   p.l2_prefetch = BITNET_GEMV1_L2_PREFETCH &&
-                  static_cast<int64_t>(p.rows_max) * B > static_cast<int64_t>(p.nslots) * slot_bytes;
+                  static_cast<int64_t>(p.rows_max) * B > static_cast<int64_t>(p.nslots) * p.R * B;
   return true;
 }
 
-template <bool U8, int NP, int NWARPS, bool FUSED, typename T, int MAXC>
+template <bool U8, int NP, int NWARPS, bool FUSED, typename T, int MAXC, bool GATE = false>
 cudaError_t launch_gemv1_w(const Gemv1Plan& p, const uint8_t* Wp, const float* gamma, int N, int K,
                             const int8_t* xq, const float* a, const int32_t* rs, const T* x, const T* gain,
-                            float eps, void* y, int yd, cudaStream_t s) {
+                            float eps, void* y, int yd, cudaStream_t s, const uint8_t* Wp2 = nullptr,
+                            const float* gamma2 = nullptr) {
   static std::atomic<bool> done[kMaxDevices] = {};
-  auto kern = gemv1_kernel<U8, NP, NWARPS, FUSED, T, MAXC>;
+  auto kern = gemv1_kernel<U8, NP, NWARPS, FUSED, T, MAXC, GATE>;
   const cudaError_t e = set_smem(kern, NWARPS == 16 ? kGemv1SmemMax : kGemv1SmemMax1, done);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(p.grid), dim3(NWARPS * 32), p.smem, s, Wp, gamma, N, K, xq, a, rs, x, gain, eps, y,
-                    yd, p.S, p.R, p.nslots, p.rows_max, p.l2_prefetch);
+  return launch_pdl(kern, dim3(p.grid), dim3(NWARPS * 32), p.smem, s, Wp, gamma, Wp2, gamma2, N, K, xq, a, rs, x,
+                    gain, eps, y, yd, p.S, p.R, p.nslots, p.rows_max, p.l2_prefetch);
 }
 
 template <bool U8, int NP, bool FUSED, typename T, int MAXC>
@@ -253,7 +255,49 @@ cudaError_t launch_fused(int M, const void* x, const void* gain, float eps, cons
   }
 }
 
+template <int NP, int MAXC>
+cudaError_t launch_upgate1_np(const Gemv1Plan& p, const __nv_bfloat16* x, const __nv_bfloat16* gain, float eps,
+                              const uint8_t* Wu, const float* gu, const uint8_t* Wg, const float* gg, int F, int D,
+                              __nv_bfloat16* h, cudaStream_t s) {
+  return launch_gemv1_w<true, NP, BITNET_GEMV1_WARPS, true, __nv_bfloat16, MAXC, true>(
+      p, Wu, gu, F, D, static_cast<const int8_t*>(nullptr), static_cast<const float*>(nullptr),
+      static_cast<const int32_t*>(nullptr), x, gain, eps, h, BITNET_BF16, s, Wg, gg);
+}
+
+template <int MAXC>
+cudaError_t launch_upgate1_c(const Gemv1Plan& p, const __nv_bfloat16* x, const __nv_bfloat16* gain, float eps,
+                             const uint8_t* Wu, const float* gu, const uint8_t* Wg, const float* gg, int F, int D,
+                             __nv_bfloat16* h, cudaStream_t s) {
+  switch (p.NP) {
+    case 1: return launch_upgate1_np<1, MAXC>(p, x, gain, eps, Wu, gu, Wg, gg, F, D, h, s);
+    case 2: return launch_upgate1_np<2, MAXC>(p, x, gain, eps, Wu, gu, Wg, gg, F, D, h, s);
+    case 3: return launch_upgate1_np<3, MAXC>(p, x, gain, eps, Wu, gu, Wg, gg, F, D, h, s);
+    default: return launch_upgate1_np<4, MAXC>(p, x, gain, eps, Wu, gu, Wg, gg, F, D, h, s);
+  }
+}
+
 }  // namespace
+
+// The decode FFN's up and gate projections for one token with the gating
+// in the epilogue (gemv1_kernel<..., GATE>): x (D bf16, optional RMSNorm
+// gain) -> h (F bf16).  *used = false (nothing launched) where the
+// one-token whole-row-slot plan does not apply.
+cudaError_t bitnet_host::launch_ffn_upgate_gemv1(const __nv_bfloat16* x, const __nv_bfloat16* gain, float eps,
+                                                 const uint8_t* Wu, const float* gu, const uint8_t* Wg,
+                                                 const float* gg, int F, int D, __nv_bfloat16* h, cudaStream_t s,
+                                                 bool* used) {
+  Gemv1Plan p;
+  *used = false;
+  if (D > kGemvXMaxBytes || !gemv1_plan(F, D, true, p, true)) return cudaSuccess;
+  const int nthr = gain != nullptr ? kQuantThreads : kGemvThreads;
+  const int per_thread = (D / 8 + nthr - 1) / nthr;
+  *used = true;
+  if (per_thread <= 1) return launch_upgate1_c<1>(p, x, gain, eps, Wu, gu, Wg, gg, F, D, h, s);
+  if (per_thread <= 2) return launch_upgate1_c<2>(p, x, gain, eps, Wu, gu, Wg, gg, F, D, h, s);
+  if (per_thread <= 4) return launch_upgate1_c<4>(p, x, gain, eps, Wu, gu, Wg, gg, F, D, h, s);
+  if (per_thread <= 8) return launch_upgate1_c<8>(p, x, gain, eps, Wu, gu, Wg, gg, F, D, h, s);
+  return launch_upgate1_c<16>(p, x, gain, eps, Wu, gu, Wg, gg, F, D, h, s);
+}
 
 BITNET_DEFINE_TAKE_ERROR(gemv)
 

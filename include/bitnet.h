@@ -455,7 +455,11 @@ bitnet_status bitnet_ste_backward_weight(const void* dY, const int8_t* x_q, cons
  * The kernel is a cooperative launch of one CTA per SM (its CTAs wait for
  * one another once, between the gating and the down projection; that wait is
  * bounded and reports BITNET_ERR_TIMEOUT through bitnet_get_device_status).
- * Asynchronous.
+ * For ONE token with large weight shares per SM (F rows x D/4 bytes above
+ * 64 KB per SM, as in the 27B-class FFN) the block instead runs as two
+ * launches of the one-token decode product: up and gate with the gating in
+ * the epilogue (x -> h), then bitnet_bitlinear_gemv on h (h -> y); the results
+ * are the same and `sync` is not touched.  Asynchronous.
  */
 bitnet_status bitnet_bitlinear_ffn_gemv(const void* x, int x_dtype, int64_t M, int64_t D, int64_t F,
                                         const void* rms_gain_in, float rms_eps_in, const uint8_t* W_up,

@@ -63,8 +63,10 @@ FFN_CASES = [
     (8, 64, 128, True, True, "bf16"),       # most CTAs own 0 or 1 feature
     (3, 1024, 4096, True, True, "f32"),
     (5, 2560, 6912, True, True, "bf16"),
-    (1, 5376, 21504, True, True, "bf16"),   # 27B-class FFN: weights stream through the ring
-    (2, 5376, 21504, True, True, "i32"),
+    (1, 5376, 21504, True, True, "bf16"),   # 27B-class FFN, one token: the gated one-token GEMV, then the down GEMV
+    (1, 5376, 21504, False, True, "f32"),   # the same without the input norm
+    (1, 3072, 12288, True, False, "i32"),   # gated one-token GEMV: 84 features per CTA, a ragged last slot
+    (2, 5376, 21504, True, True, "i32"),    # 27B-class FFN, two tokens: the one-launch kernel's rings
 ]
 
 
