@@ -71,6 +71,12 @@ cudaError_t launch_quant(const void* x, int64_t M, int K, const void* gain, floa
     if constexpr (sizeof(T) == 2) return launch_quant_t<T, 16>(x, M, K, gain, eps, xq, a, rs, s, threads);
     return cudaErrorInvalidValue;
   }
+  // With the norm, rows past the register budget are read in three passes
+  // (quant_row_norm_stream); when every row has its own SM, 1024 threads per
+  // row take the two order-free passes in one batch each.
+  constexpr int kResidentChunks = BN_QUANT_STREAM_BYTES / static_cast<int>(sizeof(Chunk8<T>));
+  if (per_thread > kResidentChunks && M <= sm_count())
+    return launch_quant_t<T, kResidentChunks + 1, 1024>(x, M, K, gain, eps, xq, a, rs, s, 1024);
   if (per_thread <= 1) return launch_quant_t<T, 1>(x, M, K, gain, eps, xq, a, rs, s);
   if (per_thread <= 2) return launch_quant_t<T, 2>(x, M, K, gain, eps, xq, a, rs, s);
   if (per_thread <= 4) return launch_quant_t<T, 4>(x, M, K, gain, eps, xq, a, rs, s);

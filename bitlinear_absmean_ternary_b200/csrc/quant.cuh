@@ -3,7 +3,8 @@
 // 8-bit activations; RMSNorm; the input is normalised, then quantised).
 //
 // 256 threads per token row; thread t owns the 8-element chunks c = t,
-// t+256, ... and keeps them in registers, so x is read from HBM once.
+// t+256, ... and keeps them in registers, so x is read from HBM once (a long
+// row with RMSNorm is read in three passes, the later ones from L1 or L2).
 // The sum of squares uses the fixed order of the oracle: each thread adds
 // RN32(v*v) over its chunks in increasing k, then the halving tree
 // l += l+128, +64, +32 (shared memory), +16 .. +1 (shuffles).
@@ -97,10 +98,152 @@ BN_DEV void sync_threads() {
   else asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory");
 }
 
+// The RMSNorm path of quant_row_cta for rows too long to keep in registers:
+// three passes over the row, each reading it again (from L1 or L2), with a
+// bounded number of chunks in registers at a time.  Pass 1 is the sum of
+// squares in the fixed order (thread t < 256 adds its chunks t, t+256, ...
+// in increasing order, then the same tree); passes 2 (max|h|) and 3 (x_q)
+// are order-free and use every thread.  The first batch of a pass is
+// requested before the barrier that ends the previous one, so each barrier
+// overlaps one memory round trip.  Same arguments, results and barrier
+// discipline as quant_row_cta.  Not inlined: compiled into the caller next to
+// the register-resident path, it made the register allocator spill the
+// callers' own loops; as a call it costs a few registers' save and restore
+// once per row.
+template <typename T, bool COHERENT, int NT, int T0>
+__device__ __noinline__ void quant_row_norm_stream(const T* __restrict__ row, int K, const T* __restrict__ gain, float rms_eps,
+                                  int8_t* xq_row, QuantScratch& sc, float& amax_out, int& sum_out) {
+  const int t = static_cast<int>(threadIdx.x) - T0;
+  const int lane = t & 31, warp = t >> 5;
+  const int nthreads = NT == 0 ? static_cast<int>(blockDim.x) : NT;
+  const int nwarps = nthreads >> 5;
+  const int nchunks = K >> 3;
+  // Chunks in flight per thread: 128 bytes of x in pass 1, 64 bytes each of
+  // x and the gain in passes 2 and 3 (more spills under a 64-register budget).
+  constexpr int NB1 = 128 / static_cast<int>(sizeof(Chunk8<T>));
+  constexpr int NB2 = 64 / static_cast<int>(sizeof(Chunk8<T>));
+  auto load_x = [&](Chunk8<T>& d, int c) {
+    if constexpr (COHERENT) d.load_cg(row + 8 * c);
+    else d.load(row + 8 * c);
+  };
+
+  float ss = 0.0f;
+  if (t < kQuantThreads) {
+#pragma unroll 1
+    for (int c0 = t; c0 < nchunks; c0 += NB1 * kQuantThreads) {
+      Chunk8<T> b[NB1];
+#pragma unroll
+      for (int j = 0; j < NB1; ++j)
+        if (c0 + j * kQuantThreads < nchunks) load_x(b[j], c0 + j * kQuantThreads);
+#pragma unroll
+      for (int j = 0; j < NB1; ++j) {
+        if (c0 + j * kQuantThreads < nchunks) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float v = b[j].get(e);
+            ss = __fadd_rn(ss, __fmul_rn(v, v));
+          }
+        }
+      }
+    }
+    sc.red[t] = ss;
+  }
+
+  // Batches of passes 2 and 3: thread t takes chunks t + nthreads * i.
+  Chunk8<T> xb[NB2], gb[NB2];
+  const int step = NB2 * nthreads;
+  auto load_batch = [&](int c0) {
+#pragma unroll
+    for (int j = 0; j < NB2; ++j) {
+      const int c = c0 + j * nthreads;
+      if (c < nchunks) {
+        load_x(xb[j], c);
+        gb[j].load(gain + 8 * c);
+      }
+    }
+  };
+  load_batch(t);
+  sync_threads<NT>();
+  const float* R = sc.red;
+  float p = __fadd_rn(__fadd_rn(__fadd_rn(R[lane], R[lane + 128]), __fadd_rn(R[lane + 64], R[lane + 192])),
+                      __fadd_rn(__fadd_rn(R[lane + 32], R[lane + 160]), __fadd_rn(R[lane + 96], R[lane + 224])));
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+    const float o = __shfl_down_sync(0xffffffffu, p, s);
+    if (lane < s) p = __fadd_rn(p, o);
+  }
+  p = __shfl_sync(0xffffffffu, p, 0);
+  const float ms = __fdiv_rn(p, static_cast<float>(K));
+  const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, rms_eps)));
+
+  float amax = 0.0f;
+#pragma unroll 1
+  for (int c0 = t; c0 < nchunks; c0 += step) {
+    if (c0 != t) load_batch(c0);
+#pragma unroll
+    for (int j = 0; j < NB2; ++j) {
+      if (c0 + j * nthreads < nchunks) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(__fmul_rn(__fmul_rn(xb[j].get(e), r), gb[j].get(e))));
+      }
+    }
+  }
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, s));
+  if (lane == 0) sc.amx[warp] = amax;
+  load_batch(t);
+  sync_threads<NT>();
+  amax = lane < nwarps ? sc.amx[lane] : 0.0f;
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, s));
+
+  int sum = 0;
+  const float s = amax == 0.0f ? 0.0f : __fdiv_rn(127.0f, amax);
+#pragma unroll 1
+  for (int c0 = t; c0 < nchunks; c0 += step) {
+    if (c0 != t) load_batch(c0);
+#pragma unroll
+    for (int j = 0; j < NB2; ++j) {
+      const int c = c0 + j * nthreads;
+      if (c < nchunks) {
+        uint32_t lo = 0, hi = 0;
+        if (amax != 0.0f) {
+          uint32_t q[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            q[e] = f32_to_s8_rne_bits(__fmul_rn(__fmul_rn(__fmul_rn(xb[j].get(e), r), gb[j].get(e)), s));
+          lo = pack4_s8(q[0], q[1], q[2], q[3]);
+          hi = pack4_s8(q[4], q[5], q[6], q[7]);
+          sum = __dp4a(static_cast<int>(lo), 0x01010101, sum);
+          sum = __dp4a(static_cast<int>(hi), 0x01010101, sum);
+        }
+        *reinterpret_cast<uint2*>(xq_row + 8 * c) = make_uint2(lo, hi);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) sc.ired[warp] = sum;
+  sync_threads<NT>();
+  int tot = lane < nwarps ? sc.ired[lane] : 0;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+  amax_out = amax;
+  sum_out = tot;
+}
+
+// Resident footprint (bytes of x per thread) above which the RMSNorm path
+// streams the row instead of keeping it in registers.
+#ifndef BN_QUANT_STREAM_BYTES
+#define BN_QUANT_STREAM_BYTES 64
+#endif
+
 // Quantises one token row with the threads of the CTA.  Every thread must
 // call it (it holds CTA-wide barriers).  Thread t owns the 8-element chunks
 // c = t, t+nt, ... (nt = all threads without RMSNorm, the first 256 with it)
-// and keeps them in registers, so the row is read once.  Writes x_q through
+// and keeps them in registers, so the row is read once (with RMSNorm and
+// more than BN_QUANT_STREAM_BYTES of x per thread, quant_row_norm_stream
+// reads it in three passes instead).  Writes x_q through
 // xq_row (global or shared memory; complete and visible to the whole CTA on
 // return); returns max|h| and sum(x_q) to every thread.  COHERENT reads the
 // row through L2 only, for a row that other CTAs of the same kernel wrote.
@@ -120,6 +263,12 @@ template <typename T, int MAXC, bool COHERENT = false, int NT = 0, int T0 = 0>
 BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict__ gain, float rms_eps,
                           int8_t* xq_row, QuantScratch& sc, float& amax_out, int& sum_out) {
   static_assert(T0 % 32 == 0 && (T0 == 0 || NT != 0), "a thread offset needs a fixed thread count");
+  if constexpr (sizeof(Chunk8<T>) * MAXC > BN_QUANT_STREAM_BYTES) {
+    if (gain != nullptr) {
+      quant_row_norm_stream<T, COHERENT, NT, T0>(row, K, gain, rms_eps, xq_row, sc, amax_out, sum_out);
+      return;
+    }
+  }
   const int t = static_cast<int>(threadIdx.x) - T0;
   const int lane = t & 31, warp = t >> 5;
   const int nthreads = NT == 0 ? static_cast<int>(blockDim.x) : NT;

@@ -52,6 +52,7 @@ B3_CASES = [
     (3, 129, 64, "f32", True, "bf16"),        # K < 80: one padded group
     (2, 1000, 4096, "bf16", False, "bf16"),
     (3, 77, 6912, "bf16", True, "f32"),      # 3 x 6960 padded bytes of x_q
+    (1, 3000, 16384, "bf16", True, "bf16"),  # the norm's row read in three passes
 ]
 
 

@@ -140,6 +140,11 @@ QUANT_CASES = [
     (4096, 6912, "student_t4", 0.0, 1.0, "bf16", False),  # the prefill down projection's input
     (511, 2560, "normal", 0.0, 1.0, "bf16", True),       # one row below the warp kernel's threshold
     (1024, 1344, "normal", 0.0, 1.0, "f32", True),       # fp32 input: a CTA per row at any M
+    # rows past the norm path's register budget, read in three passes
+    (3, 8192, "normal", 0.01, 20.0, "f32", True),        # a row per SM: 1024 threads per row
+    (200, 12288, "normal", 0.01, 20.0, "f32", True),     # more rows than SMs: 256 threads per row
+    (300, 12288, "normal", 0.005, 30.0, "bf16", True),   # bf16, 6 chunks per lane
+    (1, 21504, "normal", 0.005, 30.0, "bf16", True),     # one token, the 27B FFN's sub-norm input
 ]
 
 
@@ -307,6 +312,8 @@ FUSED_CASES = [
     (2, 5376, 10752, "bf16", True, "f32"),     # deep-ring plan with two tokens
     (1, 21501, 5376, "bf16", True, "i32"),     # ragged last group of the last CTA
     (1, 9000, 12288, "f32", True, "bf16"),     # one token, whole-row slots, f32 input with the norm
+    (1, 6144, 16384, "bf16", True, "bf16"),    # one token, the norm's row read in three passes
+    (2, 700, 10752, "f32", True, "bf16"),      # item GEMV, two f32 tokens, the same
 ]
 
 
@@ -575,6 +582,7 @@ FQ_CASES = [
     (33, 777, 1344, "f32", False, "bf16"),
     (1, 128, 64, "bf16", True, "f32"),           # one unit: a grid of one CTA quantises every row
     (9, 129, 8192, "f32", True, "i32"),
+    (16, 2048, 21504, "bf16", True, "f32"),      # the norm's rows read in three passes inside the product
 ]
 
 
