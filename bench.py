@@ -492,6 +492,12 @@ class Workload:
             self.bl.bitnet_bitlinear_gemm(self.x(i, c), self.packs[i][0][c % self.copies], self.packs[i][1],
                                           self.gains[i], EPS_RMS, y=self.buf(i, c)["y"], workspace=self.ws)
 
+    def fused_linear_host(self, i, c, x_host, y_host):
+        """The one-token/few-token decode linear with host buffers: pinned x in,
+        fused kernel, pinned y out, in one C call (bitnet_bitlinear_gemv_host)."""
+        self.bl.bitnet_bitlinear_gemv_host(x_host, self.x(i, c), self.packs[i][0][c % self.copies], self.packs[i][1],
+                                           self.buf(i, c)["y"], y_host, self.gains[i], EPS_RMS)
+
     def linear(self, i, c):
         if self.fused:
             self.fused_linear(i, c)
@@ -741,6 +747,9 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
     ys_host = [torch.empty_like(wl.buf(i, 0)["y"], device="cpu").pin_memory() for i in range(len(lins))]
     k_e2e = min(max(K, 200), 2000)
 
+    # the decode workloads' public call takes host buffers itself (one C call per linear)
+    host_call = wl.path == "gemv_fused"
+
     def e2e_loop(n, copies=True, calls=True):
         with torch.cuda.stream(stream):
             torch.cuda.synchronize(dev)
@@ -750,6 +759,9 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
             a.record(stream)
             for c in range(n):
                 for i in range(len(lins)):
+                    if copies and calls and host_call:
+                        wl.fused_linear_host(i, c, xs_host[i], ys_host[i])
+                        continue
                     if copies:
                         wl.x(i, c).copy_(xs_host[i], non_blocking=True)
                     if calls:
@@ -772,9 +784,12 @@ def run_ours(args, lins, ws: int, rank: int, local: int):
            "breakdown_us_per_step": {"copies_only": copies_ms * 1e3 / nb, "api_calls_only": calls_ms * 1e3 / nb,
                                      "api_calls_host_wall": calls_host_ms * 1e3 / nb,
                                      "kernels_back_to_back": head["ms_per_step"] * 1e3},
-           "how": "eager Python calls of the public API per step: pinned H2D copy of every input, the BitLinear "
-                  "call(s), D2H copy of every output; the breakdown repeats the loop with the copies alone and the "
-                  "calls alone"}
+           "how": ("eager Python calls of the public API per step: for each linear one bitnet_bitlinear_gemv_host "
+                   "call (pinned H2D copy of the input, the fused kernel, D2H copy of the output, issued from C)"
+                   if host_call else
+                   "eager Python calls of the public API per step: pinned H2D copy of every input (torch), the "
+                   "BitLinear call(s), D2H copy of every output (torch)") +
+                  "; the breakdown repeats the loop with torch copies alone and the device-buffer calls alone"}
     del xs_host, ys_host
 
     # ------------------------------------------------------------------ every configuration

@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
         L.bitnet_linear_upgate_gemm.restype = I
         L.bitnet_bitlinear_gemv.argtypes = [P, I, P, F, P, P, I64, I64, I64, P, I, P]
         L.bitnet_bitlinear_gemv.restype = I
+        L.bitnet_bitlinear_gemv_host.argtypes = [P, P, I, P, F, P, P, I64, I64, I64, P, P, I, P]
+        L.bitnet_bitlinear_gemv_host.restype = I
         L.bitnet_bitlinear_ffn_gemv.argtypes = [P, I, I64, I64, I64, P, F, P, P, P, P, P, F, P, P, P, P, I, P, P]
         L.bitnet_bitlinear_ffn_gemv.restype = I
         L.bitnet_pack_weights_noalloc.argtypes = [P, I64, I64, F, P, P, P]
@@ -343,6 +345,28 @@ def bitnet_bitlinear_gemv(x, W_packed, gamma, rms_gain=None, rms_eps: float = 1e
                                      _ptr(gamma), N, K, M, _ptr(y), _dtype_code(y.dtype), _stream(x.device))
     _check("bitnet_bitlinear_gemv", st)
     return y
+
+
+def bitnet_bitlinear_gemv_host(x_host, x, W_packed, gamma, y, y_host, rms_gain=None, rms_eps: float = 1e-5):
+    """bitnet_bitlinear_gemv with the tokens and the result in host memory:
+    copies x_host (M x K, pinned CPU tensor) into the device tensor x, runs the
+    fused kernel into y and copies y back into y_host (pinned CPU tensor), all
+    on the current stream.  Synchronise the stream before reading y_host."""
+    _need_cuda(x, rms_gain, W_packed, gamma, y)
+    for t in (x_host, y_host):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("x_host and y_host must be contiguous host tensors")
+    if x_host.shape != x.shape or x_host.dtype != x.dtype or y_host.shape != y.shape or y_host.dtype != y.dtype:
+        raise ValueError("host and device buffers disagree in shape or dtype")
+    M, K = x.shape
+    N = W_packed.shape[0]
+    if W_packed.shape[1] * 4 != K or tuple(y.shape) != (M, N):
+        raise ValueError("x, W_packed and y disagree on the shape")
+    st = lib().bitnet_bitlinear_gemv_host(_ptr(x_host), _ptr(x), _dtype_code(x.dtype), _ptr(rms_gain), rms_eps,
+                                          _ptr(W_packed), _ptr(gamma), N, K, M, _ptr(y), _ptr(y_host),
+                                          _dtype_code(y.dtype), _stream(x.device))
+    _check("bitnet_bitlinear_gemv_host", st)
+    return y_host
 
 
 def bitnet_bitlinear_gemm_workspace_bytes(M: int, N: int, K: int) -> int:

@@ -317,9 +317,13 @@ bitnet_status bitnet_linear_gemv(const uint8_t* W_packed, const float* gamma, in
   return from_cuda(e);
 }
 
-bitnet_status bitnet_bitlinear_gemv(const void* x, int x_dtype, const void* rms_gain, float rms_eps,
-                                    const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, int64_t M,
-                                    void* y, int y_dtype, void* stream) {
+}  // extern "C"
+
+namespace {
+
+bitnet_status check_bitlinear_gemv(const void* x, int x_dtype, const void* rms_gain, float rms_eps,
+                                   const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, int64_t M,
+                                   const void* y, int y_dtype) {
   if (x == nullptr || W_packed == nullptr || gamma == nullptr || y == nullptr) return BITNET_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(rms_gain, 16) || !aligned(W_packed, 16) || !aligned(y, 16) || !aligned(gamma, 4))
     return BITNET_ERR_INVALID_ARG;
@@ -329,12 +333,44 @@ bitnet_status bitnet_bitlinear_gemv(const void* x, int x_dtype, const void* rms_
   const int64_t kmax = x_dtype == BITNET_BF16 ? 32768 : 16384;
   if (!valid_k(K) || K > kmax || N < 1 || N > INT32_MAX || M < 1 || M > 8 || M * K > kGemvXMaxBytes)
     return BITNET_ERR_UNSUPPORTED_SHAPE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return BITNET_OK;
+}
+
+cudaError_t launch_bitlinear_gemv(const void* x, int x_dtype, const void* rms_gain, float rms_eps,
+                                  const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, int64_t M,
+                                  void* y, int y_dtype, cudaStream_t s) {
   const int n = static_cast<int>(N), k = static_cast<int>(K), m = static_cast<int>(M);
-  const cudaError_t e =
-      x_dtype == BITNET_BF16
-          ? launch_fused<__nv_bfloat16>(m, x, rms_gain, rms_eps, W_packed, gamma, n, k, y, y_dtype, s)
-          : launch_fused<float>(m, x, rms_gain, rms_eps, W_packed, gamma, n, k, y, y_dtype, s);
+  return x_dtype == BITNET_BF16
+             ? launch_fused<__nv_bfloat16>(m, x, rms_gain, rms_eps, W_packed, gamma, n, k, y, y_dtype, s)
+             : launch_fused<float>(m, x, rms_gain, rms_eps, W_packed, gamma, n, k, y, y_dtype, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+bitnet_status bitnet_bitlinear_gemv(const void* x, int x_dtype, const void* rms_gain, float rms_eps,
+                                    const uint8_t* W_packed, const float* gamma, int64_t N, int64_t K, int64_t M,
+                                    void* y, int y_dtype, void* stream) {
+  const bitnet_status st = check_bitlinear_gemv(x, x_dtype, rms_gain, rms_eps, W_packed, gamma, N, K, M, y, y_dtype);
+  if (st != BITNET_OK) return st;
+  return from_cuda(launch_bitlinear_gemv(x, x_dtype, rms_gain, rms_eps, W_packed, gamma, N, K, M, y, y_dtype,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+bitnet_status bitnet_bitlinear_gemv_host(const void* x_host, void* x, int x_dtype, const void* rms_gain,
+                                         float rms_eps, const uint8_t* W_packed, const float* gamma, int64_t N,
+                                         int64_t K, int64_t M, void* y, void* y_host, int y_dtype, void* stream) {
+  if (x_host == nullptr || y_host == nullptr) return BITNET_ERR_INVALID_ARG;
+  const bitnet_status st = check_bitlinear_gemv(x, x_dtype, rms_gain, rms_eps, W_packed, gamma, N, K, M, y, y_dtype);
+  if (st != BITNET_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t xb = static_cast<size_t>(M * K) * (x_dtype == BITNET_BF16 ? 2 : 4);
+  const size_t yb = static_cast<size_t>(M * N) * (y_dtype == BITNET_BF16 ? 2 : 4);
+  cudaError_t e = cudaMemcpyAsync(x, x_host, xb, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = launch_bitlinear_gemv(x, x_dtype, rms_gain, rms_eps, W_packed, gamma, N, K, M, y, y_dtype, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(y_host, y, yb, cudaMemcpyDeviceToHost, s);
   return from_cuda(e);
 }
 

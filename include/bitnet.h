@@ -349,6 +349,28 @@ bitnet_status bitnet_bitlinear_gemv(const void* x, int x_dtype, const void* rms_
                                     void* y, int y_dtype, void* stream);
 
 /*
+ * bitnet_bitlinear_gemv with the token rows and the output in host memory:
+ * on `stream`, one cudaMemcpyAsync of x_host (M x K, x_dtype) into x, the
+ * fused kernel, and one cudaMemcpyAsync of y (M x N, y_dtype) into y_host.
+ * The decode step of a caller whose tokens live on the host, in one call.
+ *
+ * x_host  [in]  M x K host values; page-locked (cudaHostAlloc /
+ *               cudaHostRegister) for the copy to be asynchronous, else the
+ *               copy is synchronous with respect to the host.
+ * x       [out] device staging buffer of M x K values (16-byte aligned); the
+ *               kernel reads it after the copy.
+ * y       [out] device M x N outputs; y_host [out] host copy of them, valid
+ *               once `stream` has reached the end of the call.
+ * Other arguments and errors as bitnet_bitlinear_gemv; NULL x_host or y_host
+ * returns BITNET_ERR_INVALID_ARG.  Nothing is copied when an argument is
+ * rejected.  Asynchronous: the caller synchronises `stream` before reading
+ * y_host and must keep both host buffers alive until then.
+ */
+bitnet_status bitnet_bitlinear_gemv_host(const void* x_host, void* x, int x_dtype, const void* rms_gain,
+                                         float rms_eps, const uint8_t* W_packed, const float* gamma, int64_t N,
+                                         int64_t K, int64_t M, void* y, void* y_host, int y_dtype, void* stream);
+
+/*
  * Base-3 storage of the ternary codes, 1.6 bits per weight (a ternary weight
  * holds log2(3) ~ 1.58 bits: inferownia.pl, "BitNet b1.58: era 1-bitowych
  * LLM-ów", section "Skąd te 1,58 bita"; Habr repost on juhe.plus, section

@@ -187,6 +187,21 @@ def test_fused_rejects_bad_arguments(L):
     assert call(N=0) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
 
 
+def test_fused_host_rejects_bad_arguments_before_any_copy(L):
+    def call(xh=FAKE, x=FAKE, dt=bl.BITNET_BF16, g=None, eps=1e-5, W=FAKE, gam=FAKE, N=8, K=64, M=1, y=FAKE,
+             yh=FAKE, yd=bl.BITNET_BF16):
+        return L.bitnet_bitlinear_gemv_host(xh, x, dt, g, eps, W, gam, N, K, M, y, yh, yd, None)
+
+    assert call(xh=None) == bl.BITNET_ERR_INVALID_ARG
+    assert call(yh=None) == bl.BITNET_ERR_INVALID_ARG
+    assert call(x=None) == bl.BITNET_ERR_INVALID_ARG
+    assert call(x=MIS) == bl.BITNET_ERR_INVALID_ARG
+    assert call(yd=9) == bl.BITNET_ERR_INVALID_ARG
+    assert call(g=FAKE, eps=float("nan")) == bl.BITNET_ERR_INVALID_ARG
+    assert call(M=9) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+    assert call(M=2, K=21504) == bl.BITNET_ERR_UNSUPPORTED_SHAPE
+
+
 def test_ffn_rejects_bad_arguments(L):
     def call(x=FAKE, dt=bl.BITNET_BF16, M=1, D=64, F=128, gi=None, ei=1e-5, Wu=FAKE, gu=FAKE, Wg=FAKE, gg=FAKE,
              gs=None, es=1e-5, Wd=FAKE, gd=FAKE, h=FAKE, y=FAKE, yd=bl.BITNET_BF16, sync=FAKE):

@@ -344,6 +344,43 @@ def test_fused_bitlinear_gemv_parity(dev, orc, M, N, K, dt, norm, yt):
     assert torch.equal(y, bl.bitnet_linear_gemv(P, G, xq, a, rs, out_dtype=out))
 
 
+@pytest.mark.parametrize("M,N,K,dt,norm,yt", [(1, 21504, 5376, "bf16", False, "bf16"),
+                                                (2, 1000, 4096, "f32", True, "f32"),
+                                                (1, 300, 2688, "bf16", True, "i32")])
+def test_fused_bitlinear_gemv_host_buffers(dev, orc, M, N, K, dt, norm, yt):
+    """The host-buffer form: pinned x in, pinned y out, on a side stream,
+    several calls in flight before one synchronisation; every y_host equals
+    the device path's output and the oracle's."""
+    import torch
+    W = synth.weights(N, K, 0.02, M + N, 1)
+    P, G = bl.bitnet_pack_weights(_t(W, dev), EPS_W)
+    p_ref, g_ref = orc.pack_weights(W, EPS_W)
+    g = synth.gain(K, 1, 3, dt) if norm else None
+    gd = None if g is None else _x_dev(g, dt, dev)
+    out = {"bf16": torch.bfloat16, "f32": torch.float32, "i32": torch.int32}[yt]
+    xs = [synth.activations(M, K, M + K + i, 2, "normal", 0.01, 20.0, dt) for i in range(3)]
+    x_host = [_x_dev(x, dt, dev).cpu().pin_memory() for x in xs]
+    y_host = [torch.empty((M, N), dtype=out).pin_memory() for _ in xs]
+    x_dev = [torch.empty_like(h, device=dev) for h in x_host]
+    y_dev = [torch.empty((M, N), dtype=out, device=dev) for _ in xs]
+    s = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(s):
+        for i in range(len(xs)):
+            bl.bitnet_bitlinear_gemv_host(x_host[i], x_dev[i], P, G, y_dev[i], y_host[i], gd, EPS_RMS)
+    s.synchronize()
+    for i, x in enumerate(xs):
+        xq_r, a_r, _ = orc.quant_act(x, g, EPS_RMS)
+        acc_r, y_r = orc.bitlinear(p_ref, g_ref, K, xq_r, a_r)
+        assert torch.equal(y_host[i], y_dev[i].cpu())
+        if yt == "i32":
+            np.testing.assert_array_equal(y_host[i].numpy(), acc_r)
+        elif yt == "f32":
+            assert ulp_diff_f32(y_host[i].numpy(), y_r).max() == 0
+        else:
+            yb = y_host[i].view(torch.int16).numpy().view(np.uint16)
+            assert ulp_diff_bf16(yb, orc.f32_to_bf16(y_r)).max() == 0
+
+
 # --------------------------------------------------------------------------- whole workloads
 
 _PACKED = {}
