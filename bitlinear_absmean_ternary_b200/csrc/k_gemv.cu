@@ -231,11 +231,19 @@ cudaError_t launch_fused_c(const void* x, const void* gain, float eps, const uin
   // (fewer registers, so the next launch's CTA can share the SM)
   const int nthr = gain != nullptr ? kQuantThreads : kGemvThreads;
   const int per_thread = (K / 8 + nthr - 1) / nthr;
+  if constexpr (MT == 1) {
+    // one token, a row past the norm's register budget: the instantiation
+    // with the streamed normalisation alone (MAXC 0), so that no unused
+    // register-resident chunks weigh on the kernel's register allocation
+    constexpr int kResident = BN_QUANT_STREAM_BYTES / static_cast<int>(sizeof(Chunk8<T>));
+    if (gain != nullptr && per_thread > kResident)
+      return launch_fused_t<1, T, 0>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+  }
   if (per_thread <= 1) return launch_fused_t<MT, T, 1>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
   if (per_thread <= 2) return launch_fused_t<MT, T, 2>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
   if (per_thread <= 4) return launch_fused_t<MT, T, 4>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
   if (per_thread <= 8) return launch_fused_t<MT, T, 8>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
-  if constexpr (sizeof(T) == 2) return launch_fused_t<MT, T, 16>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
+  if constexpr (sizeof(T) == 2 && MT > 1) return launch_fused_t<MT, T, 16>(x, gain, eps, Wp, gamma, N, K, y, yd, s);
   return cudaErrorInvalidValue;
 }
 
@@ -292,11 +300,14 @@ cudaError_t bitnet_host::launch_ffn_upgate_gemv1(const __nv_bfloat16* x, const _
   const int nthr = gain != nullptr ? kQuantThreads : kGemvThreads;
   const int per_thread = (D / 8 + nthr - 1) / nthr;
   *used = true;
+  // a long normalised input row: the streamed normalisation alone (MAXC 0); without a norm
+  // D <= 21504 gives at most 6 chunks per thread
+  if (gain != nullptr && per_thread > BN_QUANT_STREAM_BYTES / static_cast<int>(sizeof(Chunk8<__nv_bfloat16>)))
+    return launch_upgate1_c<0>(p, x, gain, eps, Wu, gu, Wg, gg, F, D, h, s);
   if (per_thread <= 1) return launch_upgate1_c<1>(p, x, gain, eps, Wu, gu, Wg, gg, F, D, h, s);
   if (per_thread <= 2) return launch_upgate1_c<2>(p, x, gain, eps, Wu, gu, Wg, gg, F, D, h, s);
   if (per_thread <= 4) return launch_upgate1_c<4>(p, x, gain, eps, Wu, gu, Wg, gg, F, D, h, s);
-  if (per_thread <= 8) return launch_upgate1_c<8>(p, x, gain, eps, Wu, gu, Wg, gg, F, D, h, s);
-  return launch_upgate1_c<16>(p, x, gain, eps, Wu, gu, Wg, gg, F, D, h, s);
+  return launch_upgate1_c<8>(p, x, gain, eps, Wu, gu, Wg, gg, F, D, h, s);
 }
 
 BITNET_DEFINE_TAKE_ERROR(gemv)

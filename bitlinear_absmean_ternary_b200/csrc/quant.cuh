@@ -259,9 +259,17 @@ __device__ __noinline__ void quant_row_norm_stream(const T* __restrict__ row, in
 // comes after a barrier that all readers of its previous contents passed.
 // NT: the threads taking part are the NT threads from T0 on (T0 a multiple of
 // 32; synchronised by named barrier 1), or all of the CTA's when NT == 0.
+// MAXC == 0 instantiates the streamed RMSNorm path alone (gain required): a
+// kernel built for long normalised rows then carries no register-resident
+// chunk arrays, which otherwise shape the register allocation of the rest of
+// the kernel even where they are never used.
 template <typename T, int MAXC, bool COHERENT = false, int NT = 0, int T0 = 0>
 BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict__ gain, float rms_eps,
-                          int8_t* xq_row, QuantScratch& sc, float& amax_out, int& sum_out) {
+                          int8_t* xq_row, QuantScratch& sc, float& amax_out, int& sum_out);
+
+template <typename T, int MAXC, bool COHERENT, int NT, int T0>
+BN_DEV void quant_row_regs(const T* __restrict__ row, int K, const T* __restrict__ gain, float rms_eps,
+                           int8_t* xq_row, QuantScratch& sc, float& amax_out, int& sum_out) {
   static_assert(T0 % 32 == 0 && (T0 == 0 || NT != 0), "a thread offset needs a fixed thread count");
   if constexpr (sizeof(Chunk8<T>) * MAXC > BN_QUANT_STREAM_BYTES) {
     if (gain != nullptr) {
@@ -425,6 +433,17 @@ BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict_
   for (int o = 16; o >= 1; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
   amax_out = amax;
   sum_out = tot;
+}
+
+template <typename T, int MAXC, bool COHERENT, int NT, int T0>
+BN_DEV void quant_row_cta(const T* __restrict__ row, int K, const T* __restrict__ gain, float rms_eps,
+                          int8_t* xq_row, QuantScratch& sc, float& amax_out, int& sum_out) {
+  if constexpr (MAXC == 0) {
+    static_assert(T0 % 32 == 0 && (T0 == 0 || NT != 0), "a thread offset needs a fixed thread count");
+    quant_row_norm_stream<T, COHERENT, NT, T0>(row, K, gain, rms_eps, xq_row, sc, amax_out, sum_out);
+  } else {
+    quant_row_regs<T, MAXC, COHERENT, NT, T0>(row, K, gain, rms_eps, xq_row, sc, amax_out, sum_out);
+  }
 }
 
 // Standalone kernel: one CTA per token row.  256 threads with RMSNorm (the
