@@ -145,6 +145,10 @@ QUANT_CASES = [
     (200, 12288, "normal", 0.01, 20.0, "f32", True),     # more rows than SMs: 256 threads per row
     (300, 12288, "normal", 0.005, 30.0, "bf16", True),   # bf16, 6 chunks per lane
     (1, 21504, "normal", 0.005, 30.0, "bf16", True),     # one token, the 27B FFN's sub-norm input
+    # more than two long rows per SM: persistent CTAs stream the rows through shared memory
+    (297, 12352, "normal", 0.0, 1.0, "bf16", False),     # the first M and bf16 K that take it
+    (400, 8192, "normal", 0.01, 20.0, "f32", True),      # f32 rows with the gain (one CTA per SM)
+    (400, 16384, "normal", 0.0, 1.0, "f32", False),      # 64-KB f32 rows
 ]
 
 
@@ -185,7 +189,7 @@ def test_quant_edge_tokens(dev, orc):
 
 def test_quant_edge_tokens_many_rows(dev, orc):
     """The same edge rows among 640 bf16 tokens, where one warp quantises each
-    row (a CTA per row for K = 21504): zero, one-hot, exact ties after
+    row (rows streamed through shared memory for K = 21504): zero, one-hot, exact ties after
     scaling, huge, tiny and a row whose maximum sits in its last chunk (held
     by lane 31 for K = 2560 and 6144)."""
     import torch
@@ -208,7 +212,7 @@ def test_quant_edge_tokens_many_rows(dev, orc):
             np.testing.assert_array_equal(xq.cpu().numpy(), xq_r)
             np.testing.assert_array_equal(a.cpu().numpy(), a_r)
             np.testing.assert_array_equal(rs.cpu().numpy(), rs_r)
-        # the first 511 rows alone take the CTA-per-row kernel: same codes and scales
+        # the first 511 rows alone (below the warp-per-row threshold): same codes and scales
         xq5, a5, _ = bl.bitnet_quant_act(_x_dev(x[:511], "bf16", dev), _x_dev(g, "bf16", dev), EPS_RMS)
         assert torch.equal(xq5, xq[:511]) and torch.equal(a5, a[:511])
 
