@@ -46,28 +46,40 @@ cudaError_t launch_quant_rows(const void* x, int64_t M, int K, const void* gain,
   return cudaErrorInvalidValue;
 }
 
-template <typename T, bool NORM>
-cudaError_t launch_quant_stream_t(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
+template <typename T, bool NORM, int NTHR>
+cudaError_t launch_quant_stream_n(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
                                   int32_t* rs, cudaStream_t s) {
   static std::atomic<bool> done[kMaxDevices] = {};
   // the largest ring: three 64-KB rows (bf16 K = 32768 or f32 K = 16384 with the gain)
-  const cudaError_t e = set_smem(quant_stream_kernel<T, NORM>, 3 * 65536, done);
+  const cudaError_t e = set_smem(quant_stream_kernel<T, NORM, NTHR>, 3 * 65536, done);
   if (e != cudaSuccess) return e;
   const int smem = quant_stream_smem_bytes<T, NORM>(K);
-  const int per_sm = 2 * (smem + 4096) <= 232448 ? 2 : 1;  // two CTAs when two rings fit
+  const int fit = 232448 / (smem + 4096);  // rings per SM by shared memory
+  const int most = NTHR == 256 ? 4 : 2;    // and by threads and registers
+  const int per_sm = fit > most ? most : (fit < 1 ? 1 : fit);
   const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
   const int64_t grid = M < cap ? M : cap;
-  return launch_pdl(quant_stream_kernel<T, NORM>, dim3(static_cast<unsigned>(grid)), dim3(kQsThreads),
+  return launch_pdl(quant_stream_kernel<T, NORM, NTHR>, dim3(static_cast<unsigned>(grid)), dim3(NTHR),
                     static_cast<size_t>(smem), s, static_cast<const T*>(x), static_cast<int>(M), K,
                     static_cast<const T*>(gain), eps, xq, a, rs);
 }
 
-// Rows of more than this many bytes, more than two per SM: the persistent
-// kernel that streams rows through shared memory (quant_stream.cuh).  Shorter
-// rows keep the CTA-per-row kernel: with one row in flight per CTA the
-// streaming kernel's per-row reductions dominate (measured: K = 6912 bf16 at
-// 0.46 of HBM against 0.62; K = 21504 at 0.77 against 0.64).
-constexpr int kQuantStreamMinRowBytes = 24576;
+// Rows of at least this many bytes, more than two per SM: the persistent
+// kernel that streams rows through shared memory (quant_stream.cuh), with
+// 256 threads per CTA up to kQuantStreamWideRowBytes and 512 beyond.  Shorter
+// rows keep the CTA-per-row kernel (measured, bf16 rows, back to back:
+// K = 6912 0.65 of HBM either way; K = 12288 0.86 streamed against 0.72;
+// K = 21504 0.79 against 0.65).
+constexpr int kQuantStreamMinRowBytes = 16384;
+constexpr int kQuantStreamWideRowBytes = 24576;
+
+template <typename T, bool NORM>
+cudaError_t launch_quant_stream_t(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
+                                  int32_t* rs, cudaStream_t s) {
+  if (K * static_cast<int>(sizeof(T)) <= kQuantStreamWideRowBytes)
+    return launch_quant_stream_n<T, NORM, 256>(x, M, K, gain, eps, xq, a, rs, s);
+  return launch_quant_stream_n<T, NORM, 512>(x, M, K, gain, eps, xq, a, rs, s);
+}
 
 // Token count from which the warp-per-row kernel takes over (bf16 input,
 // K <= 6144): from there on it keeps more rows in flight per SM; below, a CTA
@@ -77,7 +89,7 @@ constexpr int64_t kQuantRowsMinM = 512;
 template <typename T>
 cudaError_t launch_quant(const void* x, int64_t M, int K, const void* gain, float eps, int8_t* xq, float* a,
                          int32_t* rs, cudaStream_t s) {
-  if (K * static_cast<int>(sizeof(T)) > kQuantStreamMinRowBytes && M > 2 * static_cast<int64_t>(sm_count()))
+  if (K * static_cast<int>(sizeof(T)) >= kQuantStreamMinRowBytes && M > 2 * static_cast<int64_t>(sm_count()))
     return gain != nullptr ? launch_quant_stream_t<T, true>(x, M, K, gain, eps, xq, a, rs, s)
                            : launch_quant_stream_t<T, false>(x, M, K, gain, eps, xq, a, rs, s);
   if constexpr (sizeof(T) == 2) {

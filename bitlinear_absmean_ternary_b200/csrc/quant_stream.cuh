@@ -20,9 +20,6 @@
 
 namespace bitnet {
 
-constexpr int kQsThreads = 512;
-constexpr int kQsWarps = kQsThreads / 32;
-
 template <typename T>
 BN_DEV Chunk8<T> qs_chunk(uint32_t addr) {
   Chunk8<T> c;
@@ -37,12 +34,15 @@ BN_DEV Chunk8<T> qs_chunk(uint32_t addr) {
 }
 
 // One row from shared memory (row at shared address `rs`, the gain at `gs`
-// when NORM): writes x_q to xq_row (global), returns max|h| and sum(x_q) to
-// every thread.  Ends with a CTA barrier after the last read of the row.
-template <typename T, bool NORM>
+// when NORM) by the NTHR threads of the CTA: writes x_q to xq_row (global),
+// returns max|h| and sum(x_q) to every thread.  Ends with a CTA barrier after
+// the last read of the row.
+template <typename T, bool NORM, int NTHR>
 BN_DEV void qs_row(uint32_t rs, uint32_t gs, int K, float rms_eps, int8_t* __restrict__ xq_row, QuantScratch& sc,
                    float& amax_out, int& sum_out) {
+  static_assert(NTHR >= kQuantThreads && NTHR % 32 == 0, "the fixed-order sum needs 256 threads");
   constexpr uint32_t CB = sizeof(Chunk8<T>);  // bytes per 8-element chunk
+  constexpr int kWarps = NTHR / 32;
   const int t = static_cast<int>(threadIdx.x), lane = t & 31, warp = t >> 5;
   const int nchunks = K >> 3;
 
@@ -78,7 +78,7 @@ BN_DEV void qs_row(uint32_t rs, uint32_t gs, int K, float rms_eps, int8_t* __res
 
   // max|h| (order-free): h = RN32(RN32(v * r) * g) with the norm, else v
   float amax = 0.0f;
-  for (int c = t; c < nchunks; c += kQsThreads) {
+  for (int c = t; c < nchunks; c += NTHR) {
     const Chunk8<T> ch = qs_chunk<T>(rs + CB * c);
     if constexpr (NORM) {
       const Chunk8<T> g = qs_chunk<T>(gs + CB * c);
@@ -99,13 +99,13 @@ BN_DEV void qs_row(uint32_t rs, uint32_t gs, int K, float rms_eps, int8_t* __res
   for (int s = 16; s >= 1; s >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, s));
   if (lane == 0) sc.amx[warp] = amax;
   __syncthreads();
-  amax = lane < kQsWarps ? sc.amx[lane] : 0.0f;
+  amax = lane < kWarps ? sc.amx[lane] : 0.0f;
 #pragma unroll
   for (int s = 16; s >= 1; s >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, s));
 
   int sum = 0;
   const float s = amax == 0.0f ? 0.0f : __fdiv_rn(127.0f, amax);
-  for (int c = t; c < nchunks; c += kQsThreads) {
+  for (int c = t; c < nchunks; c += NTHR) {
     uint32_t lo = 0, hi = 0;
     if (amax != 0.0f) {
       const Chunk8<T> ch = qs_chunk<T>(rs + CB * c);
@@ -129,7 +129,7 @@ BN_DEV void qs_row(uint32_t rs, uint32_t gs, int K, float rms_eps, int8_t* __res
   for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   if (lane == 0) sc.ired[warp] = sum;
   __syncthreads();
-  int tot = lane < kQsWarps ? sc.ired[lane] : 0;
+  int tot = lane < kWarps ? sc.ired[lane] : 0;
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
   amax_out = amax;
@@ -143,10 +143,12 @@ __host__ __device__ constexpr int quant_stream_smem_bytes(int K) {
 }
 
 // Rows m = blockIdx.x, + gridDim.x, ... of x (M x K), through a ring of two
-// shared-memory row buffers.  Every wait is bounded; after a timeout (the
-// device error word is set) the CTA lets its copies in flight land and exits.
-template <typename T, bool NORM>
-__global__ void __launch_bounds__(kQsThreads, 2)
+// shared-memory row buffers, NTHR threads per CTA (256 for rows of at most
+// 24 KB, four CTAs per SM; 512 for longer rows).  Every wait is bounded; after
+// a timeout (the device error word is set) the CTA lets its copies in flight
+// land and exits.
+template <typename T, bool NORM, int NTHR>
+__global__ void __launch_bounds__(NTHR, NTHR == 256 ? 4 : 2)
     quant_stream_kernel(const T* __restrict__ x, int M, int K, const T* __restrict__ gain, float rms_eps,
                         int8_t* __restrict__ xq, float* __restrict__ a_out, int32_t* __restrict__ rowsum_out) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -182,7 +184,7 @@ __global__ void __launch_bounds__(kQsThreads, 2)
     if (!__syncthreads_and(mbar_wait(&full[b], static_cast<uint32_t>(it >> 1) & 1u))) break;
     float amax;
     int sum;
-    qs_row<T, NORM>(base + b * rb, base + 2 * rb, K, rms_eps, xq + m * K, sc, amax, sum);
+    qs_row<T, NORM, NTHR>(base + b * rb, base + 2 * rb, K, rms_eps, xq + m * K, sc, amax, sum);
     if (threadIdx.x == 0) {
       a_out[m] = amax == 0.0f ? 0.0f : __fdiv_rn(amax, 127.0f);
       if (rowsum_out != nullptr) rowsum_out[m] = sum;

@@ -146,7 +146,9 @@ QUANT_CASES = [
     (300, 12288, "normal", 0.005, 30.0, "bf16", True),   # bf16, 6 chunks per lane
     (1, 21504, "normal", 0.005, 30.0, "bf16", True),     # one token, the 27B FFN's sub-norm input
     # more than two long rows per SM: persistent CTAs stream the rows through shared memory
-    (297, 12352, "normal", 0.0, 1.0, "bf16", False),     # the first M and bf16 K that take it
+    (297, 8192, "normal", 0.0, 1.0, "bf16", False),      # the first M and bf16 K that take it (256 threads)
+    (350, 4096, "normal", 0.01, 20.0, "f32", False),     # the first f32 K that takes it
+    (297, 12352, "normal", 0.0, 1.0, "bf16", False),     # the first bf16 K past 24 KB rows (512 threads)
     (400, 8192, "normal", 0.01, 20.0, "f32", True),      # f32 rows with the gain (one CTA per SM)
     (400, 16384, "normal", 0.0, 1.0, "f32", False),      # 64-KB f32 rows
 ]
