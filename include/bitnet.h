@@ -24,9 +24,10 @@
  *   - Every pointer must be 16-byte aligned.
  *   - Errors are returned as bitnet_status; nothing is launched when an
  *     argument is rejected.  No C++ exception crosses this boundary.
- *   - The product entry points (bitnet_linear_gemv, bitnet_linear_gemm,
- *     bitnet_linear_upgate_gemm, bitnet_bitlinear_gemv, bitnet_bitlinear_gemm,
- *     bitnet_bitlinear_ffn_gemv, bitnet_bitlinear_gemv_b3) are launched with programmatic dependent
+ *   - The product entry points (bitnet_linear_gemv, bitnet_linear_gemm and
+ *     its _stream_k form, bitnet_linear_upgate_gemm, bitnet_bitlinear_gemv,
+ *     bitnet_bitlinear_gemm and its _stream_k form, bitnet_bitlinear_ffn_gemv,
+ *     bitnet_bitlinear_gemv_b3) are launched with programmatic dependent
  *     launch: they start while the previous kernel on the stream finishes,
  *     and request their first packed-weight tiles BEFORE waiting for it
  *     (the weights of a layer never depend on the layer before).  So the
